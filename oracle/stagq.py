@@ -1,0 +1,453 @@
+"""CPU oracle for the StagQ multi-precision GEMV -- TEST INFRASTRUCTURE ONLY.
+
+This module is the plain, slow, fp64 statement of what the StagQ format
+computes, written from the StagQ paper ("StagQ: Constraint-Driven
+Multi-Precision Weight Quantization for LLMs", arXiv 2610.05977). Only the
+test-suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import it; the product (the CUDA library and its Python
+binding) never does, and it shares no code with them.
+
+It covers three things:
+
+* the encoder of Sections 3.1-3.6 (+ Appendices B and E) for synthetic
+  weights: side record, clipping, initial pair, uniform codebooks, per-group
+  pair choice by Eq. (5)-(6), nearest-rounding base, sign planes (Eq. (7));
+* the decoder: composite integer Eq. (8), affine map Eq. (10) (with the
+  additive form Eq. (9) kept as a cross-check), complete reconstruction
+  Eq. (4);
+* the GEMV ``y = W_hat x`` as an fp64 dot product.
+
+Every place where the paper is silent and a reading had to be taken is
+marked "Reading:" below. Parity status of each function: all functions are
+pinned by the ``-m "not gpu"`` tests (Figure 1 worked example, closed forms,
+invariants, brute force); the Eq. (5) pair search is pinned only by brute
+force on tiny groups, because the paper prints no fitted pair values.
+
+Array conventions: ``W`` is [out, inp] (row = output channel, K = inp),
+groups are runs of ``group`` consecutive entries along K inside one row.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+# Appendix B: the initial pair places four levels symmetrically, the outer
+# two 6 % in from each end of the group range.
+INIT_EDGE_FRACTION = 0.06
+# Section 3.1: weight of the floor term in Eq. (5).
+FLOOR_LAMBDA = 4.0
+# Section 3.1: two sixteen-entry codebooks per matrix.
+CODEBOOK_SIZE = 16
+# Reading: a group whose clipped range is zero gets this step so that
+# log2(s0) stays finite (fp16's smallest positive value).
+DEGENERATE_STEP = 2.0 ** -24
+
+
+@dataclass
+class Fields:
+    """Logical fields of one encoded matrix (no physical layout)."""
+
+    out: int
+    inp: int
+    group: int
+    n_planes: int               # refinement planes stored: b_3 .. b_{2+n_planes}
+    q: np.ndarray               # uint8 [out, inp], base digit 0..3
+    planes: np.ndarray          # uint8 [n_planes, out, inp], b_k in {0, 1}
+    pair_idx: np.ndarray        # uint8 [out, inp // group]; hi nibble = log2(s) index
+    cb_log2s: np.ndarray        # float16 [16]
+    cb_lo_over_s: np.ndarray    # float16 [16]
+    row_ptr: np.ndarray         # int64 [out + 1]  (side record, CSR)
+    col: np.ndarray             # int64 [nnz], sorted inside each row
+    val: np.ndarray             # float16 [nnz], the recorded value P
+
+    @property
+    def depth(self) -> int:
+        """Stream depth N of Section 3: base + planes, i.e. the top precision."""
+        return 2 + self.n_planes
+
+    @property
+    def nnz(self) -> int:
+        return int(self.col.shape[0])
+
+
+# --------------------------------------------------------------------------
+# Grid algebra (Sections 3.2-3.4)
+# --------------------------------------------------------------------------
+
+def half_step(s, k: int):
+    """Eq. (7): refinement half-step t_k = alpha_k = s / 2^(k-1), k >= 3."""
+    return s / 2.0 ** (k - 1)
+
+
+def grid_at(lo, s, M: int):
+    """Eq. (10): origin lo_M and spacing s_M of the precision-M grid.
+
+    s_M = s / 2^(M-2) and lo_M = lo - s (2^(M-2) - 1) / 2^(M-1).
+    """
+    s_M = s / 2.0 ** (M - 2)
+    lo_M = lo - s * (2.0 ** (M - 2) - 1.0) / 2.0 ** (M - 1)
+    return lo_M, s_M
+
+
+def reach(s, N: int):
+    """Eq. (6): rho = s * sum_{k=3}^{N} 2^-(k-1), the furthest the planes move
+    the base reconstruction."""
+    return s * sum(2.0 ** -(k - 1) for k in range(3, N + 1))
+
+
+def composite_level(q, planes, M: int):
+    """Eq. (8): u_M = q 2^(M-2) + sum_{k=3}^{M} b_k 2^(M-k).
+
+    ``planes`` is a sequence whose entry k-3 holds b_k; only b_3..b_M are read.
+    """
+    u = np.asarray(q, dtype=np.int64) * (1 << (M - 2))
+    for k in range(3, M + 1):
+        u = u + np.asarray(planes[k - 3], dtype=np.int64) * (1 << (M - k))
+    return u
+
+
+def reconstruct_additive(lo, s, q, planes, M: int):
+    """Eq. (9): lo + s q + sum_{k=3}^{M} (2 b_k - 1) s / 2^(k-1).
+
+    Kept as an independent statement of the main stream; Eq. (10) is what the
+    decoder uses, and the tests check that the two agree.
+    """
+    w = lo + s * np.asarray(q, dtype=np.float64)
+    for k in range(3, M + 1):
+        b = np.asarray(planes[k - 3], dtype=np.float64)
+        w = w + (2.0 * b - 1.0) * half_step(s, k)
+    return w
+
+
+def reconstruct_affine(lo, s, u, M: int):
+    """Eq. (10): W_main^(M) = lo_M + s_M u_M."""
+    lo_M, s_M = grid_at(lo, s, M)
+    return lo_M + s_M * np.asarray(u, dtype=np.float64)
+
+
+# --------------------------------------------------------------------------
+# Digit encoding of one value under a fixed pair (Sections 3.3 and 3.6)
+# --------------------------------------------------------------------------
+
+def base_digit(w, lo, s):
+    """Appendix E: the base code is nearest rounding onto the four levels
+    lo + s q, q in {0..3}.
+
+    Reading: round half up, q = clamp(floor((w - lo)/s + 1/2), 0, 3).
+    """
+    q = np.floor((np.asarray(w, dtype=np.float64) - lo) / s + 0.5)
+    return np.clip(q, 0, 3).astype(np.int64)
+
+
+def encode_digits(w, lo, s, N: int):
+    """Base digit, then each refinement plane k = 3..N stores the sign of the
+    residual left by the preceding prefix (Section 3.6), with sign(0) := +1
+    (Section 3.3); plane k moves the reconstruction by +-t_k (Eq. (7)).
+
+    Returns (q, [b_3..b_N], [W^(2)..W^(N)]) with the reconstructions computed
+    step by step as the encoder walks the prefix.
+    """
+    w = np.asarray(w, dtype=np.float64)
+    q = base_digit(w, lo, s)
+    recon = lo + s * q.astype(np.float64)
+    recons = [recon]
+    bits = []
+    for k in range(3, N + 1):
+        r = w - recon
+        b = (r >= 0.0).astype(np.int64)
+        recon = recon + (2.0 * b - 1.0) * half_step(s, k)
+        bits.append(b)
+        recons.append(recon)
+    return q, bits, recons
+
+
+# --------------------------------------------------------------------------
+# Encoder stages (Sections 3.1, 3.5, 3.6; Appendices B and E)
+# --------------------------------------------------------------------------
+
+def side_record_count(out: int, inp: int, density: float) -> int:
+    """Reading: the record holds round(density * out * inp) entries (half up)."""
+    return int(np.floor(density * out * inp + 0.5))
+
+
+def select_side_record(W: np.ndarray, density: float) -> np.ndarray:
+    """Pre-grid hold-out for the synthetic workloads: the largest-|w| entries.
+
+    Reading: the workloads name a global top-|w| density in place of the
+    paper's per-group ratio / gain criteria (Section 3.5); ties in |w| go to
+    the smaller flat row-major index. Returns a bool mask [out, inp].
+    """
+    out, inp = W.shape
+    k = side_record_count(out, inp, density)
+    mask = np.zeros(out * inp, dtype=bool)
+    if k == 0:
+        return mask.reshape(out, inp)
+    a = np.abs(W.astype(np.float64)).reshape(-1)
+    if k >= a.size:
+        mask[:] = True
+        return mask.reshape(out, inp)
+    # threshold = k-th largest |w|; everything above it is in, ties at it are
+    # filled in increasing flat index.
+    thr = np.partition(a, a.size - k)[a.size - k]
+    above = np.flatnonzero(a > thr)
+    tied = np.flatnonzero(a == thr)
+    mask[above] = True
+    mask[tied[: k - above.size]] = True
+    return mask.reshape(out, inp)
+
+
+def clip_held_out(W: np.ndarray, mask: np.ndarray, group: int):
+    """Section 3.1: in the pair fit, every held-out entry is clipped to the next
+    value inward.
+
+    Reading: the next value inward is the group's largest retained value for a
+    held-out entry >= 0 and its smallest retained value for one < 0 (a held-out
+    entry is never inside the retained range, since the record takes the
+    largest |w|). Returns (clipped values [out, inp] fp64, bool [out, ngroups]
+    marking groups with no retained entry).
+    """
+    out, inp = W.shape
+    ng = inp // group
+    V = W.astype(np.float64).reshape(out, ng, group)
+    M = mask.reshape(out, ng, group)
+    mx = np.where(M, -np.inf, V).max(axis=2)
+    mn = np.where(M, np.inf, V).min(axis=2)
+    empty = ~np.any(~M, axis=2)
+    repl = np.where(V >= 0.0, mx[:, :, None], mn[:, :, None])
+    Vc = np.where(M, repl, V)
+    Vc = np.where(empty[:, :, None], 0.0, Vc)
+    return Vc.reshape(out, inp), empty
+
+
+def initial_pairs(Vc: np.ndarray, group: int):
+    """Appendix B: the initial pair puts four levels symmetrically, the outer
+    two 6 % in from the group's ends (a step of 0.29 of the range).
+
+    lo0 = min + 0.06 R, top = max - 0.06 R, s0 = (top - lo0) / 3, R = max - min.
+    Reading: a group of zero range gets s0 = 2^-24. Returns (lo0, s0), each
+    [out, ngroups] fp64.
+    """
+    out, inp = Vc.shape
+    G = Vc.reshape(out, inp // group, group)
+    mn = G.min(axis=2)
+    mx = G.max(axis=2)
+    R = mx - mn
+    lo0 = mn + INIT_EDGE_FRACTION * R
+    top = mx - INIT_EDGE_FRACTION * R
+    s0 = (top - lo0) / 3.0
+    s0 = np.where(R > 0.0, s0, DEGENERATE_STEP)
+    return lo0, s0
+
+
+def uniform_codebook(values: np.ndarray) -> np.ndarray:
+    """Appendix E, uniform placement: sixteen evenly spaced points over the
+    range of the initial pairs, stored as fp16 (Section 3.1 / Appendix E).
+
+    c_i = vmin + i (vmax - vmin) / 15, rounded to fp16 (nearest even).
+    Reading: with no values at all the codebook is all zeros.
+    """
+    if values.size == 0:
+        return np.zeros(CODEBOOK_SIZE, dtype=np.float16)
+    vmin = float(values.min())
+    vmax = float(values.max())
+    cb = [vmin + i * (vmax - vmin) / (CODEBOOK_SIZE - 1) for i in range(CODEBOOK_SIZE)]
+    return np.array(cb, dtype=np.float64).astype(np.float16)
+
+
+def fit_codebooks(lo0: np.ndarray, s0: np.ndarray, empty: np.ndarray):
+    """Section 3.1: one codebook in log2(s) and one in lo/s per matrix, fitted
+    to the initial pairs of the groups that keep at least one entry."""
+    keep = ~empty
+    cb_log2s = uniform_codebook(np.log2(s0[keep]))
+    cb_lo_over_s = uniform_codebook(lo0[keep] / s0[keep])
+    return cb_log2s, cb_lo_over_s
+
+
+def pair_table(cb_log2s: np.ndarray, cb_lo_over_s: np.ndarray):
+    """The 256 (lo, s) combinations of Section 3.1, indexed a*16 + b with
+    a = log2(s) index (high nibble) and b = lo/s index (low nibble).
+
+    s = 2^(cb_log2s[a]), lo = cb_lo_over_s[b] * s, in fp64 from the fp16
+    codebook values. Reading: nibble order high = log2(s).
+    """
+    a = np.repeat(np.arange(CODEBOOK_SIZE), CODEBOOK_SIZE)
+    b = np.tile(np.arange(CODEBOOK_SIZE), CODEBOOK_SIZE)
+    s = np.exp2(cb_log2s.astype(np.float64)[a])
+    lo = cb_lo_over_s.astype(np.float64)[b] * s
+    return lo, s
+
+
+def pair_cost(V: np.ndarray, lo, s, N: int):
+    """Eq. (5) with E_c = 1 (x ~ N(0,1) gives unit channel mean squares):
+
+    D = 1/(N-1) sum_{M=2}^{N} sum_c (V_c - W_c^(M))^2
+        + lambda sum_c max(|V_c - W_c^(2)| - rho, 0)^2          (Eq. (6))
+
+    with W^(M) the digit encoding of ``encode_digits`` under (lo, s) and rho
+    from ``reach``. ``V`` is [..., g] (the clipped group), lo and s broadcast
+    against V[..., 0]. Returns D with V's leading shape.
+    """
+    lo = np.asarray(lo, dtype=np.float64)[..., None]
+    s = np.asarray(s, dtype=np.float64)[..., None]
+    _, _, recons = encode_digits(V, lo, s, N)
+    first = 0.0
+    for rec in recons:                       # M = 2 .. N
+        first = first + np.sum((V - rec) ** 2, axis=-1)
+    first = first / (N - 1)
+    rho = reach(s, N)
+    floor = np.sum(np.maximum(np.abs(V - recons[0]) - rho, 0.0) ** 2, axis=-1)
+    return first + FLOOR_LAMBDA * floor
+
+
+def choose_pairs(Vc: np.ndarray, group: int, N: int, lo_tab, s_tab, empty,
+                 mode: str = "search", lo0=None, s0=None, cb_log2s=None,
+                 cb_lo_over_s=None, chunk: int = 256) -> np.ndarray:
+    """Per-group pair choice.
+
+    mode "search" (Section 3.1): the combination minimising Eq. (5) over all
+    256; Reading: ties go to the smallest index a*16+b.
+    mode "fast" (a labelled shortcut for very large stacks, not the paper's
+    rule): the nearest codebook entry to log2(s0) and to lo0/s0 separately,
+    ties to the smaller index.
+    Groups with no retained entry get pair 0 (their digits are all zero).
+    """
+    out, inp = Vc.shape
+    ng = inp // group
+    if mode == "fast":
+        ls = np.log2(s0)
+        r = lo0 / s0
+        da = np.abs(cb_log2s.astype(np.float64)[None, None, :] - ls[:, :, None])
+        db = np.abs(cb_lo_over_s.astype(np.float64)[None, None, :] - r[:, :, None])
+        a = np.argmin(da, axis=2)
+        b = np.argmin(db, axis=2)
+        idx = (a * CODEBOOK_SIZE + b).astype(np.uint8)
+    elif mode == "search":
+        G = Vc.reshape(out * ng, group)
+        idx = np.empty(out * ng, dtype=np.uint8)
+        for s0_ in range(0, G.shape[0], chunk):
+            Vg = G[s0_:s0_ + chunk][:, None, :]                 # [c, 1, g]
+            D = pair_cost(Vg, lo_tab[None, :], s_tab[None, :], N)   # [c, 256]
+            idx[s0_:s0_ + chunk] = np.argmin(D, axis=1).astype(np.uint8)
+        idx = idx.reshape(out, ng)
+    else:
+        raise ValueError(f"unknown pair mode {mode!r}")
+    return np.where(empty, 0, idx).astype(np.uint8)
+
+
+def encode(W: np.ndarray, group: int = 128, n_planes: int = 2,
+           density: float = 0.005, mode: str = "search") -> Fields:
+    """Figure 3's encoder for synthetic weights (no AWQ scale: with x ~ N(0,1)
+    every channel scale is equal; no post-grid guard):
+
+    1. side record: top-|w| entries (``select_side_record``), P = fp16 value;
+    2. clip held-out entries inward for the fit (``clip_held_out``);
+    3. initial pairs (Appendix B), 4. uniform codebooks (Appendix E),
+    5. pair per group (Eq. (5) search, or the labelled fast rule),
+    6. base by nearest rounding, 7. sign planes k = 3..N; held-out positions
+       store zero digits (Reading: the planes skip them, Section 3.6, and the
+       paper gives no stored value -- zeros make the main stream decode to
+       lo_M there, which Eq. (4) then masks).
+    """
+    W = np.asarray(W)
+    if W.dtype != np.float16:
+        raise TypeError("W must be fp16")
+    out, inp = W.shape
+    if group <= 0 or inp % group:
+        raise ValueError("group must divide the input dimension")
+    N = 2 + n_planes
+    ng = inp // group
+
+    mask = select_side_record(W, density)
+    Vc, empty = clip_held_out(W, mask, group)
+    lo0, s0 = initial_pairs(Vc, group)
+    cb_log2s, cb_lo_over_s = fit_codebooks(lo0, s0, empty)
+    lo_tab, s_tab = pair_table(cb_log2s, cb_lo_over_s)
+    pair_idx = choose_pairs(Vc, group, N, lo_tab, s_tab, empty, mode=mode,
+                            lo0=lo0, s0=s0, cb_log2s=cb_log2s,
+                            cb_lo_over_s=cb_lo_over_s)
+
+    lo_g = lo_tab[pair_idx.astype(np.int64)]             # [out, ng]
+    s_g = s_tab[pair_idx.astype(np.int64)]
+    lo_w = np.repeat(lo_g, group, axis=1)
+    s_w = np.repeat(s_g, group, axis=1)
+    q, bits, _ = encode_digits(W.astype(np.float64), lo_w, s_w, N)
+    q = np.where(mask, 0, q).astype(np.uint8)
+    planes = np.zeros((n_planes, out, inp), dtype=np.uint8)
+    for k in range(n_planes):
+        planes[k] = np.where(mask, 0, bits[k]).astype(np.uint8)
+
+    rows, cols = np.nonzero(mask)                         # row-major order
+    row_ptr = np.zeros(out + 1, dtype=np.int64)
+    np.add.at(row_ptr, rows + 1, 1)
+    row_ptr = np.cumsum(row_ptr)
+    val = W[rows, cols].astype(np.float16)
+    return Fields(out=out, inp=inp, group=group, n_planes=n_planes, q=q,
+                  planes=planes, pair_idx=pair_idx.astype(np.uint8),
+                  cb_log2s=cb_log2s, cb_lo_over_s=cb_lo_over_s,
+                  row_ptr=row_ptr, col=cols.astype(np.int64), val=val)
+
+
+# --------------------------------------------------------------------------
+# Decoder and GEMV (Eq. (4), (8), (10))
+# --------------------------------------------------------------------------
+
+def held_out_mask(F: Fields, rows=None) -> np.ndarray:
+    """The mask m of Eq. (4), rebuilt from the CSR side record."""
+    rows = np.arange(F.out) if rows is None else np.asarray(rows)
+    m = np.zeros((rows.size, F.inp), dtype=bool)
+    for i, r in enumerate(rows):
+        m[i, F.col[F.row_ptr[r]:F.row_ptr[r + 1]]] = True
+    return m
+
+
+def check_precision(F: Fields, M: int) -> None:
+    """A p_M read needs the base plus planes 3..M of the stored stream."""
+    if not (2 <= M <= F.depth):
+        raise ValueError(f"precision {M} outside 2..{F.depth}")
+
+
+def decode_levels(F: Fields, M: int, rows=None) -> np.ndarray:
+    """Eq. (8) per weight: the integer u_M read from the first M-2 planes."""
+    check_precision(F, M)
+    sl = slice(None) if rows is None else np.asarray(rows)
+    return composite_level(F.q[sl], [F.planes[k][sl] for k in range(F.n_planes)], M)
+
+
+def group_pairs(F: Fields, rows=None):
+    """fp64 (lo, s) of every group, from the 8-bit pair index and codebooks."""
+    lo_tab, s_tab = pair_table(F.cb_log2s, F.cb_lo_over_s)
+    idx = F.pair_idx if rows is None else F.pair_idx[np.asarray(rows)]
+    return lo_tab[idx.astype(np.int64)], s_tab[idx.astype(np.int64)]
+
+
+def decode(F: Fields, M: int, rows=None) -> np.ndarray:
+    """Eq. (4): W_hat^(M) = (1 - m) * (lo_M + s_M u_M) + P, fp64 [rows, inp]."""
+    u = decode_levels(F, M, rows)
+    lo_g, s_g = group_pairs(F, rows)
+    lo_w = np.repeat(lo_g, F.group, axis=1)
+    s_w = np.repeat(s_g, F.group, axis=1)
+    main = reconstruct_affine(lo_w, s_w, u, M)
+    rows_ = np.arange(F.out) if rows is None else np.asarray(rows)
+    m = held_out_mask(F, rows_)
+    P = np.zeros_like(main)
+    for i, r in enumerate(rows_):
+        sl = slice(F.row_ptr[r], F.row_ptr[r + 1])
+        P[i, F.col[sl]] = F.val[sl].astype(np.float64)
+    return np.where(m, 0.0, main) + P
+
+
+def gemv(F: Fields, M: int, x: np.ndarray, rows=None) -> np.ndarray:
+    """y = W_hat^(M) x in fp64 for x [n, inp] (fp16 values taken exactly);
+    returns [n, len(rows)] (all rows by default)."""
+    x = np.atleast_2d(np.asarray(x)).astype(np.float64)
+    What = decode(F, M, rows)
+    return x @ What.T
+
+
+def model_bytes(out: int, inp: int, group: int, nnz: int, M: int, n: int = 1) -> int:
+    """Bytes a p_M GEMV must move: the base and M-2 planes (M bits per weight),
+    one pair byte per group, the CSR record (4 B per entry + 4 B per row
+    pointer), x and y in fp16."""
+    return (out * inp * M) // 8 + (out * inp) // group + 4 * nnz + 4 * (out + 1) \
+        + 2 * n * inp + 2 * n * out

@@ -1,0 +1,64 @@
+"""Planted mistakes in the oracle (CPU only): each plausible slip -- a dropped
+term, a wrong sign, a wrong exponent, swapped nibbles -- must make at least
+one pin in test_oracle_pins fail."""
+import numpy as np
+import pytest
+
+from oracle import stagq as O
+import tests.test_oracle_pins as P
+
+
+def _fails(fn, *args):
+    try:
+        fn(*args)
+    except AssertionError:
+        return True
+    return False
+
+
+def _grid_wrong_sign(lo, s, M):
+    s_M = s / 2.0 ** (M - 2)
+    return lo + s * (2.0 ** (M - 2) - 1.0) / 2.0 ** (M - 1), s_M
+
+
+def _grid_wrong_spacing(lo, s, M):
+    s_M = s / 2.0 ** (M - 1)
+    return lo - s * (2.0 ** (M - 2) - 1.0) / 2.0 ** (M - 1), s_M
+
+
+def _half_step_wrong(s, k):
+    return s / 2.0 ** (k - 2)
+
+
+def _composite_dropped_plane(q, planes, M):
+    u = np.asarray(q, dtype=np.int64) * (1 << (M - 2))
+    for k in range(3, M):          # b_M dropped
+        u = u + np.asarray(planes[k - 3], dtype=np.int64) * (1 << (M - k))
+    return u
+
+
+def _pair_table_swapped(cb_log2s, cb_lo_over_s):
+    a = np.tile(np.arange(16), 16)             # nibbles swapped
+    b = np.repeat(np.arange(16), 16)
+    s = np.exp2(cb_log2s.astype(np.float64)[a])
+    return cb_lo_over_s.astype(np.float64)[b] * s, s
+
+
+def _base_digit_truncating(w, lo, s):
+    return np.clip(np.floor((np.asarray(w, dtype=np.float64) - lo) / s), 0, 3).astype(np.int64)
+
+
+@pytest.mark.parametrize("name,mutant,pins", [
+    ("grid_at", _grid_wrong_sign, ["test_eq9_equals_eq10_all_digit_patterns", "test_figure1_every_prefix_is_a_grid_point"]),
+    ("grid_at", _grid_wrong_spacing, ["test_every_precision_is_a_uniform_grid", "test_midpoint_split_is_the_mmse_split"]),
+    ("half_step", _half_step_wrong, ["test_figure1_worked_example", "test_sign_planes_equal_nearest_level_rounding"]),
+    ("composite_level", _composite_dropped_plane, ["test_eq9_equals_eq10_all_digit_patterns"]),
+    ("pair_table", _pair_table_swapped, ["test_gemv_against_scalar_brute_force"]),
+    ("base_digit", _base_digit_truncating, ["test_sign_planes_equal_nearest_level_rounding"]),
+])
+def test_planted_mistake_is_caught(monkeypatch, name, mutant, pins):
+    monkeypatch.setattr(O, name, mutant)
+    for pin in pins:
+        fn = getattr(P, pin)
+        args = (2,) if pin == "test_gemv_against_scalar_brute_force" else ()
+        assert _fails(fn, *args), f"{pin} did not catch the mutant of {name}"
