@@ -1,0 +1,220 @@
+/*
+ * stagq.h -- C ABI of the StagQ multi-precision GEMV library (libstagq.so).
+ *
+ * The operation (StagQ paper, "StagQ: Constraint-Driven Multi-Precision Weight
+ * Quantization for LLMs", arXiv 2610.05977):
+ *
+ *   y = W_hat^(M) x,   W_hat^(M) = (1 - m) .* (lo_M + s_M u_M) + P          (Eq. 4, 10)
+ *
+ * u_M is the composite integer of the first M-2 refinement planes on top of
+ * the 2-bit base (Eq. 8); (lo_M, s_M) follow in closed form from one 8-bit
+ * (lo, s) pair per group (Section 3.1, Eq. 10); m / P is the sparse side
+ * record of held-out weights (Eq. 4). The read precision M ("bits") is
+ * chosen per call, from 2 up to 2 + n_planes, from ONE stored stream; a
+ * p_M read touches only the base and the first M-2 planes (Section 3.3).
+ *
+ * Conventions for every entry point:
+ *  - Shapes are out x in (row = output channel; K = in). Groups are runs of
+ *    `group` consecutive weights along K inside one row.
+ *  - fp16 values are passed as IEEE binary16 bit patterns (uint16_t).
+ *  - Functions return a status code (STAGQ_OK = 0 on success); no C++
+ *    exception crosses this boundary. stagq_last_error() gives a detail
+ *    message for the calling thread's most recent failure.
+ *  - Pointers documented as "host" must be host memory; "device" must be
+ *    device memory of the handle's GPU. The library never frees a caller's
+ *    pointer.
+ */
+#ifndef STAGQ_H
+#define STAGQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------- status */
+#define STAGQ_OK 0
+#define STAGQ_EINVAL 1   /* bad argument: null pointer, bits out of range, n out of range, bad shape */
+#define STAGQ_EFORMAT 2  /* malformed stream: row_ptr not monotone, col >= in, bad file header */
+#define STAGQ_ENOMEM 3   /* host or device allocation failed */
+#define STAGQ_ECUDA 4    /* a CUDA runtime call failed (detail in stagq_last_error) */
+#define STAGQ_EIO 5      /* file could not be read or written */
+#define STAGQ_ENODEV 6   /* no usable sm_100 device */
+
+/* Limits of this implementation. */
+#define STAGQ_MAX_PLANES 4      /* stream depth N = 2 + n_planes <= 6 (the paper evaluates N = 6) */
+#define STAGQ_MAX_BATCH 4       /* columns of x per call in stagq_gemv_n */
+#define STAGQ_MAX_IN 32768      /* K; side-record columns are stored as uint16 */
+#define STAGQ_IN_MULTIPLE 128   /* K must be a multiple of this (16-byte plane rows) */
+
+/* Pair search mode of the encoder (Section 3.1). */
+#define STAGQ_PAIR_SEARCH 0     /* argmin of Eq. (5) over all 256 codebook pairs */
+#define STAGQ_PAIR_FAST 1       /* nearest codebook entry per coordinate (labelled shortcut) */
+
+/* Flags of stagq_gemv_ex. */
+#define STAGQ_Y_F32 1u          /* y is fp32 instead of fp16 */
+
+typedef struct stagq_matrix* stagq_handle;   /* opaque; owned by the library */
+
+/*
+ * Logical fields of one encoded matrix (Sections 3.3-3.6): one byte per
+ * digit, no physical layout. Filled by stagq_encode, consumed by stagq_pack.
+ * All arrays are host memory owned by the caller.
+ *   q         [out*in]            base digit 0..3, row-major
+ *   planes    [n_planes*out*in]   b_k in {0,1}; plane k (k = 3..2+n_planes) at offset (k-3)*out*in
+ *   pair_idx  [out*(in/group)]    8-bit pair: high nibble = log2(s) codebook index, low = lo/s index
+ *   row_ptr   [out+1]             side record (CSR): entries of row r are [row_ptr[r], row_ptr[r+1])
+ *   col       [nnz]               column of each held-out weight, increasing inside a row
+ *   val       [nnz]               recorded fp16 value P (pre-grid guard, Eq. 4)
+ * Held-out positions carry zero digits (q = 0, all b_k = 0).
+ */
+typedef struct {
+    int32_t out, in, group, n_planes;
+    int64_t nnz;
+    uint16_t codebook_log2s[16];
+    uint16_t codebook_lo_over_s[16];
+    uint8_t* q;
+    uint8_t* planes;
+    uint8_t* pair_idx;
+    int32_t* row_ptr;
+    uint16_t* col;
+    uint16_t* val;
+} stagq_fields;
+
+/*
+ * Packed, plane-major stream (Section 3.3: base first, then the planes in
+ * order of k, so a shallower read skips the deeper planes). Host memory,
+ * owned by the caller.
+ *   planes: stagq_stream_plane_bytes(out, in, n_planes) bytes =
+ *           [base: out*in/4 B][plane 3: out*in/8 B]...[plane 2+n_planes: out*in/8 B]
+ *           Each plane is row-major; inside a row the weights are stored in
+ *           64-weight lane chunks whose bit order is the library's own.
+ *   pair_idx, row_ptr, col, val: as in stagq_fields.
+ */
+typedef struct {
+    int32_t out, in, group, n_planes;
+    int64_t nnz;
+    uint16_t codebook_log2s[16];
+    uint16_t codebook_lo_over_s[16];
+    const uint8_t* planes;
+    const uint8_t* pair_idx;
+    const int32_t* row_ptr;
+    const uint16_t* col;
+    const uint16_t* val;
+} stagq_host_stream;
+
+typedef struct {
+    int32_t out, in, group, n_planes;
+    int64_t nnz;
+    int32_t device;
+    int64_t device_bytes;     /* bytes the handle holds on the GPU */
+} stagq_info_t;
+
+/* ------------------------------------------------------------- encoding */
+
+/* Number of side-record entries for a density: round(density*out*in), half up. */
+int64_t stagq_side_record_count(int32_t out, int32_t in, double density);
+
+/*
+ * Encoder of Sections 3.1-3.6 / Appendices B, E for a synthetic fp16 matrix
+ * (host, multithreaded): global top-|w| side record with `density`, held-out
+ * entries clipped inward for the fit, initial pair (Appendix B), uniform fp16
+ * codebooks (Appendix E), pair per group by `pair_mode`, nearest-rounding
+ * base, sign planes (Eq. 7), zero digits at held-out positions.
+ *   w        host [out*in] fp16 bits, row-major
+ *   f        caller sets out, in, group, n_planes and points every array at a
+ *            buffer of the documented size, with nnz = stagq_side_record_count(...);
+ *            the encoder fills codebooks and arrays.
+ *   n_threads  0 = all hardware threads.
+ * Errors: STAGQ_EINVAL (null, group does not divide in, n_planes > STAGQ_MAX_PLANES,
+ *         nnz mismatch, in > STAGQ_MAX_IN), STAGQ_ENOMEM.
+ */
+int stagq_encode(const uint16_t* w, double density, int32_t pair_mode, int32_t n_threads,
+                 stagq_fields* f);
+
+/* Size in bytes of the packed plane region: out*in/4 + n_planes*out*in/8. */
+int64_t stagq_stream_plane_bytes(int32_t out, int32_t in, int32_t n_planes);
+
+/*
+ * Packer (host): lays the logical digits of `f` out plane-major into
+ * `planes_out` (stagq_stream_plane_bytes bytes, caller-owned).
+ * Errors: STAGQ_EINVAL (null, in not a multiple of STAGQ_IN_MULTIPLE, digit out of range).
+ */
+int stagq_pack(const stagq_fields* f, uint8_t* planes_out);
+
+/*
+ * Host re-read of a packed stream: u_M (Eq. 8) per weight into u_out
+ * (host [out*in], row-major), using the same bit manipulations as the GPU
+ * kernels. For checking a stream on a machine without a GPU; no GEMV runs here.
+ */
+int stagq_unpack_levels_host(const stagq_host_stream* s, int bits, uint8_t* u_out);
+
+/* Serialise a stream to a file (one checkpoint serving every precision,
+ * Section 1) and read it back straight onto a GPU. */
+int stagq_save(const stagq_host_stream* s, const char* path);
+int stagq_load_file(const char* path, int device, stagq_handle* out);
+
+/* ------------------------------------------------------------ the GEMV */
+
+/*
+ * Copy a stream to GPU `device` and build the per-precision (lo_M, s_M)
+ * tables (Eq. 10, computed in fp64 on the host, stored fp32).
+ * The caller keeps ownership of every host array; the handle owns its device
+ * copies until stagq_free.
+ * Errors: STAGQ_EINVAL, STAGQ_EFORMAT (row_ptr not monotone or not ending at
+ * nnz, col >= in), STAGQ_ENOMEM, STAGQ_ENODEV, STAGQ_ECUDA.
+ */
+int stagq_load(const stagq_host_stream* s, int device, stagq_handle* out);
+
+/*
+ * y = W_hat^(bits) x for one vector (n = 1), asynchronously on `cuda_stream`
+ * (a cudaStream_t; NULL = the legacy default stream).
+ *   bits   2 .. 2 + n_planes
+ *   x      device [in]  fp16
+ *   y      device [out] fp16 (fp32 accumulation, rounded to nearest even)
+ * Calls on one handle may run concurrently: the GEMV uses no scratch memory.
+ * Errors: STAGQ_EINVAL (null handle/pointer, bits out of range), STAGQ_ECUDA (launch failure).
+ */
+int stagq_gemv(stagq_handle h, int bits, const void* x, void* y, void* cuda_stream);
+
+/* n columns (1 <= n <= STAGQ_MAX_BATCH): x device [n*in], y device [n*out], row-major. */
+int stagq_gemv_n(stagq_handle h, int bits, const void* x, int n, void* y, void* cuda_stream);
+
+/* As stagq_gemv_n; flags STAGQ_Y_F32 makes y fp32. */
+int stagq_gemv_ex(stagq_handle h, int bits, const void* x, int n, void* y, uint32_t flags,
+                  void* cuda_stream);
+
+/*
+ * End-to-end call with HOST buffers: copies x (host [n*in] fp16) to the
+ * device, runs the GEMV and copies y (host [n*out] fp16) back, all on
+ * `cuda_stream`, and returns after the copy of y has completed. Uses a
+ * device staging buffer owned by the handle, so calls on one handle must
+ * not overlap.
+ */
+int stagq_gemv_host(stagq_handle h, int bits, const void* x_host, int n, void* y_host,
+                    void* cuda_stream);
+
+/* Test hook: u_M per weight (device [out*in] uint8, row-major), decoded on the GPU. */
+int stagq_decode_levels(stagq_handle h, int bits, uint8_t* u_dev, void* cuda_stream);
+
+/*
+ * Algorithmic bytes of one call (the roofline numerator):
+ *   out*in*bits/8 (base + bits-2 planes) + out*in/group (pairs)
+ *   + 4*nnz + 4*(out+1) (side record) + 2*n*in (x) + 2*n*out (y).
+ * Returns -1 for a bad handle or bits.
+ */
+int64_t stagq_bytes(stagq_handle h, int bits, int n);
+
+int stagq_info(stagq_handle h, stagq_info_t* info);
+
+/* Release the handle's device memory. Null-safe. */
+void stagq_free(stagq_handle h);
+
+const char* stagq_strerror(int status);
+const char* stagq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* STAGQ_H */

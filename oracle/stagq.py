@@ -39,8 +39,9 @@ INIT_EDGE_FRACTION = 0.06
 FLOOR_LAMBDA = 4.0
 # Section 3.1: two sixteen-entry codebooks per matrix.
 CODEBOOK_SIZE = 16
-# Reading: a group whose clipped range is zero gets this step so that
-# log2(s0) stays finite (fp16's smallest positive value).
+# Reading: a group whose clipped range is zero has no initial step; it gets
+# this placeholder, stays out of the codebook fit and takes its pair by the
+# Eq. (5) search in every mode.
 DEGENERATE_STEP = 2.0 ** -24
 
 
@@ -225,8 +226,8 @@ def initial_pairs(Vc: np.ndarray, group: int):
     two 6 % in from the group's ends (a step of 0.29 of the range).
 
     lo0 = min + 0.06 R, top = max - 0.06 R, s0 = (top - lo0) / 3, R = max - min.
-    Reading: a group of zero range gets s0 = 2^-24. Returns (lo0, s0), each
-    [out, ngroups] fp64.
+    Reading: a group of zero range gets s0 = 2^-24 and is flagged. Returns
+    (lo0, s0, flat), each [out, ngroups]; flat marks the zero-range groups.
     """
     out, inp = Vc.shape
     G = Vc.reshape(out, inp // group, group)
@@ -236,8 +237,9 @@ def initial_pairs(Vc: np.ndarray, group: int):
     lo0 = mn + INIT_EDGE_FRACTION * R
     top = mx - INIT_EDGE_FRACTION * R
     s0 = (top - lo0) / 3.0
-    s0 = np.where(R > 0.0, s0, DEGENERATE_STEP)
-    return lo0, s0
+    flat = ~(R > 0.0)
+    s0 = np.where(flat, DEGENERATE_STEP, s0)
+    return lo0, s0, flat
 
 
 def uniform_codebook(values: np.ndarray) -> np.ndarray:
@@ -255,10 +257,11 @@ def uniform_codebook(values: np.ndarray) -> np.ndarray:
     return np.array(cb, dtype=np.float64).astype(np.float16)
 
 
-def fit_codebooks(lo0: np.ndarray, s0: np.ndarray, empty: np.ndarray):
+def fit_codebooks(lo0: np.ndarray, s0: np.ndarray, skip: np.ndarray):
     """Section 3.1: one codebook in log2(s) and one in lo/s per matrix, fitted
-    to the initial pairs of the groups that keep at least one entry."""
-    keep = ~empty
+    to the initial pairs of the groups not marked in ``skip`` (Reading: groups
+    with no retained entry or zero range have no initial pair to fit)."""
+    keep = ~skip
     cb_log2s = uniform_codebook(np.log2(s0[keep]))
     cb_lo_over_s = uniform_codebook(lo0[keep] / s0[keep])
     return cb_log2s, cb_lo_over_s
@@ -293,16 +296,22 @@ def pair_cost(V: np.ndarray, lo, s, N: int):
     _, _, recons = encode_digits(V, lo, s, N)
     first = 0.0
     for rec in recons:                       # M = 2 .. N
-        first = first + np.sum((V - rec) ** 2, axis=-1)
+        first = first + _sum_in_order((V - rec) ** 2)
     first = first / (N - 1)
     rho = reach(s, N)
-    floor = np.sum(np.maximum(np.abs(V - recons[0]) - rho, 0.0) ** 2, axis=-1)
+    floor = _sum_in_order(np.maximum(np.abs(V - recons[0]) - rho, 0.0) ** 2)
     return first + FLOOR_LAMBDA * floor
+
+
+def _sum_in_order(a):
+    """Sum over the last axis in index order c = 0, 1, ... (a fixed rounding
+    order, so that any other implementation of Eq. (5) can reproduce it)."""
+    return np.cumsum(a, axis=-1)[..., -1]
 
 
 def choose_pairs(Vc: np.ndarray, group: int, N: int, lo_tab, s_tab, empty,
                  mode: str = "search", lo0=None, s0=None, cb_log2s=None,
-                 cb_lo_over_s=None, chunk: int = 256) -> np.ndarray:
+                 cb_lo_over_s=None, flat=None, chunk: int = 256) -> np.ndarray:
     """Per-group pair choice.
 
     mode "search" (Section 3.1): the combination minimising Eq. (5) over all
@@ -310,7 +319,8 @@ def choose_pairs(Vc: np.ndarray, group: int, N: int, lo_tab, s_tab, empty,
     mode "fast" (a labelled shortcut for very large stacks, not the paper's
     rule): the nearest codebook entry to log2(s0) and to lo0/s0 separately,
     ties to the smaller index.
-    Groups with no retained entry get pair 0 (their digits are all zero).
+    Groups with no retained entry get pair 0 (their digits are all zero);
+    zero-range groups (``flat``) are searched in both modes.
     """
     out, inp = Vc.shape
     ng = inp // group
@@ -322,6 +332,10 @@ def choose_pairs(Vc: np.ndarray, group: int, N: int, lo_tab, s_tab, empty,
         a = np.argmin(da, axis=2)
         b = np.argmin(db, axis=2)
         idx = (a * CODEBOOK_SIZE + b).astype(np.uint8)
+        if flat is not None and np.any(flat & ~empty):
+            sel = flat & ~empty
+            searched = choose_pairs(Vc, group, N, lo_tab, s_tab, empty, mode="search")
+            idx = np.where(sel, searched, idx)
     elif mode == "search":
         G = Vc.reshape(out * ng, group)
         idx = np.empty(out * ng, dtype=np.uint8)
@@ -336,7 +350,8 @@ def choose_pairs(Vc: np.ndarray, group: int, N: int, lo_tab, s_tab, empty,
 
 
 def encode(W: np.ndarray, group: int = 128, n_planes: int = 2,
-           density: float = 0.005, mode: str = "search") -> Fields:
+           density: float = 0.005, mode: str = "search", rows=None,
+           row_block: int = 512) -> Fields:
     """Figure 3's encoder for synthetic weights (no AWQ scale: with x ~ N(0,1)
     every channel scale is equal; no post-grid guard):
 
@@ -348,6 +363,11 @@ def encode(W: np.ndarray, group: int = 128, n_planes: int = 2,
        store zero digits (Reading: the planes skip them, Section 3.6, and the
        paper gives no stored value -- zeros make the main stream decode to
        lo_M there, which Eq. (4) then masks).
+
+    Steps 1-4 look at the whole matrix (global record, per-matrix codebooks).
+    With ``rows`` given, steps 5-7 run only for those rows and the returned
+    Fields hold just them (out = len(rows)); the encoding of a row depends on
+    nothing else. Rows are processed ``row_block`` at a time to bound memory.
     """
     W = np.asarray(W)
     if W.dtype != np.float16:
@@ -360,30 +380,37 @@ def encode(W: np.ndarray, group: int = 128, n_planes: int = 2,
 
     mask = select_side_record(W, density)
     Vc, empty = clip_held_out(W, mask, group)
-    lo0, s0 = initial_pairs(Vc, group)
-    cb_log2s, cb_lo_over_s = fit_codebooks(lo0, s0, empty)
+    lo0, s0, flat = initial_pairs(Vc, group)
+    cb_log2s, cb_lo_over_s = fit_codebooks(lo0, s0, empty | flat)
     lo_tab, s_tab = pair_table(cb_log2s, cb_lo_over_s)
-    pair_idx = choose_pairs(Vc, group, N, lo_tab, s_tab, empty, mode=mode,
-                            lo0=lo0, s0=s0, cb_log2s=cb_log2s,
-                            cb_lo_over_s=cb_lo_over_s)
 
-    lo_g = lo_tab[pair_idx.astype(np.int64)]             # [out, ng]
-    s_g = s_tab[pair_idx.astype(np.int64)]
-    lo_w = np.repeat(lo_g, group, axis=1)
-    s_w = np.repeat(s_g, group, axis=1)
-    q, bits, _ = encode_digits(W.astype(np.float64), lo_w, s_w, N)
-    q = np.where(mask, 0, q).astype(np.uint8)
-    planes = np.zeros((n_planes, out, inp), dtype=np.uint8)
-    for k in range(n_planes):
-        planes[k] = np.where(mask, 0, bits[k]).astype(np.uint8)
+    rows = np.arange(out) if rows is None else np.asarray(rows, dtype=np.int64)
+    n = rows.size
+    pair_idx = np.empty((n, ng), dtype=np.uint8)
+    q = np.empty((n, inp), dtype=np.uint8)
+    planes = np.empty((n_planes, n, inp), dtype=np.uint8)
+    for b0 in range(0, n, row_block):
+        rb = rows[b0:b0 + row_block]
+        sl = slice(b0, b0 + rb.size)
+        pair_idx[sl] = choose_pairs(Vc[rb], group, N, lo_tab, s_tab, empty[rb], mode=mode,
+                                    lo0=lo0[rb], s0=s0[rb], cb_log2s=cb_log2s,
+                                    cb_lo_over_s=cb_lo_over_s, flat=flat[rb])
+        lo_w = np.repeat(lo_tab[pair_idx[sl].astype(np.int64)], group, axis=1)
+        s_w = np.repeat(s_tab[pair_idx[sl].astype(np.int64)], group, axis=1)
+        qb, bits, _ = encode_digits(W[rb].astype(np.float64), lo_w, s_w, N)
+        m = mask[rb]
+        q[sl] = np.where(m, 0, qb)
+        for k in range(n_planes):
+            planes[k, sl] = np.where(m, 0, bits[k])
 
-    rows, cols = np.nonzero(mask)                         # row-major order
-    row_ptr = np.zeros(out + 1, dtype=np.int64)
-    np.add.at(row_ptr, rows + 1, 1)
+    sub = mask[rows]
+    r_idx, cols = np.nonzero(sub)                         # row-major order
+    row_ptr = np.zeros(n + 1, dtype=np.int64)
+    np.add.at(row_ptr, r_idx + 1, 1)
     row_ptr = np.cumsum(row_ptr)
-    val = W[rows, cols].astype(np.float16)
-    return Fields(out=out, inp=inp, group=group, n_planes=n_planes, q=q,
-                  planes=planes, pair_idx=pair_idx.astype(np.uint8),
+    val = W[rows[r_idx], cols].astype(np.float16)
+    return Fields(out=n, inp=inp, group=group, n_planes=n_planes, q=q,
+                  planes=planes, pair_idx=pair_idx,
                   cb_log2s=cb_log2s, cb_lo_over_s=cb_lo_over_s,
                   row_ptr=row_ptr, col=cols.astype(np.int64), val=val)
 

@@ -1,0 +1,300 @@
+"""StagQ multi-precision batch-one GEMV on B200 (sm_100a).
+
+Thin ctypes binding of ``libstagq.so`` (see ``include/stagq.h``): the
+functions below carry the C ABI's names and only marshal arguments. Every
+step of the GEMV runs in the library's CUDA kernels; PyTorch is used only for
+device memory and streams. If the library is missing this package raises --
+there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libstagq.so")
+
+STAGQ_OK = 0
+STAGQ_PAIR_SEARCH = 0
+STAGQ_PAIR_FAST = 1
+STAGQ_Y_F32 = 1
+STAGQ_MAX_PLANES = 4
+STAGQ_MAX_BATCH = 4
+
+_c_p = ctypes.c_void_p
+_i32, _i64, _u32, _dbl = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_double
+
+
+class _Fields(ctypes.Structure):
+    _fields_ = [("out", _i32), ("in_", _i32), ("group", _i32), ("n_planes", _i32), ("nnz", _i64),
+                ("codebook_log2s", ctypes.c_uint16 * 16), ("codebook_lo_over_s", ctypes.c_uint16 * 16),
+                ("q", _c_p), ("planes", _c_p), ("pair_idx", _c_p), ("row_ptr", _c_p),
+                ("col", _c_p), ("val", _c_p)]
+
+
+class _HostStream(ctypes.Structure):
+    _fields_ = [("out", _i32), ("in_", _i32), ("group", _i32), ("n_planes", _i32), ("nnz", _i64),
+                ("codebook_log2s", ctypes.c_uint16 * 16), ("codebook_lo_over_s", ctypes.c_uint16 * 16),
+                ("planes", _c_p), ("pair_idx", _c_p), ("row_ptr", _c_p), ("col", _c_p), ("val", _c_p)]
+
+
+class _Info(ctypes.Structure):
+    _fields_ = [("out", _i32), ("in_", _i32), ("group", _i32), ("n_planes", _i32), ("nnz", _i64),
+                ("device", _i32), ("device_bytes", _i64)]
+
+
+_SIGNATURES = {
+    "stagq_side_record_count": (_i64, [_i32, _i32, _dbl]),
+    "stagq_encode": (ctypes.c_int, [_c_p, _dbl, _i32, _i32, ctypes.POINTER(_Fields)]),
+    "stagq_stream_plane_bytes": (_i64, [_i32, _i32, _i32]),
+    "stagq_pack": (ctypes.c_int, [ctypes.POINTER(_Fields), _c_p]),
+    "stagq_unpack_levels_host": (ctypes.c_int, [ctypes.POINTER(_HostStream), ctypes.c_int, _c_p]),
+    "stagq_save": (ctypes.c_int, [ctypes.POINTER(_HostStream), ctypes.c_char_p]),
+    "stagq_load_file": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_int, ctypes.POINTER(_c_p)]),
+    "stagq_load": (ctypes.c_int, [ctypes.POINTER(_HostStream), ctypes.c_int, ctypes.POINTER(_c_p)]),
+    "stagq_gemv": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, _c_p, _c_p]),
+    "stagq_gemv_n": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _c_p]),
+    "stagq_gemv_ex": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _u32, _c_p]),
+    "stagq_gemv_host": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _c_p]),
+    "stagq_decode_levels": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, _c_p]),
+    "stagq_bytes": (_i64, [_c_p, ctypes.c_int, ctypes.c_int]),
+    "stagq_info": (ctypes.c_int, [_c_p, ctypes.POINTER(_Info)]),
+    "stagq_free": (None, [_c_p]),
+    "stagq_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+    "stagq_last_error": (ctypes.c_char_p, []),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libstagq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                               "`python -m quantized_gemv_stagq_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+class StagqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        L = lib()
+        msg = L.stagq_strerror(status).decode()
+        detail = L.stagq_last_error().decode()
+        super().__init__(f"{where}: {msg} ({detail})")
+        self.status = status
+
+
+def _check(status: int, where: str) -> None:
+    if status != STAGQ_OK:
+        raise StagqError(status, where)
+
+
+def _ptr(a) -> int:
+    return a.ctypes.data if a is not None and a.size else 0
+
+
+# ------------------------------------------------------------------ host side
+
+@dataclass
+class Fields:
+    """Logical fields of an encoded matrix (numpy, host)."""
+    out: int
+    inp: int
+    group: int
+    n_planes: int
+    q: np.ndarray            # uint8 [out, inp]
+    planes: np.ndarray       # uint8 [n_planes, out, inp]
+    pair_idx: np.ndarray     # uint8 [out, inp // group]
+    cb_log2s: np.ndarray     # uint16 [16] fp16 bits
+    cb_lo_over_s: np.ndarray  # uint16 [16] fp16 bits
+    row_ptr: np.ndarray      # int32 [out + 1]
+    col: np.ndarray          # uint16 [nnz]
+    val: np.ndarray          # uint16 [nnz] fp16 bits
+
+    @property
+    def nnz(self) -> int:
+        return int(self.col.shape[0])
+
+    def _c(self) -> _Fields:
+        f = _Fields(self.out, self.inp, self.group, self.n_planes, self.nnz)
+        f.codebook_log2s[:] = [int(v) for v in self.cb_log2s]
+        f.codebook_lo_over_s[:] = [int(v) for v in self.cb_lo_over_s]
+        f.q, f.planes, f.pair_idx = _ptr(self.q), _ptr(self.planes), _ptr(self.pair_idx)
+        f.row_ptr, f.col, f.val = _ptr(self.row_ptr), _ptr(self.col), _ptr(self.val)
+        return f
+
+
+@dataclass
+class HostStream:
+    """Packed plane-major stream (numpy, host)."""
+    out: int
+    inp: int
+    group: int
+    n_planes: int
+    planes: np.ndarray       # uint8, stagq_stream_plane_bytes bytes
+    pair_idx: np.ndarray
+    cb_log2s: np.ndarray
+    cb_lo_over_s: np.ndarray
+    row_ptr: np.ndarray
+    col: np.ndarray
+    val: np.ndarray
+
+    @property
+    def nnz(self) -> int:
+        return int(self.col.shape[0])
+
+    def _c(self) -> _HostStream:
+        s = _HostStream(self.out, self.inp, self.group, self.n_planes, self.nnz)
+        s.codebook_log2s[:] = [int(v) for v in self.cb_log2s]
+        s.codebook_lo_over_s[:] = [int(v) for v in self.cb_lo_over_s]
+        s.planes, s.pair_idx, s.row_ptr = _ptr(self.planes), _ptr(self.pair_idx), _ptr(self.row_ptr)
+        s.col, s.val = _ptr(self.col), _ptr(self.val)
+        return s
+
+
+def stagq_side_record_count(out: int, inp: int, density: float) -> int:
+    return int(lib().stagq_side_record_count(out, inp, density))
+
+
+def stagq_stream_plane_bytes(out: int, inp: int, n_planes: int) -> int:
+    return int(lib().stagq_stream_plane_bytes(out, inp, n_planes))
+
+
+def stagq_encode(w: np.ndarray, group: int = 128, n_planes: int = 2, density: float = 0.005,
+                 mode: str = "search", n_threads: int = 0) -> Fields:
+    """Encode an fp16 [out, inp] matrix (library encoder, host)."""
+    w = np.ascontiguousarray(w, dtype=np.float16)
+    out, inp = w.shape
+    nnz = stagq_side_record_count(out, inp, density)
+    F = Fields(out, inp, group, n_planes,
+               q=np.empty((out, inp), np.uint8),
+               planes=np.empty((n_planes, out, inp), np.uint8),
+               pair_idx=np.empty((out, inp // group), np.uint8),
+               cb_log2s=np.zeros(16, np.uint16), cb_lo_over_s=np.zeros(16, np.uint16),
+               row_ptr=np.empty(out + 1, np.int32), col=np.empty(nnz, np.uint16),
+               val=np.empty(nnz, np.uint16))
+    cf = F._c()
+    m = {"search": STAGQ_PAIR_SEARCH, "fast": STAGQ_PAIR_FAST}[mode]
+    _check(lib().stagq_encode(w.ctypes.data, density, m, n_threads, ctypes.byref(cf)), "stagq_encode")
+    F.cb_log2s = np.array(cf.codebook_log2s[:], dtype=np.uint16)
+    F.cb_lo_over_s = np.array(cf.codebook_lo_over_s[:], dtype=np.uint16)
+    return F
+
+
+def stagq_pack(F: Fields) -> HostStream:
+    """Lay the digits of F out plane-major (library packer, host)."""
+    planes = np.empty(stagq_stream_plane_bytes(F.out, F.inp, F.n_planes), np.uint8)
+    q = np.ascontiguousarray(F.q, dtype=np.uint8)
+    pl = np.ascontiguousarray(F.planes, dtype=np.uint8)
+    G = Fields(F.out, F.inp, F.group, F.n_planes, q, pl, F.pair_idx, F.cb_log2s, F.cb_lo_over_s,
+               F.row_ptr, F.col, F.val)
+    cf = G._c()
+    _check(lib().stagq_pack(ctypes.byref(cf), planes.ctypes.data), "stagq_pack")
+    return HostStream(F.out, F.inp, F.group, F.n_planes, planes,
+                      np.ascontiguousarray(F.pair_idx, np.uint8),
+                      np.asarray(F.cb_log2s, np.uint16), np.asarray(F.cb_lo_over_s, np.uint16),
+                      np.ascontiguousarray(F.row_ptr, np.int32), np.ascontiguousarray(F.col, np.uint16),
+                      np.ascontiguousarray(F.val, np.uint16))
+
+
+def stagq_unpack_levels_host(S: HostStream, bits: int) -> np.ndarray:
+    u = np.empty((S.out, S.inp), np.uint8)
+    cs = S._c()
+    _check(lib().stagq_unpack_levels_host(ctypes.byref(cs), bits, u.ctypes.data), "stagq_unpack_levels_host")
+    return u
+
+
+def stagq_save(S: HostStream, path: str) -> None:
+    cs = S._c()
+    _check(lib().stagq_save(ctypes.byref(cs), path.encode()), "stagq_save")
+
+
+# ------------------------------------------------------------------ GPU side
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+class Matrix:
+    """A stream loaded onto one GPU (owns a stagq_handle)."""
+
+    def __init__(self, handle: int):
+        self.handle = ctypes.c_void_p(handle)
+        info = _Info()
+        _check(lib().stagq_info(self.handle, ctypes.byref(info)), "stagq_info")
+        self.out, self.inp, self.group = info.out, info.in_, info.group
+        self.n_planes, self.nnz, self.device = info.n_planes, info.nnz, info.device
+        self.device_bytes = info.device_bytes
+
+    def free(self) -> None:
+        if self.handle is not None and self.handle.value:
+            lib().stagq_free(self.handle)
+        self.handle = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def stagq_load(S: HostStream, device: int = 0) -> Matrix:
+    h = ctypes.c_void_p()
+    cs = S._c()
+    _check(lib().stagq_load(ctypes.byref(cs), device, ctypes.byref(h)), "stagq_load")
+    return Matrix(h.value)
+
+
+def stagq_load_file(path: str, device: int = 0) -> Matrix:
+    h = ctypes.c_void_p()
+    _check(lib().stagq_load_file(path.encode(), device, ctypes.byref(h)), "stagq_load_file")
+    return Matrix(h.value)
+
+
+def stagq_gemv_ex(m: Matrix, bits: int, x, y, n: int = 1, flags: int = 0, stream=None) -> None:
+    """x, y: CUDA tensors (x fp16 [n, inp]; y fp16 or fp32 [n, out])."""
+    _check(lib().stagq_gemv_ex(m.handle, bits, x.data_ptr(), n, y.data_ptr(), flags,
+                               _stream_ptr(stream)), "stagq_gemv_ex")
+
+
+def stagq_gemv(m: Matrix, bits: int, x, y, stream=None) -> None:
+    _check(lib().stagq_gemv(m.handle, bits, x.data_ptr(), y.data_ptr(), _stream_ptr(stream)), "stagq_gemv")
+
+
+def stagq_gemv_n(m: Matrix, bits: int, x, n: int, y, stream=None) -> None:
+    _check(lib().stagq_gemv_n(m.handle, bits, x.data_ptr(), n, y.data_ptr(), _stream_ptr(stream)),
+           "stagq_gemv_n")
+
+
+def stagq_gemv_host(m: Matrix, bits: int, x_host: np.ndarray, y_host: np.ndarray, n: int = 1,
+                    stream=None) -> None:
+    """Host buffers (pinned or pageable numpy arrays): copies in and out, synchronous."""
+    _check(lib().stagq_gemv_host(m.handle, bits, x_host.ctypes.data, n, y_host.ctypes.data,
+                                 _stream_ptr(stream)), "stagq_gemv_host")
+
+
+def stagq_decode_levels(m: Matrix, bits: int, u_dev, stream=None) -> None:
+    _check(lib().stagq_decode_levels(m.handle, bits, u_dev.data_ptr(), _stream_ptr(stream)),
+           "stagq_decode_levels")
+
+
+def stagq_bytes(m: Matrix, bits: int, n: int = 1) -> int:
+    return int(lib().stagq_bytes(m.handle, bits, n))
+
+
+def stagq_free(m: Matrix) -> None:
+    m.free()

@@ -1,0 +1,251 @@
+// C ABI of libstagq.so: handle lifecycle, loading a stream onto a GPU, and the
+// GEMV entry points. See include/stagq.h for the contract of each function.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "device_matrix.hpp"
+#include "host_common.hpp"
+#include "stream.hpp"
+
+struct stagq_matrix {
+  int device = -1;
+  stagq::DeviceMatrix dm{};
+  void* d_mem = nullptr;
+  size_t d_bytes = 0;
+  void* d_stage = nullptr;      // x / y staging for stagq_gemv_host
+  size_t stage_bytes = 0;
+};
+
+namespace stagq {
+namespace {
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(STAGQ_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+// Restores the caller's current device on scope exit.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) == cudaSuccess && cudaSetDevice(dev) == cudaSuccess) ok = true;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Per-precision (lo_M, s_M c_M) for the 256 pairs, Eq. (10) in fp64, stored fp32.
+void build_tables(const stagq_host_stream* s, std::vector<float2>& t) {
+  const int N = 2 + s->n_planes;
+  t.assign((size_t)(N - 1) * 256, make_float2(0.f, 0.f));
+  for (int M = 2; M <= N; ++M) {
+    for (int p = 0; p < 256; ++p) {
+      const double sp = std::exp2(half_to_double(s->codebook_log2s[p >> 4]));
+      const double lo = half_to_double(s->codebook_lo_over_s[p & 15]) * sp;
+      const double sM = sp / std::ldexp(1.0, M - 2);
+      const double loM = lo - sp * (std::ldexp(1.0, M - 2) - 1.0) / std::ldexp(1.0, M - 1);
+      t[(size_t)(M - 2) * 256 + p] = make_float2((float)loM, (float)(sM * composite_factor(M)));
+    }
+  }
+}
+
+int check_handle_bits(stagq_handle h, int bits) {
+  if (!h) return fail(STAGQ_EINVAL, "null handle");
+  if (bits < 2 || bits > 2 + h->dm.n_planes) return fail(STAGQ_EINVAL, "bits outside 2..2+n_planes");
+  return STAGQ_OK;
+}
+
+}  // namespace
+}  // namespace stagq
+
+using namespace stagq;
+
+extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* out) {
+  if (!out) return fail(STAGQ_EINVAL, "stagq_load: null output handle");
+  *out = nullptr;
+  int st = validate_stream(s);
+  if (st) return st;
+  int ndev = 0;
+  cudaError_t e = cudaGetDeviceCount(&ndev);
+  if (e != cudaSuccess || ndev == 0) return fail(STAGQ_ENODEV, "no CUDA device");
+  if (device < 0 || device >= ndev) return fail(STAGQ_EINVAL, "device index out of range");
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+  if (prop.major != 10) return fail(STAGQ_ENODEV, std::string("kernels are built for sm_100a; device is ") + prop.name);
+
+  DeviceGuard guard(device);
+  if (!guard.ok) return fail(STAGQ_ECUDA, "cudaSetDevice failed");
+
+  const int64_t out_ = s->out, in = s->in;
+  const int np = s->n_planes;
+  const size_t base_bytes = (size_t)(out_ * in / 4), plane_bytes = (size_t)(out_ * in / 8);
+  const size_t pair_bytes = (size_t)(out_ * (in / s->group));
+  const size_t rp_bytes = (size_t)(out_ + 1) * 4, ent_bytes = (size_t)s->nnz * 4;
+  const size_t tab_bytes = (size_t)(np + 1) * 256 * sizeof(float2);
+  size_t off = 0;
+  const size_t o_base = off; off = align_up(off + base_bytes, 256);
+  size_t o_plane[STAGQ_MAX_PLANES] = {};
+  for (int k = 0; k < np; ++k) { o_plane[k] = off; off = align_up(off + plane_bytes, 256); }
+  const size_t o_pair = off; off = align_up(off + pair_bytes, 256);
+  const size_t o_rp = off; off = align_up(off + rp_bytes, 256);
+  const size_t o_ent = off; off = align_up(off + (ent_bytes ? ent_bytes : 4), 256);
+  const size_t o_tab = off; off = align_up(off + tab_bytes, 256);
+  const size_t total = off;
+
+  stagq_matrix* h = new (std::nothrow) stagq_matrix();
+  if (!h) return fail(STAGQ_ENOMEM, "host allocation failed");
+  h->device = device;
+  e = cudaMalloc(&h->d_mem, total);
+  if (e != cudaSuccess) {
+    delete h;
+    cudaGetLastError();
+    return fail(STAGQ_ENOMEM, std::string("cudaMalloc of stream failed: ") + cudaGetErrorString(e));
+  }
+  h->d_bytes = total;
+  uint8_t* d = static_cast<uint8_t*>(h->d_mem);
+
+  std::vector<uint32_t> ent((size_t)s->nnz);
+  for (int64_t i = 0; i < s->nnz; ++i) ent[i] = (uint32_t)s->col[i] | ((uint32_t)s->val[i] << 16);
+  std::vector<float2> tabs;
+  build_tables(s, tabs);
+
+  struct Copy { size_t off; const void* src; size_t n; };
+  std::vector<Copy> copies = {{o_base, s->planes, base_bytes}};
+  for (int k = 0; k < np; ++k) copies.push_back({o_plane[k], s->planes + base_bytes + (size_t)k * plane_bytes, plane_bytes});
+  copies.push_back({o_pair, s->pair_idx, pair_bytes});
+  copies.push_back({o_rp, s->row_ptr, rp_bytes});
+  if (ent_bytes) copies.push_back({o_ent, ent.data(), ent_bytes});
+  copies.push_back({o_tab, tabs.data(), tab_bytes});
+  for (const Copy& c : copies) {
+    e = cudaMemcpy(d + c.off, c.src, c.n, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+      cudaFree(h->d_mem);
+      delete h;
+      return cuda_fail(e, "cudaMemcpy of stream");
+    }
+  }
+  DeviceMatrix& m = h->dm;
+  m.out = s->out; m.in = s->in; m.group = s->group; m.n_planes = np; m.nnz = s->nnz;
+  m.base = d + o_base;
+  for (int k = 0; k < 4; ++k) m.plane[k] = k < np ? d + o_plane[k] : nullptr;
+  m.pair = d + o_pair;
+  m.row_ptr = reinterpret_cast<const int32_t*>(d + o_rp);
+  m.entries = reinterpret_cast<const uint32_t*>(d + o_ent);
+  m.tables = reinterpret_cast<const float2*>(d + o_tab);
+  m.num_sms = prop.multiProcessorCount;
+  *out = h;
+  return STAGQ_OK;
+}
+
+extern "C" int stagq_load_file(const char* path, int device, stagq_handle* out) {
+  HostStreamBuffers buf;
+  int st = read_stream_file(path, &buf);
+  if (st) return st;
+  return stagq_load(&buf.view, device, out);
+}
+
+extern "C" int stagq_gemv_ex(stagq_handle h, int bits, const void* x, int n, void* y, uint32_t flags,
+                             void* cuda_stream) {
+  int st = check_handle_bits(h, bits);
+  if (st) return st;
+  if (!x || !y) return fail(STAGQ_EINVAL, "null x or y");
+  if (n < 1 || n > STAGQ_MAX_BATCH) return fail(STAGQ_EINVAL, "n outside 1..STAGQ_MAX_BATCH");
+  if (reinterpret_cast<uintptr_t>(x) % 16) return fail(STAGQ_EINVAL, "x must be 16-byte aligned");
+  if (flags & ~STAGQ_Y_F32) return fail(STAGQ_EINVAL, "unknown flags");
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return fail(STAGQ_ECUDA, "cudaSetDevice failed");
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  const int yf32 = (flags & STAGQ_Y_F32) ? 1 : 0;
+  const size_t ysz = yf32 ? 4 : 2;
+  for (int j = 0; j < n; ++j) {
+    const void* xj = static_cast<const uint8_t*>(x) + (size_t)j * h->dm.in * 2;
+    void* yj = static_cast<uint8_t*>(y) + (size_t)j * h->dm.out * ysz;
+    cudaError_t e = launch_gemv(h->dm, bits, xj, yj, yf32, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMV launch");
+  }
+  return STAGQ_OK;
+}
+
+extern "C" int stagq_gemv(stagq_handle h, int bits, const void* x, void* y, void* cuda_stream) {
+  return stagq_gemv_ex(h, bits, x, 1, y, 0u, cuda_stream);
+}
+
+extern "C" int stagq_gemv_n(stagq_handle h, int bits, const void* x, int n, void* y, void* cuda_stream) {
+  return stagq_gemv_ex(h, bits, x, n, y, 0u, cuda_stream);
+}
+
+extern "C" int stagq_gemv_host(stagq_handle h, int bits, const void* x_host, int n, void* y_host,
+                               void* cuda_stream) {
+  int st = check_handle_bits(h, bits);
+  if (st) return st;
+  if (!x_host || !y_host) return fail(STAGQ_EINVAL, "null x or y");
+  if (n < 1 || n > STAGQ_MAX_BATCH) return fail(STAGQ_EINVAL, "n outside 1..STAGQ_MAX_BATCH");
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return fail(STAGQ_ECUDA, "cudaSetDevice failed");
+  const size_t xb = (size_t)n * h->dm.in * 2, yb = (size_t)n * h->dm.out * 2;
+  const size_t need = align_up(xb, 256) + yb;
+  if (h->stage_bytes < need) {
+    if (h->d_stage) cudaFree(h->d_stage);
+    h->d_stage = nullptr;
+    h->stage_bytes = 0;
+    cudaError_t e = cudaMalloc(&h->d_stage, need);
+    if (e != cudaSuccess) { cudaGetLastError(); return fail(STAGQ_ENOMEM, "staging allocation failed"); }
+    h->stage_bytes = need;
+  }
+  uint8_t* dx = static_cast<uint8_t*>(h->d_stage);
+  uint8_t* dy = dx + align_up(xb, 256);
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t e = cudaMemcpyAsync(dx, x_host, xb, cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "copy of x");
+  st = stagq_gemv_ex(h, bits, dx, n, dy, 0u, cuda_stream);
+  if (st) return st;
+  e = cudaMemcpyAsync(y_host, dy, yb, cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "copy of y");
+  e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  return STAGQ_OK;
+}
+
+extern "C" int stagq_decode_levels(stagq_handle h, int bits, uint8_t* u_dev, void* cuda_stream) {
+  int st = check_handle_bits(h, bits);
+  if (st) return st;
+  if (!u_dev) return fail(STAGQ_EINVAL, "null output");
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return fail(STAGQ_ECUDA, "cudaSetDevice failed");
+  cudaError_t e = launch_decode_levels(h->dm, bits, u_dev, static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return STAGQ_OK;
+}
+
+extern "C" int64_t stagq_bytes(stagq_handle h, int bits, int n) {
+  if (!h || bits < 2 || bits > 2 + h->dm.n_planes || n < 1) return -1;
+  const int64_t out = h->dm.out, in = h->dm.in;
+  return out * in * bits / 8 + out * in / h->dm.group + 4 * h->dm.nnz + 4 * (out + 1) + 2 * (int64_t)n * in +
+         2 * (int64_t)n * out;
+}
+
+extern "C" int stagq_info(stagq_handle h, stagq_info_t* info) {
+  if (!h || !info) return fail(STAGQ_EINVAL, "null argument");
+  info->out = h->dm.out; info->in = h->dm.in; info->group = h->dm.group; info->n_planes = h->dm.n_planes;
+  info->nnz = h->dm.nnz; info->device = h->device;
+  info->device_bytes = (int64_t)(h->d_bytes + h->stage_bytes);
+  return STAGQ_OK;
+}
+
+extern "C" void stagq_free(stagq_handle h) {
+  if (!h) return;
+  DeviceGuard guard(h->device);
+  if (h->d_mem) cudaFree(h->d_mem);
+  if (h->d_stage) cudaFree(h->d_stage);
+  delete h;
+}

@@ -1,0 +1,131 @@
+"""Host side of libstagq.so (CPU only): exported symbols, encoder and packer
+against the oracle, the byte-scaling property of the layout, error paths."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import quantized_gemv_stagq_b200 as Q
+from oracle import stagq as O
+from quantized_gemv_stagq_b200 import synth
+from tests.helpers import fields_equal, to_lib_fields
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "stagq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(stagq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_function():
+    names = _declared_functions()
+    assert len(names) >= 18
+    L = Q.lib()
+    for n in names:
+        assert hasattr(L, n), f"libstagq.so does not export {n}"
+
+
+@pytest.mark.parametrize("out,inp,g,npl,dens,mode", [
+    (64, 512, 128, 2, 0.005, "search"),
+    (48, 256, 64, 4, 0.01, "search"),
+    (32, 256, 64, 0, 0.0, "search"),
+    (16, 256, 16, 2, 0.02, "search"),
+    (256, 1024, 128, 2, 0.005, "fast"),
+    (40, 384, 128, 3, 1.0, "search"),
+    (8, 128, 64, 1, 0.3, "fast"),
+])
+def test_encoder_matches_oracle_bit_exactly(out, inp, g, npl, dens, mode):
+    W = synth.weights(out, inp, seed=out * 7 + inp)
+    F = O.encode(W, group=g, n_planes=npl, density=dens, mode=mode)
+    P = Q.stagq_encode(W, group=g, n_planes=npl, density=dens, mode=mode, n_threads=3)
+    eq = fields_equal(F, P)
+    assert all(eq.values()), eq
+
+
+def test_encoder_handles_constant_and_zero_groups():
+    W = np.zeros((4, 256), np.float16)
+    W[1, :128] = np.float16(0.25)
+    W[2] = synth.weights(1, 256, seed=3)[0]
+    for mode in ("search", "fast"):
+        F = O.encode(W, group=128, n_planes=2, density=0.01, mode=mode)
+        P = Q.stagq_encode(W, group=128, n_planes=2, density=0.01, mode=mode)
+        eq = fields_equal(F, P)
+        assert all(eq.values()), (mode, eq)
+
+
+@pytest.mark.parametrize("npl,g", [(0, 64), (1, 128), (2, 128), (3, 64), (4, 64)])
+def test_packed_levels_reread_on_host_equal_oracle_levels(npl, g):
+    W = synth.weights(24, 640, seed=npl)
+    F = O.encode(W, group=g, n_planes=npl, density=0.01, mode="fast")
+    S = Q.stagq_pack(to_lib_fields(F))
+    assert S.planes.size == 24 * 640 * (2 + npl) // 8
+    for M in range(2, 3 + npl):
+        assert np.array_equal(Q.stagq_unpack_levels_host(S, M), O.decode_levels(F, M)), M
+
+
+def test_p_bit_read_touches_only_the_first_p_minus_2_planes():
+    """Section 3.3: a shallower read skips the deeper planes. Overwriting every
+    plane deeper than p leaves the p-bit read unchanged; overwriting plane p
+    changes it."""
+    W = synth.weights(16, 512, seed=5)
+    F = O.encode(W, group=128, n_planes=4, density=0.005, mode="fast")
+    S = Q.stagq_pack(to_lib_fields(F))
+    out, inp = 16, 512
+    rng = np.random.default_rng(0)
+    for p in range(2, 7):
+        ref = Q.stagq_unpack_levels_host(S, p)
+        end = out * inp // 4 + (p - 2) * (out * inp // 8)    # bytes a p-read may touch
+        T = Q.HostStream(**{**S.__dict__, "planes": S.planes.copy()})
+        T.planes[end:] = rng.integers(0, 256, T.planes.size - end, dtype=np.uint8)
+        assert np.array_equal(Q.stagq_unpack_levels_host(T, p), ref)
+        if p > 2:
+            T2 = Q.HostStream(**{**S.__dict__, "planes": S.planes.copy()})
+            T2.planes[end - out * inp // 8:end] ^= 0xFF
+            assert not np.array_equal(Q.stagq_unpack_levels_host(T2, p), ref)
+
+
+def test_plane_bytes_and_side_record_count():
+    assert Q.stagq_stream_plane_bytes(14336, 4096, 2) == 14336 * 4096 // 4 + 2 * 14336 * 4096 // 8
+    assert Q.stagq_side_record_count(14336, 4096, 0.005) == O.side_record_count(14336, 4096, 0.005) == 293601
+    assert Q.stagq_side_record_count(512, 512, 0.005) == 1311
+
+
+def _stream(out=8, inp=256, npl=2, dens=0.02):
+    W = synth.weights(out, inp, seed=1)
+    return Q.stagq_pack(Q.stagq_encode(W, group=128, n_planes=npl, density=dens, mode="fast"))
+
+
+def test_error_paths_return_status_codes():
+    W = synth.weights(8, 192, seed=1)
+    with pytest.raises(Q.StagqError) as e:   # in not a multiple of 128
+        Q.stagq_pack(Q.stagq_encode(W, group=64, n_planes=2, density=0.0, mode="fast"))
+    assert e.value.status == 1
+    S = _stream()
+    with pytest.raises(Q.StagqError) as e:
+        Q.stagq_unpack_levels_host(S, 5)          # bits > 2 + n_planes
+    assert e.value.status == 1
+    bad = Q.HostStream(**{**S.__dict__, "row_ptr": S.row_ptr.copy()})
+    bad.row_ptr[3] = bad.row_ptr[4] + 1           # not monotone
+    with pytest.raises(Q.StagqError) as e:
+        Q.stagq_load(bad, 0)
+    assert e.value.status == 2
+    bad = Q.HostStream(**{**S.__dict__, "col": S.col.copy()})
+    bad.col[0] = 256                              # col >= in
+    with pytest.raises(Q.StagqError) as e:
+        Q.stagq_save(bad, "/tmp/never_written.stagq")
+    assert e.value.status == 2
+    with pytest.raises(Q.StagqError) as e:
+        Q.stagq_save(S, "/nonexistent_dir/x.stagq")
+    assert e.value.status == 5
+
+
+def test_stream_file_header(tmp_path):
+    S = _stream()
+    p = str(tmp_path / "m.stagq")
+    Q.stagq_save(S, p)
+    raw = open(p, "rb").read()
+    assert raw[:8] == b"STAGQS1\0"
+    assert len(raw) == 8 + 4 * 4 + 8 + 64 + S.planes.size + S.pair_idx.size + 4 * (S.out + 1) + 4 * S.nnz

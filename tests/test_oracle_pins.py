@@ -100,7 +100,7 @@ def test_initial_pair_matches_appendix_b_constants():
     """Appendix B: four symmetric levels, outer two 6 % in from each end, a step
     of 0.29 of the group range."""
     V = np.array([[0.0, 0.3, 0.7, 1.0] * 2])
-    lo0, s0 = O.initial_pairs(V, 8)
+    lo0, s0, flat = O.initial_pairs(V, 8)
     R = 1.0
     assert math.isclose(lo0[0, 0], 0.06 * R)
     assert math.isclose(lo0[0, 0] + 3 * s0[0, 0], R - 0.06 * R)
@@ -314,7 +314,7 @@ def test_codebooks_are_uniform_over_initial_pair_range():
     F = O.encode(W, group=128, n_planes=2, density=0.005, mode="fast")
     m = O.select_side_record(W, 0.005)
     Vc, empty = O.clip_held_out(W, m, 128)
-    lo0, s0 = O.initial_pairs(Vc, 128)
+    lo0, s0, flat = O.initial_pairs(Vc, 128)
     ls = np.log2(s0)
     assert F.cb_log2s[0] == np.float16(ls.min()) and F.cb_log2s[-1] == np.float16(ls.max())
     exact = ls.min() + np.arange(16) * (ls.max() - ls.min()) / 15
