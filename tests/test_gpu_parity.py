@@ -1,0 +1,182 @@
+"""GPU parity of the StagQ GEMV against the CPU oracle (needs a B200).
+
+Small cases: the GPU reads a stream packed from the ORACLE's fields, and y is
+compared element by element with the oracle's fp64 GEMV. Full Llama-3.1-8B
+shapes: the library encoder feeds the GPU (as in bench.py), the oracle encodes
+the same weights independently, and sampled rows are compared (fields and y).
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import quantized_gemv_stagq_b200 as Q
+from oracle import stagq as O
+from quantized_gemv_stagq_b200 import synth
+from tests.helpers import check_close, fields_equal, to_lib_fields
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _needs_cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    Q.lib()
+
+
+def _load(F):
+    return Q.stagq_load(Q.stagq_pack(to_lib_fields(F)), 0)
+
+
+def _gemv(m, bits, x_np, f32=True):
+    x = torch.from_numpy(np.ascontiguousarray(x_np)).cuda()
+    n = x.shape[0]
+    y = torch.empty(n, m.out, dtype=torch.float32 if f32 else torch.float16, device="cuda")
+    Q.stagq_gemv_ex(m, bits, x, y, n=n, flags=Q.STAGQ_Y_F32 if f32 else 0)
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+SMALL = [
+    # out, in, group, n_planes, density, pair mode, seed
+    (512, 512, 128, 2, 0.005, "search", 1),     # the tiny workload
+    (96, 2048, 64, 4, 0.01, "fast", 2),         # deep stream, p2..p6
+    (37, 640, 128, 2, 0.005, "fast", 3),        # fewer rows than SMs; ragged K (10 chunks)
+    (300, 5120, 128, 2, 0.001, "fast", 4),      # K = 2.5 warp tiles
+    (1, 4096, 128, 2, 0.01, "fast", 5),         # a single row
+    (160, 1024, 64, 3, 0.0, "fast", 6),         # no side record
+    (64, 768, 128, 2, 1.0, "fast", 7),          # everything held out
+    (200, 4096, 128, 1, 0.02, "fast", 8),       # one plane
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}x{c[1]}g{c[2]}p{c[3]}d{c[4]}")
+def test_decoded_levels_bit_exact(case):
+    out, inp, g, npl, dens, mode, seed = case
+    F = O.encode(synth.weights(out, inp, seed), g, npl, dens, mode)
+    m = _load(F)
+    u = torch.empty(out, inp, dtype=torch.uint8, device="cuda")
+    for M in range(2, 3 + npl):
+        Q.stagq_decode_levels(m, M, u)
+        torch.cuda.synchronize()
+        assert np.array_equal(u.cpu().numpy(), O.decode_levels(F, M)), f"p{M}"
+    m.free()
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}x{c[1]}g{c[2]}p{c[3]}d{c[4]}")
+def test_gemv_matches_oracle(case):
+    out, inp, g, npl, dens, mode, seed = case
+    F = O.encode(synth.weights(out, inp, seed), g, npl, dens, mode)
+    m = _load(F)
+    x = synth.activations(1, inp, seed + 100)
+    for M in range(2, 3 + npl):
+        ref = O.gemv(F, M, x)
+        check_close(_gemv(m, M, x, f32=True), ref, f"fp32 y p{M}")
+        check_close(_gemv(m, M, x, f32=False).astype(np.float64), ref, f"fp16 y p{M}")
+    m.free()
+
+
+def test_gemv_activation_edge_cases():
+    out, inp = 256, 2048
+    F = O.encode(synth.weights(out, inp, 11), 128, 2, 0.005, "fast")
+    m = _load(F)
+    rng = np.random.default_rng(0)
+    xs = {
+        "zeros": np.zeros((1, inp), np.float16),
+        "one_hot": np.eye(1, inp, 1234, dtype=np.float16),
+        "large": (rng.standard_normal((1, inp)) * 300).astype(np.float16),
+        "tiny": (rng.standard_normal((1, inp)) * 1e-4).astype(np.float16),
+        "mixed_scale": np.concatenate([rng.standard_normal(inp // 2) * 1e3,
+                                       rng.standard_normal(inp // 2) * 1e-3]).astype(np.float16)[None],
+    }
+    for name, x in xs.items():
+        for M in (2, 3, 4):
+            y = _gemv(m, M, x)
+            ref = O.gemv(F, M, x)
+            if name == "zeros":
+                assert not np.any(y), name
+            else:
+                check_close(y, ref, f"{name} p{M}")
+    m.free()
+
+
+def test_gemv_is_deterministic_and_reentrant():
+    F = O.encode(synth.weights(1024, 4096, 21), 128, 2, 0.005, "fast")
+    m = _load(F)
+    x = torch.from_numpy(synth.activations(1, 4096, 22)).cuda()
+    ys = []
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    for st in (s1, s2, s1):
+        y = torch.empty(1, 1024, dtype=torch.float32, device="cuda")
+        with torch.cuda.stream(st):
+            Q.stagq_gemv_ex(m, 3, x, y, flags=Q.STAGQ_Y_F32, stream=st)
+        ys.append(y)
+    torch.cuda.synchronize()
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
+    m.free()
+
+
+def test_host_buffer_call_and_file_round_trip(tmp_path):
+    F = O.encode(synth.weights(384, 1024, 31), 128, 2, 0.005, "fast")
+    S = Q.stagq_pack(to_lib_fields(F))
+    m = Q.stagq_load(S, 0)
+    path = str(tmp_path / "w.stagq")
+    Q.stagq_save(S, path)
+    mf = Q.stagq_load_file(path, 0)
+    x = synth.activations(1, 1024, 32)
+    for M in (2, 3, 4):
+        y_dev = _gemv(m, M, x, f32=False)
+        y_file = _gemv(mf, M, x, f32=False)
+        y_host = np.empty((1, 384), np.float16)
+        Q.stagq_gemv_host(m, M, x, y_host)
+        assert np.array_equal(y_dev.view(np.uint16), y_file.view(np.uint16))
+        assert np.array_equal(y_dev.view(np.uint16), y_host.view(np.uint16))
+        assert Q.stagq_bytes(m, M) == O.model_bytes(384, 1024, 128, F.nnz, M)
+    m.free()
+    mf.free()
+
+
+def test_bad_calls_return_errors():
+    F = O.encode(synth.weights(64, 512, 41), 128, 2, 0.005, "fast")
+    m = _load(F)
+    x = torch.zeros(1, 512, dtype=torch.float16, device="cuda")
+    y = torch.zeros(1, 64, dtype=torch.float16, device="cuda")
+    for bits in (1, 5, 7):
+        with pytest.raises(Q.StagqError) as e:
+            Q.stagq_gemv(m, bits, x, y)
+        assert e.value.status == 1
+    with pytest.raises(Q.StagqError):
+        Q.stagq_gemv_n(m, 2, x, 0, y)
+    with pytest.raises(Q.StagqError):
+        Q.stagq_gemv_ex(m, 2, x, y, flags=8)
+    m.free()
+
+
+LLAMA = list(synth.LLAMA31_8B_LINEARS.items())
+SAMPLE_ROWS = 48
+
+
+@pytest.mark.parametrize("name,shape", [(n, s) for n, s in LLAMA if n in ("q_proj", "k_proj", "gate_proj", "down_proj")])
+def test_full_size_llama_sampled_rows(name, shape):
+    """The bench's workload and launch: library encoder -> GPU; oracle encodes
+    the same weights itself; fields and y agree on sampled rows."""
+    out, inp = shape
+    W = synth.weights(out, inp, seed=1000 + out + inp)
+    P = Q.stagq_encode(W, 128, 2, 0.005, "fast")
+    m = Q.stagq_load(Q.stagq_pack(P), 0)
+    rng = np.random.default_rng(out)
+    rows = np.unique(np.concatenate([[0, out - 1], rng.choice(out, SAMPLE_ROWS, replace=False)]))
+    F = O.encode(W, 128, 2, 0.005, "fast", rows=rows)
+    Psub = Q.Fields(F.out, inp, 128, 2, P.q[rows], P.planes[:, rows], P.pair_idx[rows],
+                    P.cb_log2s, P.cb_lo_over_s,
+                    np.concatenate([[0], np.cumsum(np.diff(P.row_ptr)[rows])]).astype(np.int32),
+                    np.concatenate([P.col[P.row_ptr[r]:P.row_ptr[r + 1]] for r in rows]),
+                    np.concatenate([P.val[P.row_ptr[r]:P.row_ptr[r + 1]] for r in rows]))
+    eq = fields_equal(F, Psub)
+    assert all(eq.values()), eq
+    x = synth.activations(1, inp, seed=7)
+    for M in (2, 3, 4):
+        y = _gemv(m, M, x, f32=False)[0]
+        check_close(y[rows].astype(np.float64), O.gemv(F, M, x)[0], f"{name} p{M}")
+        assert np.all(np.isfinite(y))
+    m.free()
