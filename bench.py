@@ -1,0 +1,376 @@
+"""StagQ batch-one GEMV benchmark on B200.
+
+Workload (one step): the seven linears of one Llama-3.1-8B layer (q/k/v/o,
+gate/up, down; out x in as in the model), synthetic weights, group 128, base +
+2 refinement planes, 0.5 % side record, x fp16 N(0,1), batch 1, each GEMV run
+at 2, 3 and 4 bits -- 21 GEMVs per step. Every step is one CUDA-graph replay;
+steps rotate over several device copies of the layer so every read comes from
+HBM (copies x bytes >> L2).
+
+Prints one JSON line. ``value`` is the whole job's algorithmic HBM traffic
+(planes read at the chosen precision + pairs + side record + x + y) divided by
+device time, in GB/s. Per-GEMV microseconds for every shape and precision are
+in ``per_gemv``.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl stagq|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "batch-1 GEMV µs and achieved HBM GB/s (% of roofline) at 2/3/4 bits"
+WORKLOAD = "llama31_8b_linears_b1"
+BITS = (2, 3, 4)
+GROUP, N_PLANES, DENSITY = 128, 2, 0.005
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["quantized_gemv_stagq_b200/csrc/gemv.cu", "quantized_gemv_stagq_b200/csrc/layout.cuh"]
+
+
+def _args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="stagq", choices=["stagq", "reference"])
+    p.add_argument("--copies", type=int, default=6, help="device copies of the layer rotated over")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _kernel_hash():
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _ncu_traffic():
+    """dram bytes per launch of the dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "gemv_dram_traffic.txt")
+    try:
+        kv = {}
+        for line in open(path):
+            if line.strip() and not line.startswith("#") and " " in line:
+                k, v = line.split(None, 1)
+                kv[k] = v.strip()
+        if kv.get("kernel_source_sha256_16") != _kernel_hash():
+            return None, None
+        return float(kv["dram_bytes_per_launch_full"]), kv.get("kernel", "")
+    except Exception:
+        return None, None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [t.strip() for t in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+def _layer_shapes():
+    from quantized_gemv_stagq_b200 import synth
+    return list(synth.LLAMA31_8B_LINEARS.items())
+
+
+# ------------------------------------------------------------------ reference arm
+
+class OracleSample:
+    """The oracle's GEMV (decode + fp64 dot) of the q_proj shape at 2/3/4 bits:
+    the CPU statement of one precision sweep of the hot path."""
+
+    def __init__(self):
+        from oracle import stagq as O
+        from quantized_gemv_stagq_b200 import synth
+        self.O = O
+        self.out, self.inp = synth.LLAMA31_8B_LINEARS["q_proj"]
+        W = synth.weights(self.out, self.inp, seed=11)
+        self.F = O.encode(W, GROUP, N_PLANES, DENSITY, "fast")
+        self.x = synth.activations(1, self.inp, seed=12)
+        try:
+            from threadpoolctl import threadpool_info
+            self.threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        except Exception:
+            self.threads = os.cpu_count() or 1
+
+    def one(self, b):
+        """One GEMV at b bits; returns (bytes, seconds)."""
+        t0 = time.perf_counter()
+        self.O.gemv(self.F, b, self.x)
+        return self.O.model_bytes(self.out, self.inp, GROUP, self.F.nnz, b), time.perf_counter() - t0
+
+    def text(self, n):
+        return (f"oracle GEMV (decode + fp64 dot) of q_proj {self.out}x{self.inp}, {n} call(s) cycling "
+                f"p2/p3/p4")
+
+
+def cpu_oracle_sample(target_s: float = 12.0):
+    """Bounded CPU baseline: rounds of OracleSample until ~target_s."""
+    S = OracleSample()
+    nb, el, n = 0, 0.0, 0
+    while el < target_s or n % len(BITS):
+        b, t = S.one(BITS[n % len(BITS)])
+        nb, el, n = nb + b, el + t, n + 1
+    return nb / el / 1e9, el, S.text(n), S.threads
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    S = OracleSample()
+    for w in range(args.warmup):
+        S.one(BITS[w % len(BITS)])
+    nb, el = 0, 0.0
+    for k in range(args.steps):       # a step: one oracle GEMV, precisions cycling
+        b, t = S.one(BITS[k % len(BITS)])
+        nb, el = nb + b, el + t
+    value = nb / el / 1e9
+    sample = S.text(args.steps)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * el / max(args.steps, 1), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "sample": sample, "group": GROUP,
+                                        "n_planes": N_PLANES, "side_record_density": DENSITY, "batch": 1},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": S.threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_stagq(args):
+    import torch
+    import quantized_gemv_stagq_b200 as Q
+    from quantized_gemv_stagq_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = local
+
+    # ---- encode one layer (library encoder, fast pair rule), load C copies
+    shapes = _layer_shapes()
+    streams = []
+    for li, (name, (out, inp)) in enumerate(shapes):
+        W = synth.weights(out, inp, seed=100 + li)
+        P = Q.stagq_encode(W, GROUP, N_PLANES, DENSITY, "fast")
+        streams.append((name, out, inp, Q.stagq_pack(P), P.nnz))
+        del W, P
+    C = max(2, args.copies)
+    mats = [[Q.stagq_load(s, dev) for (_, _, _, s, _) in streams] for _ in range(C)]
+    xs = [torch.from_numpy(synth.activations(1, inp, seed=200 + i)).cuda() for i, (_, _, inp, _, _) in enumerate(streams)]
+    ys = [torch.empty(1, out, dtype=torch.float16, device="cuda") for (_, out, _, _, _) in streams]
+    step_bytes = sum(Q.stagq_bytes(mats[0][i], b, 1) for b in BITS for i in range(len(streams)))
+    stored = sum(m.device_bytes for m in mats[0])
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+
+    stream = torch.cuda.Stream()
+
+    def step_launches(c):
+        for b in BITS:
+            for i in range(len(streams)):
+                Q.stagq_gemv(mats[c][i], b, xs[i], ys[i], stream=stream)
+
+    # ---- one CUDA graph per copy
+    graphs = []
+    with torch.cuda.stream(stream):
+        step_launches(0)  # warm the launch path outside capture
+    torch.cuda.synchronize()
+    for c in range(C):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step_launches(c)
+        graphs.append(g)
+    torch.cuda.synchronize()
+
+    for w in range(max(args.warmup, 3)):
+        graphs[w % C].replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for s in range(args.steps):
+            graphs[s % C].replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+
+    # ---- per-GEMV timing (same kernels, one shape/precision at a time)
+    per = {}
+    reps = 4 * C
+    with torch.cuda.stream(stream):
+        for b in BITS:
+            for i, (name, out, inp, _, nnz) in enumerate(streams):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for r in range(reps):
+                        Q.stagq_gemv(mats[(r + 1) % C][i], b, xs[i], ys[i], stream=stream)
+                g.replay()
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a0.record(stream)
+                for _ in range(5):
+                    g.replay()
+                a1.record(stream)
+                torch.cuda.synchronize()
+                us = a0.elapsed_time(a1) * 1e3 / (5 * reps)
+                nb = Q.stagq_bytes(mats[0][i], b, 1)
+                per.setdefault(f"p{b}", {})[name] = {"us": round(us, 3), "bytes": nb, "gbs": round(nb / us / 1e3, 1)}
+                del g
+    clk = clocks.stop()
+
+    if dist:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+
+    # ---- end to end through the C ABI with host buffers
+    e2e_steps = max(2, min(args.steps, 10))
+    xh = [x.cpu().pin_memory().numpy() for x in xs]
+    yh = [torch.empty((1, out), dtype=torch.float16).pin_memory().numpy() for (_, out, _, _, _) in streams]
+    for i in range(len(streams)):
+        Q.stagq_gemv_host(mats[0][i], 2, xh[i], yh[i], stream=stream)
+    h2d = sum(2 * inp for b in BITS for (_, _, inp, _, _) in streams)
+    d2h = sum(2 * out for b in BITS for (_, out, _, _, _) in streams)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for s in range(e2e_steps):
+        for b in BITS:
+            for i in range(len(streams)):
+                Q.stagq_gemv_host(mats[s % C][i], b, xh[i], yh[i], stream=stream)
+    e2e_s = time.perf_counter() - t0
+    e2e_gbs = step_bytes * e2e_steps / e2e_s / 1e9
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak, peak_kind = _peaks()
+    value = world * step_bytes * args.steps / (ms * 1e-3) / 1e9
+    # dominant kernel: the (shape, precision) with the largest share of a step
+    dom_key, dom = max(((f"{name}@{pb}", d) for pb, dd in per.items() for name, d in dd.items()),
+                       key=lambda kv: kv[1]["us"])
+    traffic, _ = _ncu_traffic()
+    cpu = None
+    if not args.no_cpu_baseline:
+        v, s, sample, threads = cpu_oracle_sample()
+        cpu = {"value": round(v, 4), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample}
+    step_us = {pb: round(sum(d["us"] for d in dd.values()), 2) for pb, dd in per.items()}
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int32 dot (u8 codes x i16 x) + fp32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "linears_out_x_in": {n: [o, i] for n, (o, i) in shapes}, "bits": list(BITS),
+                   "group": GROUP, "n_planes": N_PLANES, "side_record_density": DENSITY, "batch": 1,
+                   "pair_rule": "fast", "gemvs_per_step": len(BITS) * len(shapes),
+                   "l2": f"inputs larger than L2: {C} rotating device copies x {stored / 1e6:.0f} MB stored, "
+                         f"{step_bytes / 1e6:.0f} MB read per step vs L2 {l2 / 1e6:.0f} MB",
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "frac_of_hbm": round(value / world / peak, 4),
+        "per_gemv": per, "us_per_precision_layer": step_us,
+        "roofline": {"bound": "hbm", "kernel": f"gemv_kernel {dom_key}", "achieved": dom["gbs"], "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dom["gbs"] / peak, 4),
+                     "traffic": traffic, "algorithmic_bytes": dom["bytes"]},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "api": "stagq_gemv_host (host x/y, copies + sync per call)"},
+        "gpu_launches": len(BITS) * len(shapes) * args.steps,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_stagq(args)
+
+
+if __name__ == "__main__":
+    main()

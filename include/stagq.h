@@ -41,6 +41,7 @@ extern "C" {
 #define STAGQ_ECUDA 4    /* a CUDA runtime call failed (detail in stagq_last_error) */
 #define STAGQ_EIO 5      /* file could not be read or written */
 #define STAGQ_ENODEV 6   /* no usable sm_100 device */
+#define STAGQ_ETIMEOUT 7 /* a kernel gave up waiting for its own data (reported by stagq_check) */
 
 /* Limits of this implementation. */
 #define STAGQ_MAX_PLANES 4      /* stream depth N = 2 + n_planes <= 6 (the paper evaluates N = 6) */
@@ -173,7 +174,8 @@ int stagq_load(const stagq_host_stream* s, int device, stagq_handle* out);
  *   bits   2 .. 2 + n_planes
  *   x      device [in]  fp16
  *   y      device [out] fp16 (fp32 accumulation, rounded to nearest even)
- * Calls on one handle may run concurrently: the GEMV uses no scratch memory.
+ * Calls on one handle may run concurrently: the GEMV uses no scratch memory
+ * (each CTA stages its rows in its own shared memory).
  * Errors: STAGQ_EINVAL (null handle/pointer, bits out of range), STAGQ_ECUDA (launch failure).
  */
 int stagq_gemv(stagq_handle h, int bits, const void* x, void* y, void* cuda_stream);
@@ -205,6 +207,15 @@ int stagq_decode_levels(stagq_handle h, int bits, uint8_t* u_dev, void* cuda_str
  * Returns -1 for a bad handle or bits.
  */
 int64_t stagq_bytes(stagq_handle h, int bits, int n);
+
+/*
+ * Synchronise the handle's device and report whether any GEMV on this handle
+ * gave up waiting for its data since the last check (every wait inside the
+ * kernels is bounded to about 2 s; on expiry the kernel records it in a status
+ * word and returns, leaving y undefined). Clears the status. Returns STAGQ_OK
+ * or STAGQ_ETIMEOUT (or STAGQ_ECUDA if the device reports an error).
+ */
+int stagq_check(stagq_handle h);
 
 int stagq_info(stagq_handle h, stagq_info_t* info);
 

@@ -62,6 +62,7 @@ _SIGNATURES = {
     "stagq_decode_levels": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, _c_p]),
     "stagq_bytes": (_i64, [_c_p, ctypes.c_int, ctypes.c_int]),
     "stagq_info": (ctypes.c_int, [_c_p, ctypes.POINTER(_Info)]),
+    "stagq_check": (ctypes.c_int, [_c_p]),
     "stagq_free": (None, [_c_p]),
     "stagq_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "stagq_last_error": (ctypes.c_char_p, []),
@@ -294,6 +295,11 @@ def stagq_decode_levels(m: Matrix, bits: int, u_dev, stream=None) -> None:
 
 def stagq_bytes(m: Matrix, bits: int, n: int = 1) -> int:
     return int(lib().stagq_bytes(m.handle, bits, n))
+
+
+def stagq_check(m: Matrix) -> None:
+    """Synchronise and raise if a kernel on this handle gave up on a wait."""
+    _check(lib().stagq_check(m.handle), "stagq_check")
 
 
 def stagq_free(m: Matrix) -> None:

@@ -16,6 +16,8 @@
 struct stagq_matrix {
   int device = -1;
   stagq::DeviceMatrix dm{};
+  stagq::GemvPlan plan[7]{};     // per precision (index = bits)
+  bool plan_ok[7]{};
   void* d_mem = nullptr;
   size_t d_bytes = 0;
   void* d_stage = nullptr;      // x / y staging for stagq_gemv_host
@@ -89,7 +91,8 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   const int64_t out_ = s->out, in = s->in;
   const int np = s->n_planes;
   const size_t base_bytes = (size_t)(out_ * in / 4), plane_bytes = (size_t)(out_ * in / 8);
-  const size_t pair_bytes = (size_t)(out_ * (in / s->group));
+  const size_t pair_row = (size_t)(in / s->group), pair_stride = align_up(pair_row, 16);
+  const size_t pair_bytes = (size_t)out_ * pair_stride;
   const size_t rp_bytes = (size_t)(out_ + 1) * 4, ent_bytes = (size_t)s->nnz * 4;
   const size_t tab_bytes = (size_t)(np + 1) * 256 * sizeof(float2);
   size_t off = 0;
@@ -100,6 +103,7 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   const size_t o_rp = off; off = align_up(off + rp_bytes, 256);
   const size_t o_ent = off; off = align_up(off + (ent_bytes ? ent_bytes : 4), 256);
   const size_t o_tab = off; off = align_up(off + tab_bytes, 256);
+  const size_t o_status = off; off = align_up(off + 4, 256);
   const size_t total = off;
 
   stagq_matrix* h = new (std::nothrow) stagq_matrix();
@@ -118,11 +122,13 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   for (int64_t i = 0; i < s->nnz; ++i) ent[i] = (uint32_t)s->col[i] | ((uint32_t)s->val[i] << 16);
   std::vector<float2> tabs;
   build_tables(s, tabs);
+  std::vector<uint8_t> pairs(pair_bytes, 0);
+  for (int64_t r = 0; r < out_; ++r) std::memcpy(&pairs[(size_t)r * pair_stride], s->pair_idx + (size_t)r * pair_row, pair_row);
 
   struct Copy { size_t off; const void* src; size_t n; };
   std::vector<Copy> copies = {{o_base, s->planes, base_bytes}};
   for (int k = 0; k < np; ++k) copies.push_back({o_plane[k], s->planes + base_bytes + (size_t)k * plane_bytes, plane_bytes});
-  copies.push_back({o_pair, s->pair_idx, pair_bytes});
+  copies.push_back({o_pair, pairs.data(), pair_bytes});
   copies.push_back({o_rp, s->row_ptr, rp_bytes});
   if (ent_bytes) copies.push_back({o_ent, ent.data(), ent_bytes});
   copies.push_back({o_tab, tabs.data(), tab_bytes});
@@ -134,15 +140,52 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
       return cuda_fail(e, "cudaMemcpy of stream");
     }
   }
+  e = cudaMemset(d + o_status, 0, 4);
+  if (e != cudaSuccess) {
+    cudaFree(h->d_mem);
+    delete h;
+    return cuda_fail(e, "cudaMemset of status");
+  }
+  int smem_limit = 0;
+  e = cudaDeviceGetAttribute(&smem_limit, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+  if (e != cudaSuccess) {
+    cudaFree(h->d_mem);
+    delete h;
+    return cuda_fail(e, "cudaDeviceGetAttribute");
+  }
   DeviceMatrix& m = h->dm;
   m.out = s->out; m.in = s->in; m.group = s->group; m.n_planes = np; m.nnz = s->nnz;
   m.base = d + o_base;
   for (int k = 0; k < 4; ++k) m.plane[k] = k < np ? d + o_plane[k] : nullptr;
   m.pair = d + o_pair;
+  m.pair_stride = (int32_t)pair_stride;
+  m.status = reinterpret_cast<uint32_t*>(d + o_status);
+  m.smem_limit = smem_limit;
   m.row_ptr = reinterpret_cast<const int32_t*>(d + o_rp);
   m.entries = reinterpret_cast<const uint32_t*>(d + o_ent);
   m.tables = reinterpret_cast<const float2*>(d + o_tab);
   m.num_sms = prop.multiProcessorCount;
+  // entries per stage of the row partition every precision uses
+  {
+    int grid = 0, rs = 0;
+    stage_partition(s->out, s->in, m.num_sms, &grid, &rs);
+    int64_t most = 0;
+    for (int b = 0; b < grid; ++b) {
+      const int64_t ra = (int64_t)b * s->out / grid, rb = (int64_t)(b + 1) * s->out / grid;
+      for (int64_t q = ra; q < rb; q += rs) {
+        const int64_t qe = q + rs < rb ? q + rs : rb;
+        const int64_t cnt = (int64_t)s->row_ptr[qe] - s->row_ptr[q];
+        if (cnt > most) most = cnt;
+      }
+    }
+    m.ecap = (int)(most < kMaxEntryCap ? most : kMaxEntryCap);
+  }
+  for (int b = 2; b <= 2 + np; ++b) h->plan_ok[b] = make_plan(m, b, &h->plan[b]);
+  if (!h->plan_ok[2]) {
+    cudaFree(h->d_mem);
+    delete h;
+    return fail(STAGQ_EINVAL, "shape cannot be planned on this device");
+  }
   *out = h;
   return STAGQ_OK;
 }
@@ -167,10 +210,11 @@ extern "C" int stagq_gemv_ex(stagq_handle h, int bits, const void* x, int n, voi
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   const int yf32 = (flags & STAGQ_Y_F32) ? 1 : 0;
   const size_t ysz = yf32 ? 4 : 2;
+  if (!h->plan_ok[bits]) return fail(STAGQ_EINVAL, "no launch plan for this precision");
   for (int j = 0; j < n; ++j) {
     const void* xj = static_cast<const uint8_t*>(x) + (size_t)j * h->dm.in * 2;
     void* yj = static_cast<uint8_t*>(y) + (size_t)j * h->dm.out * ysz;
-    cudaError_t e = launch_gemv(h->dm, bits, xj, yj, yf32, stream);
+    cudaError_t e = launch_gemv(h->dm, h->plan[bits], bits, xj, yj, yf32, stream);
     if (e != cudaSuccess) return cuda_fail(e, "GEMV launch");
   }
   return STAGQ_OK;
@@ -232,6 +276,20 @@ extern "C" int64_t stagq_bytes(stagq_handle h, int bits, int n) {
   const int64_t out = h->dm.out, in = h->dm.in;
   return out * in * bits / 8 + out * in / h->dm.group + 4 * h->dm.nnz + 4 * (out + 1) + 2 * (int64_t)n * in +
          2 * (int64_t)n * out;
+}
+
+extern "C" int stagq_check(stagq_handle h) {
+  if (!h) return fail(STAGQ_EINVAL, "null handle");
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return fail(STAGQ_ECUDA, "cudaSetDevice failed");
+  uint32_t word = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  e = cudaMemcpy(&word, h->dm.status, 4, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (!word) return STAGQ_OK;
+  cudaMemset(h->dm.status, 0, 4);
+  return fail(STAGQ_ETIMEOUT, "a GEMV kernel gave up waiting for its data (status " + std::to_string(word) + ")");
 }
 
 extern "C" int stagq_info(stagq_handle h, stagq_info_t* info) {

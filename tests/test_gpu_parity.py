@@ -47,6 +47,8 @@ SMALL = [
     (160, 1024, 64, 3, 0.0, "fast", 6),         # no side record
     (64, 768, 128, 2, 1.0, "fast", 7),          # everything held out
     (200, 4096, 128, 1, 0.02, "fast", 8),       # one plane
+    (296, 4096, 128, 2, 0.6, "fast", 9),        # > 2048 record entries per stage (overflow path)
+    (300, 32768, 128, 4, 0.005, "fast", 10),    # widest K: 16 K-warps, one-row stages at p6
 ]
 
 
@@ -73,6 +75,7 @@ def test_gemv_matches_oracle(case):
         ref = O.gemv(F, M, x)
         check_close(_gemv(m, M, x, f32=True), ref, f"fp32 y p{M}")
         check_close(_gemv(m, M, x, f32=False).astype(np.float64), ref, f"fp16 y p{M}")
+    Q.stagq_check(m)
     m.free()
 
 
@@ -179,4 +182,5 @@ def test_full_size_llama_sampled_rows(name, shape):
         y = _gemv(m, M, x, f32=False)[0]
         check_close(y[rows].astype(np.float64), O.gemv(F, M, x)[0], f"{name} p{M}")
         assert np.all(np.isfinite(y))
+    Q.stagq_check(m)
     m.free()
