@@ -41,13 +41,13 @@ extern "C" {
 #define STAGQ_ECUDA 4    /* a CUDA runtime call failed (detail in stagq_last_error) */
 #define STAGQ_EIO 5      /* file could not be read or written */
 #define STAGQ_ENODEV 6   /* no usable sm_100 device */
-#define STAGQ_ETIMEOUT 7 /* a kernel gave up waiting for its own data (reported by stagq_check) */
 
 /* Limits of this implementation. */
 #define STAGQ_MAX_PLANES 4      /* stream depth N = 2 + n_planes <= 6 (the paper evaluates N = 6) */
 #define STAGQ_MAX_BATCH 4       /* columns of x per call in stagq_gemv_n */
 #define STAGQ_MAX_IN 32768      /* K; side-record columns are stored as uint16 */
 #define STAGQ_IN_MULTIPLE 128   /* K must be a multiple of this (16-byte plane rows) */
+/* The group size of a loadable stream is a power of two, at least 64, dividing K. */
 
 /* Pair search mode of the encoder (Section 3.1). */
 #define STAGQ_PAIR_SEARCH 0     /* argmin of Eq. (5) over all 256 codebook pairs */
@@ -209,11 +209,9 @@ int stagq_decode_levels(stagq_handle h, int bits, uint8_t* u_dev, void* cuda_str
 int64_t stagq_bytes(stagq_handle h, int bits, int n);
 
 /*
- * Synchronise the handle's device and report whether any GEMV on this handle
- * gave up waiting for its data since the last check (every wait inside the
- * kernels is bounded to about 2 s; on expiry the kernel records it in a status
- * word and returns, leaving y undefined). Clears the status. Returns STAGQ_OK
- * or STAGQ_ETIMEOUT (or STAGQ_ECUDA if the device reports an error).
+ * Synchronise the handle's device and report any CUDA error raised by work
+ * queued on it (the GEMV entry points are asynchronous and only report launch
+ * errors). Returns STAGQ_OK or STAGQ_ECUDA.
  */
 int stagq_check(stagq_handle h);
 

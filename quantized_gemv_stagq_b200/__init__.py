@@ -298,7 +298,7 @@ def stagq_bytes(m: Matrix, bits: int, n: int = 1) -> int:
 
 
 def stagq_check(m: Matrix) -> None:
-    """Synchronise and raise if a kernel on this handle gave up on a wait."""
+    """Synchronise the handle's device and raise on any pending CUDA error."""
     _check(lib().stagq_check(m.handle), "stagq_check")
 
 

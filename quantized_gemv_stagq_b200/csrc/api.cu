@@ -101,9 +101,8 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   for (int k = 0; k < np; ++k) { o_plane[k] = off; off = align_up(off + plane_bytes, 256); }
   const size_t o_pair = off; off = align_up(off + pair_bytes, 256);
   const size_t o_rp = off; off = align_up(off + rp_bytes, 256);
-  const size_t o_ent = off; off = align_up(off + (ent_bytes ? ent_bytes : 4), 256);
+  const size_t o_ent = off; off = align_up(off + ent_bytes + 16, 256);  // +16: 16-byte staged reads
   const size_t o_tab = off; off = align_up(off + tab_bytes, 256);
-  const size_t o_status = off; off = align_up(off + 4, 256);
   const size_t total = off;
 
   stagq_matrix* h = new (std::nothrow) stagq_matrix();
@@ -122,6 +121,16 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   for (int64_t i = 0; i < s->nnz; ++i) ent[i] = (uint32_t)s->col[i] | ((uint32_t)s->val[i] << 16);
   std::vector<float2> tabs;
   build_tables(s, tabs);
+  // most side-record entries in one CTA's row range
+  int32_t max_cta = 0;
+  {
+    const int grid = gemv_grid(s->out, prop.multiProcessorCount);
+    for (int b = 0; b < grid; ++b) {
+      const int64_t ra = (int64_t)b * s->out / grid, rb = (int64_t)(b + 1) * s->out / grid;
+      const int64_t n = (int64_t)s->row_ptr[rb] - s->row_ptr[ra];
+      if (n > max_cta) max_cta = (int32_t)n;
+    }
+  }
   std::vector<uint8_t> pairs(pair_bytes, 0);
   for (int64_t r = 0; r < out_; ++r) std::memcpy(&pairs[(size_t)r * pair_stride], s->pair_idx + (size_t)r * pair_row, pair_row);
 
@@ -140,12 +149,6 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
       return cuda_fail(e, "cudaMemcpy of stream");
     }
   }
-  e = cudaMemset(d + o_status, 0, 4);
-  if (e != cudaSuccess) {
-    cudaFree(h->d_mem);
-    delete h;
-    return cuda_fail(e, "cudaMemset of status");
-  }
   int smem_limit = 0;
   e = cudaDeviceGetAttribute(&smem_limit, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
   if (e != cudaSuccess) {
@@ -159,27 +162,12 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   for (int k = 0; k < 4; ++k) m.plane[k] = k < np ? d + o_plane[k] : nullptr;
   m.pair = d + o_pair;
   m.pair_stride = (int32_t)pair_stride;
-  m.status = reinterpret_cast<uint32_t*>(d + o_status);
   m.smem_limit = smem_limit;
   m.row_ptr = reinterpret_cast<const int32_t*>(d + o_rp);
   m.entries = reinterpret_cast<const uint32_t*>(d + o_ent);
   m.tables = reinterpret_cast<const float2*>(d + o_tab);
+  m.max_cta_entries = max_cta;
   m.num_sms = prop.multiProcessorCount;
-  // entries per stage of the row partition every precision uses
-  {
-    int grid = 0, rs = 0;
-    stage_partition(s->out, s->in, m.num_sms, &grid, &rs);
-    int64_t most = 0;
-    for (int b = 0; b < grid; ++b) {
-      const int64_t ra = (int64_t)b * s->out / grid, rb = (int64_t)(b + 1) * s->out / grid;
-      for (int64_t q = ra; q < rb; q += rs) {
-        const int64_t qe = q + rs < rb ? q + rs : rb;
-        const int64_t cnt = (int64_t)s->row_ptr[qe] - s->row_ptr[q];
-        if (cnt > most) most = cnt;
-      }
-    }
-    m.ecap = (int)(most < kMaxEntryCap ? most : kMaxEntryCap);
-  }
   for (int b = 2; b <= 2 + np; ++b) h->plan_ok[b] = make_plan(m, b, &h->plan[b]);
   if (!h->plan_ok[2]) {
     cudaFree(h->d_mem);
@@ -282,14 +270,11 @@ extern "C" int stagq_check(stagq_handle h) {
   if (!h) return fail(STAGQ_EINVAL, "null handle");
   DeviceGuard guard(h->device);
   if (!guard.ok) return fail(STAGQ_ECUDA, "cudaSetDevice failed");
-  uint32_t word = 0;
   cudaError_t e = cudaDeviceSynchronize();
-  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-  e = cudaMemcpy(&word, h->dm.status, 4, cudaMemcpyDeviceToHost);
-  if (e != cudaSuccess) return cuda_fail(e, "status read");
-  if (!word) return STAGQ_OK;
-  cudaMemset(h->dm.status, 0, 4);
-  return fail(STAGQ_ETIMEOUT, "a GEMV kernel gave up waiting for its data (status " + std::to_string(word) + ")");
+  if (e != cudaSuccess) return cuda_fail(e, "work on the handle's device failed");
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pending CUDA error");
+  return STAGQ_OK;
 }
 
 extern "C" int stagq_info(stagq_handle h, stagq_info_t* info) {

@@ -6,10 +6,10 @@
 
 namespace stagq {
 
-constexpr int kMaxConsumerWarps = 16;   // + 1 producer warp per CTA
-constexpr int kMaxStageRows = 32;       // rows per stage (one producer lane per row)
-constexpr int kMaxRowsPerCta = 2048;    // row_ptr of a CTA's range is cached in shared memory
-constexpr int kMaxEntryCap = 2048;      // side-record entries prefetched per stage
+constexpr int kMaxConsumerWarps = 16;   // warps per CTA
+constexpr int kMaxRowsPerCta = 2048;    // a CTA's row_ptr / slice offsets live in shared memory
+constexpr int kPrefetchGroups = 4;      // deepest cp.async prefetch (batches in flight per lane)
+constexpr int kSliceWeights = 2048;     // K weights per K slice (one warp: 32 lanes x 64)
 
 struct DeviceMatrix {
   int32_t out, in, group, n_planes;
@@ -19,21 +19,20 @@ struct DeviceMatrix {
   const uint8_t* pair;        // 8-bit pairs, row stride pair_stride (in/group padded to 16)
   int32_t pair_stride;
   const int32_t* row_ptr;     // [out+1]
-  const uint32_t* entries;    // [nnz]: column | (fp16 value << 16), 16 bytes of padding after
+  const uint32_t* entries;    // [nnz]: column | (fp16 value << 16), then 16 bytes of padding
+  int32_t max_cta_entries;    // most side-record entries in one CTA's row range
   const float2* tables;       // [n_planes+1][256]: (lo_M, s_M * c_M) for M = 2..2+n_planes
-  uint32_t* status;           // device word: nonzero if a kernel gave up on a wait
   int num_sms;
   int smem_limit;             // opt-in shared memory per block
-  int ecap;                   // side-record entries to prefetch per stage
 };
 
 // How one GEMV is laid out over the GPU (see gemv.cu).
 struct GemvPlan {
   int grid;              // CTAs (one per SM unless rows per CTA would exceed kMaxRowsPerCta)
-  int KW, RG, up;        // K-warps, row groups, rows per row group per stage
-  int rows_per_stage;    // RG * up (<= kMaxStageRows)
-  int slots;             // shared-memory ring depth
-  int ecap;              // entries prefetched per stage
+  int KW, RG, up;        // K slices, row groups, rows per batch
+  int depth;             // batches each lane keeps in flight (2..kPrefetchGroups)
+  int ent_cap;           // side-record entries staged per CTA (0: read from global memory)
+  int group_shift;       // log2(group)
   int pair_stride;
   int max_rows_per_cta;
   int pdl;               // launch with programmatic dependent launch
@@ -41,8 +40,8 @@ struct GemvPlan {
 
 // Plan for a GEMV at `bits`; returns false if the shape cannot be planned.
 bool make_plan(const DeviceMatrix& m, int bits, GemvPlan* plan);
-// Rows per stage / grid of the plan used for every precision (entry cap sizing).
-void stage_partition(int out, int in, int num_sms, int* grid, int* rows_per_stage);
+int k_slices(int in);
+int gemv_grid(int out, int num_sms);
 uint32_t gemv_smem_bytes(const GemvPlan& plan, int in, int bits);
 
 // y = W_hat^(bits) x for n = 1. y is fp16 (y_f32 = 0) or fp32.

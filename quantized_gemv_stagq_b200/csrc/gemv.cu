@@ -8,28 +8,25 @@
 // zero, so the main stream decoded lo_M there and the correction is v - lo_M).
 //
 // How (design for B200; batch-one GEMV is bound by HBM, so no tensor cores):
-//  * one CTA per SM owns a contiguous, balanced range of rows, cut into
-//    "stages" of R_s consecutive rows. Because every plane is row-major, a
-//    stage is one contiguous byte range per plane: a producer warp streams
-//    base + planes 3..M (only those: a p_M read never touches deeper planes)
-//    + pair bytes with 1-D bulk copies (cp.async.bulk, mbarrier completion)
-//    into a ring of shared-memory slots, as far ahead as the ring allows, and
-//    prefetches each stage's side-record entries with cp.async;
+//  * one CTA per SM owns a contiguous, balanced range of rows; its warps are
+//    KW "K slices" (2048 weights of K each: 32 lanes x one 64-weight chunk)
+//    times RG row groups, and each warp walks its rows UP at a time;
+//  * the CTA's pair bytes and side-record entries are staged in shared memory
+//    once, up front; every lane streams its own chunk bytes -- 16 base bytes
+//    + 8 bytes per read plane (a p_M read never touches deeper planes) -- with
+//    cp.async into its own shared-memory ring, several batches ahead, so the
+//    loop has no barrier: cp.async.wait_group is the only ordering;
 //  * x is converted once per CTA to 16-bit fixed point with a power-of-two
-//    scale per 64-element chunk (|error| <= 2^-16 max|x_chunk|); each consumer
-//    lane keeps its chunk's 64 activations in registers for every row;
-//  * consumer warps = KW "K-warps" (2048 weights of K each) x RG row groups.
-//    A lane turns 16 base bytes (+ 8 bytes per plane) of one 64-weight chunk
-//    into code bytes / nibble composites (layout.cuh) and feeds them to dp2a
-//    integer dot products (exact in int32); the group affine is applied once
-//    per chunk in fp32; rows are reduced across lanes by a transposed shuffle;
-//  * each stage row's side-record correction is computed by one consumer warp
-//    (lanes over entries); the producer warp then adds the K-warp partials in
-//    a fixed order, adds the correction and stores y -- deterministic, no
-//    atomics, no workspace, no second launch (the K split of Appendix G's
-//    atomic-add kernel becomes a fixed-order shared-memory reduction);
-//  * every mbarrier wait is bounded in time; on expiry the kernel records an
-//    error in the handle's status word and returns.
+//    scale per 64-element chunk (|error| <= 2^-16 max|x_chunk|); each lane
+//    keeps its chunk's 64 activations in registers for every row;
+//  * a lane turns its chunk into code bytes / nibble composites (layout.cuh)
+//    and feeds them to dp2a integer dot products (exact in int32); the group
+//    affine is applied once per chunk in fp32 and a transposed shuffle reduces
+//    the batch's rows to one partial per (row, K slice) in shared memory;
+//  * a final pass per row adds the held-out entries, x_c (v - lo_M), and the
+//    KW partials in a fixed order and stores y -- deterministic, no atomics,
+//    no workspace, no second launch (the K split of Appendix G's atomic-add
+//    kernel becomes this reduction).
 #include <cuda_fp16.h>
 
 #include <cstdint>
@@ -42,66 +39,13 @@ namespace stagq {
 namespace {
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait, then give up
 
 // ------------------------------------------------------------ PTX helpers
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-__device__ __forceinline__ uint64_t global_timer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(b)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(b)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(b)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_addr(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
-  if (mbar_try_wait(b, parity)) return true;
-  const uint64_t t0 = global_timer();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(b, parity)) return true;
-    if ((i & 63u) == 0 && global_timer() - t0 > kWaitLimitNs) return false;
-  }
-}
-// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* b) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(b)) : "memory");
-}
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-__device__ __forceinline__ void fence_barrier_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -221,11 +165,24 @@ struct GemvKernelArgs {
   int y_f32;
 };
 
+// Copies of 16 / 8 bytes that read `n` of them (0 or all) and zero-fill
+// the rest, so a predicate needs no branch. `src` must be a valid address.
+__device__ __forceinline__ void cp_async16z(uint32_t dst, const void* src, uint32_t n) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async8z(uint32_t dst, const void* src, uint32_t n) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Shared-memory carve-up, identical on host (plan) and device.
 struct SmemLayout {
-  uint32_t full, ent, empty;        // mbarrier arrays [S]
-  uint32_t xq, xh, xscale, xsum, tab, rp, partial, corr, slots;
-  uint32_t slot_bytes, s_base, s_plane, s_pair, s_ent;
+  uint32_t xq, xh, xscale, xsum, tab, rp, pairs, ents, partial, ring;
+  uint32_t warp_ring;  // bytes of one warp's ring
   uint32_t total;
 };
 
@@ -233,114 +190,119 @@ __host__ __device__ inline uint32_t align_up_u32(uint32_t v, uint32_t a) { retur
 
 __host__ __device__ inline SmemLayout smem_layout(const GemvPlan& p, int in, int M) {
   SmemLayout L;
-  const uint32_t S = p.slots, Rs = p.rows_per_stage, nchunk = in / kChunk;
+  const uint32_t nchunk = in / kChunk, R = p.max_rows_per_cta, W = p.KW * p.RG;
   uint32_t o = 0;
-  L.full = o; o += 8 * S;
-  L.ent = o; o += 8 * S;
-  L.empty = o; o += 8 * S;
-  o = align_up_u32(o, 16);
   L.xq = o; o += 2 * in;
   L.xh = o; o += 2 * in;
   L.xscale = o; o += 4 * nchunk;
   L.xsum = o; o += 4 * nchunk;
   o = align_up_u32(o, 16);
   L.tab = o; o += 256 * 8;
-  L.rp = o; o += 4 * (p.max_rows_per_cta + 1);
+  L.rp = o; o += 4 * (R + 1);
   o = align_up_u32(o, 16);
-  L.partial = o; o += 4 * S * p.KW * Rs;
-  L.corr = o; o += 4 * S * Rs;
+  L.pairs = o; o += R * p.pair_stride;
+  o = align_up_u32(o, 16);
+  L.ents = o; o += 4 * (p.ent_cap + 4);
+  L.partial = o; o += 4 * p.KW * R;
   o = align_up_u32(o, 128);
-  L.slots = o;
-  L.s_base = 0;
-  L.s_plane = Rs * (in / 4);
-  L.s_pair = L.s_plane + (M - 2) * Rs * (in / 8);
-  L.s_ent = align_up_u32(L.s_pair + Rs * p.pair_stride, 16);
-  L.slot_bytes = align_up_u32(L.s_ent + 4 * p.ecap, 128);
-  o += S * L.slot_bytes;
+  L.ring = o;
+  L.warp_ring = (uint32_t)(p.depth + 1) * p.up * 32u * (16 + 8 * (M - 2));
+  o += W * L.warp_ring;
   L.total = o;
   return L;
 }
 
-template <int M, int UP>
-__global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(const GemvKernelArgs a) {
+template <int M, int UP, int D>
+__global__ void __launch_bounds__(kMaxConsumerWarps * 32, 1) gemv_kernel(const GemvKernelArgs a) {
+  constexpr int NS = D + 1;                         // ring slots: D in flight + the one read
+  constexpr uint32_t RB = 32u * (16 + 8 * (M - 2));  // one row: base | planes, over 32 lanes
+  constexpr uint32_t SLOT = UP * RB;
   extern __shared__ __align__(128) uint8_t smem[];
   const GemvPlan& P = a.plan;
   const int in = a.m.in;
   const int nchunk = in / kChunk;
   const SmemLayout L = smem_layout(P, in, M);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.full);
-  uint64_t* ent_full = reinterpret_cast<uint64_t*>(smem + L.ent);
-  uint64_t* empty = reinterpret_cast<uint64_t*>(smem + L.empty);
   int16_t* xq = reinterpret_cast<int16_t*>(smem + L.xq);
   __half* xh = reinterpret_cast<__half*>(smem + L.xh);
   float* xscale = reinterpret_cast<float*>(smem + L.xscale);
   float* xsum = reinterpret_cast<float*>(smem + L.xsum);
   float2* tab = reinterpret_cast<float2*>(smem + L.tab);
-  int* rp = reinterpret_cast<int*>(smem + L.rp);
-  float* partial = reinterpret_cast<float*>(smem + L.partial);  // [S][KW][Rs]
-  float* corr = reinterpret_cast<float*>(smem + L.corr);        // [S][Rs]
-  uint8_t* slots = smem + L.slots;
+  int* rp = reinterpret_cast<int*>(smem + L.rp);                // [rows + 1] row_ptr
+  uint8_t* pairs = smem + L.pairs;                              // [rows][pair_stride]
+  uint32_t* ents = reinterpret_cast<uint32_t*>(smem + L.ents);  // staged side record
+  float* partial = reinterpret_cast<float*>(smem + L.partial);  // [rows][KW]
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int KW = P.KW, RG = P.RG, Wc = KW * RG, Rs = P.rows_per_stage, S = P.slots;
-  const bool producer = warp == Wc;
-  const int64_t r0 = (int64_t)blockIdx.x * a.m.out / gridDim.x;
-  const int64_t r1 = (int64_t)(blockIdx.x + 1) * a.m.out / gridDim.x;
-  const int rows = (int)(r1 - r0);
-  const int nst = (rows + Rs - 1) / Rs;
-  const uint32_t plane_row = in / 8, base_row = in / 4;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthreads = blockDim.x;
+  const int KW = P.KW, RG = P.RG, ps = P.pair_stride;
+  const int kw = warp % KW, rg = warp / KW;
+  const int c = kw * 32 + lane;  // this lane's 64-weight chunk
+  const bool active = c < nchunk;
+  const int gidx = (c * kChunk) >> P.group_shift;
+  const int r0 = (int)((int64_t)blockIdx.x * a.m.out / gridDim.x);
+  const int rows = (int)((int64_t)(blockIdx.x + 1) * a.m.out / gridDim.x) - r0;
+  const int rows_rg = rows > rg ? (rows - rg + RG - 1) / RG : 0;  // rows of this row group
+  const int nb = (rows_rg + UP - 1) / UP;                         // batches
+  const uint32_t ring = smem_addr(smem + L.ring) + (uint32_t)warp * L.warp_ring;  // shared address
+  const uint8_t* const ring_g = smem + L.ring + (size_t)warp * L.warp_ring;       // same, generic
 
-  if (tid == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&ent_full[s], 32);
-      mbar_init(&empty[s], Wc);
-    }
-    fence_barrier_init();
-  }
-  __syncthreads();
-
-  // Producer: bulk copies of one stage's planes + pair bytes into its slot.
-  auto issue_planes = [&](int st) {
-    const int slot = st % S;
-    const int64_t row0 = r0 + (int64_t)st * Rs;
-    const uint32_t n = (uint32_t)min(Rs, rows - st * Rs);
-    uint8_t* dst = slots + (size_t)slot * L.slot_bytes;
-    const uint32_t bb = n * base_row, pb = n * plane_row, qb = n * P.pair_stride;
-    mbar_arrive_expect_tx(&full[slot], bb + (M - 2) * pb + qb);
-    bulk_load(dst + L.s_base, a.m.base + row0 * base_row, bb, &full[slot]);
+  // Issue state: the next row (index mi within the row group) to prefetch.
+  const int64_t stride_b = (int64_t)RG * (in / 4), stride_p = (int64_t)RG * (in / 8);
+  const uint8_t* ib = a.m.base + (int64_t)(r0 + rg) * (in / 4) + c * kBaseChunkBytes;
+  const uint8_t* ip[M > 2 ? M - 2 : 1];
 #pragma unroll
-    for (int k = 0; k < M - 2; ++k)
-      bulk_load(dst + L.s_plane + k * Rs * plane_row, a.m.plane[k] + row0 * plane_row, pb, &full[slot]);
-    bulk_load(dst + L.s_pair, a.m.pair + row0 * P.pair_stride, qb, &full[slot]);
-  };
-  // Producer warp: side-record entries of one stage (first ecap of them).
-  auto issue_entries = [&](int st) {
-    const int slot = st % S;
-    const int lr0 = st * Rs, lr1 = min(lr0 + Rs, rows);
-    const int e0 = rp[lr0], n = min(rp[lr1] - e0, P.ecap);
-    uint32_t* dst = reinterpret_cast<uint32_t*>(slots + (size_t)slot * L.slot_bytes + L.s_ent);
-    for (int e = lane; e < n; e += 32) cp_async4(dst + e, a.m.entries + e0 + e);
-    cp_async_arrive_noinc(&ent_full[slot]);
-  };
+  for (int k = 0; k < M - 2; ++k) ip[k] = a.m.plane[k] + (int64_t)(r0 + rg) * (in / 8) + c * kPlaneChunkBytes;
+  const uint8_t* const safe = a.m.base;  // a valid address for zero-byte copies
+  int left = active ? rows_rg : 0;        // rows still to prefetch
+  uint32_t slot_i = 0;
 
-  if (producer) {
-    if (lane == 0)
-      for (int st = 0; st < min(S, nst); ++st) issue_planes(st);
-    for (int i = lane; i <= rows; i += 32) rp[i] = __ldg(a.m.row_ptr + r0 + i);
-    __syncwarp();
-    for (int st = 0; st < min(S, nst); ++st) issue_entries(st);
+#define STAGQ_ISSUE_BATCH()                                                                    \
+  {                                                                                            \
+    uint32_t rec = ring + slot_i * SLOT + lane * 16;                                           \
+    _Pragma("unroll") for (int u = 0; u < UP; ++u) {                                           \
+      const bool ok = u < left;                                                                \
+      cp_async16z(rec, ok ? ib : safe, ok ? 16u : 0u);                                         \
+      _Pragma("unroll") for (int k = 0; k < M - 2; ++k)                                        \
+        cp_async8z(rec - lane * 8 + 512 + k * 256, ok ? ip[k] : safe, ok ? 8u : 0u);           \
+      ib += stride_b;                                                                          \
+      _Pragma("unroll") for (int k = 0; k < M - 2; ++k) ip[k] += stride_p;                     \
+      rec += RB;                                                                               \
+    }                                                                                          \
+    left -= UP;                                                                                \
+    slot_i = slot_i + 1 == NS ? 0 : slot_i + 1;                                                \
+    cp_async_commit();                                                                         \
   }
-  // Let the next kernel in the stream start its own prologue early; x (which a
-  // previous kernel may have produced) is read only after the dependency wait.
-  grid_launch_dependents();
-  grid_dependency_wait();
 
-  if (!producer) {
-    for (int i = tid; i < 256; i += Wc * 32) tab[i] = a.table[i];
-    // x -> fixed point; a task is 8 consecutive values, 8 tasks form a chunk.
+  // Copy order (cp.async groups): this CTA's pair bytes, the weights of
+  // batches 0..D-1, then its side record -- so batch b can start as soon as
+  // the pair bytes and its own weights have landed.
+  {
+    const uint32_t pdst = smem_addr(pairs);
+    const uint8_t* psrc = a.m.pair + (int64_t)r0 * ps;
+    for (int i = tid * 16; i < rows * ps; i += nthreads * 16) cp_async16z(pdst + i, psrc + i, 16u);
+    cp_async_commit();
+  }
+#pragma unroll
+  for (int b = 0; b < D; ++b) STAGQ_ISSUE_BATCH();
+  grid_launch_dependents();
+  if (tid < 256) tab[tid] = a.table[tid];
+  for (int i = tid; i <= rows; i += nthreads) rp[i] = __ldg(a.m.row_ptr + r0 + i);
+  const int e_begin = __ldg(a.m.row_ptr + r0), e_end = __ldg(a.m.row_ptr + r0 + rows);
+  const int e_base = e_begin & ~3;  // staged from a 16-byte boundary
+  const bool staged = (e_end - e_base) <= P.ent_cap;
+  {
+    if (staged) {
+      const uint32_t edst = smem_addr(ents);
+      const uint32_t* esrc = a.m.entries + e_base;
+      const int n16 = (e_end - e_base + 3) >> 2;  // 16-byte chunks; the entries array is padded
+      for (int i = tid; i < n16; i += nthreads) cp_async16z(edst + 16 * i, esrc + 4 * i, 16u);
+    }
+    cp_async_commit();
+  }
+  grid_dependency_wait();  // x may come from the previous kernel
+  {
+    // x -> 16-bit fixed point; a task is 8 values, 8 tasks form a 64-value chunk.
     const int n8 = in / 8;
-    for (int i0 = warp * 32; i0 < n8; i0 += Wc * 32) {
+    for (int i0 = warp * 32; i0 < n8; i0 += nthreads) {
       const int i = i0 + lane;
       const bool v = i < n8;
       uint4 raw = make_uint4(0u, 0u, 0u, 0u);
@@ -384,124 +346,84 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32 + 32, 1) gemv_kernel(co
       }
     }
   }
+  // Pair bytes are group 0: with D + 1 newer groups allowed pending it has landed.
+  cp_async_wait_group<D + 1>();
   __syncthreads();
 
-  if (!producer) {
-    // ------------------------------------------------------------ consumers
-    const int kw = warp % KW, rg = warp / KW;
-    const int c = kw * 32 + lane;  // this lane's 64-weight chunk
-    const bool active = c < nchunk;
-    const int gidx = (c * kChunk) / a.m.group;
-    uint32_t X[32];
-    float xs = 0.f, xsm = 0.f;
-    if (active) {
-      const uint4* src = reinterpret_cast<const uint4*>(xq + c * kChunk);
+  uint32_t X[32];
+  float xs, xsm;
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(xq + (active ? c : 0) * kChunk);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint4 t = src[k];
-        X[4 * k] = t.x;
-        X[4 * k + 1] = t.y;
-        X[4 * k + 2] = t.z;
-        X[4 * k + 3] = t.w;
-      }
-      xs = xscale[c];
-      xsm = xsum[c];
-    } else {
-#pragma unroll
-      for (int k = 0; k < 32; ++k) X[k] = 0u;
+    for (int k = 0; k < 8; ++k) {
+      const uint4 t = src[k];
+      X[4 * k] = t.x;
+      X[4 * k + 1] = t.y;
+      X[4 * k + 2] = t.z;
+      X[4 * k + 3] = t.w;
     }
+    xs = active ? xscale[c] : 0.f;
+    xsm = active ? xsum[c] : 0.f;
+  }
 
-    for (int st = 0; st < nst; ++st) {
-      const int slot = st % S;
-      const uint32_t par = (uint32_t)(st / S) & 1u;
-      const int n = min(Rs, rows - st * Rs);
-      const uint8_t* sd = slots + (size_t)slot * L.slot_bytes;
-      if (!mbar_wait(&full[slot], par)) {
-        if (lane == 0) atomicOr(a.m.status, 1u);
-        return;
-      }
-      float v[UP];
+  uint32_t slot_c = 0;
+  const uint8_t* pr = pairs + rg * ps + gidx;  // pair byte of the row being consumed
+  const int pr_step = RG * ps;
+  float* pw_out = partial + rg * KW + kw;
+  for (int b = 0; b < nb; ++b) {
+    // Groups so far: pairs, batches 0..D-1, side record, then one refill per
+    // iteration. Batch b < D is group b + 1, batch b >= D group b + 2.
+    if (b < D) cp_async_wait_group<D>();
+    else cp_async_wait_group<D - 1>();
+    const uint8_t* rec = ring_g + slot_c * SLOT + lane * 16;
+    const int valid = rows_rg - UP * b;  // rows of this batch that exist
+    float v[UP];
 #pragma unroll
-      for (int u = 0; u < UP; ++u) {
-        const int row = rg + RG * u;  // stage-local
-        v[u] = 0.f;
-        if (row < n && active) {
-          const uint4 b4 = *reinterpret_cast<const uint4*>(sd + L.s_base + row * base_row + c * kBaseChunkBytes);
-          const uint32_t B[4] = {b4.x, b4.y, b4.z, b4.w};
-          uint2 Pw[M > 2 ? M - 2 : 1];
+    for (int u = 0; u < UP; ++u) {
+      const uint4 b4 = *reinterpret_cast<const uint4*>(rec + u * RB);
+      const uint32_t B[4] = {b4.x, b4.y, b4.z, b4.w};
+      uint2 Pw[M > 2 ? M - 2 : 1];
 #pragma unroll
-          for (int k = 0; k < M - 2; ++k)
-            Pw[k] = *reinterpret_cast<const uint2*>(sd + L.s_plane + (k * Rs + row) * plane_row +
-                                                   c * kPlaneChunkBytes);
-          const int tot = chunk_dot<M>(X, B, Pw);
-          const float2 lm = tab[sd[L.s_pair + row * P.pair_stride + gidx]];
-          v[u] = fmaf(lm.y, (float)tot * xs, lm.x * xsm);
-        }
-      }
-      const float s = transposed_reduce<UP>(v, lane);
-      const int u_of_lane = lane / (32 / UP);
-      if ((lane & (32 / UP - 1)) == 0) {
-        const int row = rg + RG * u_of_lane;
-        if (row < n) partial[(slot * KW + kw) * Rs + row] = s;
-      }
-      // side-record corrections of the stage rows assigned to this warp
-      const int first = (st * Rs) % Wc;
-      int j = warp - first;
-      if (j < 0) j += Wc;
-      if (j < n) {
-        if (!mbar_wait(&ent_full[slot], par)) {
-          if (lane == 0) atomicOr(a.m.status, 2u);
-          return;
-        }
-        const uint32_t* se = reinterpret_cast<const uint32_t*>(sd + L.s_ent);
-        const int est = rp[st * Rs];
-        for (; j < n; j += Wc) {
-          const int e0 = rp[st * Rs + j], e1 = rp[st * Rs + j + 1];
-          float cs = 0.f;
-          for (int e = e0 + lane; e < e1; e += 32) {
-            const int le = e - est;
-            const uint32_t en = le < P.ecap ? se[le] : __ldg(a.m.entries + e);
-            const int col = (int)(en & 0xFFFFu);
-            const float val = __half2float(__ushort_as_half((unsigned short)(en >> 16)));
-            const float lo = tab[sd[L.s_pair + j * P.pair_stride + col / a.m.group]].x;
-            cs = fmaf(__half2float(xh[col]), val - lo, cs);
-          }
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) cs += __shfl_xor_sync(kFull, cs, off);
-          if (lane == 0) corr[slot * Rs + j] = cs;
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);
+      for (int k = 0; k < M - 2; ++k)
+        Pw[k] = *reinterpret_cast<const uint2*>(rec - lane * 8 + u * RB + 512 + k * 256);
+      const int tot = chunk_dot<M>(X, B, Pw);
+      const float2 lm = tab[u < valid ? pr[u * pr_step] : 0];
+      v[u] = fmaf(lm.y, (float)tot * xs, lm.x * xsm);
     }
-  } else {
-    // ------------------------------------------------------------- producer
-    for (int st = 0; st < nst; ++st) {
-      const int slot = st % S;
-      const uint32_t par = (uint32_t)(st / S) & 1u;
-      const int n = min(Rs, rows - st * Rs);
-      if (!mbar_wait(&empty[slot], par)) {
-        if (lane == 0) atomicOr(a.m.status, 4u);
-        break;
-      }
-      if (lane < n) {
-        float acc = 0.f;
-        for (int k = 0; k < KW; ++k) acc += partial[(slot * KW + k) * Rs + lane];
-        acc += corr[slot * Rs + lane];
-        const int64_t r = r0 + (int64_t)st * Rs + lane;
-        if (a.y_f32) reinterpret_cast<float*>(a.y)[r] = acc;
-        else reinterpret_cast<__half*>(a.y)[r] = __float2half_rn(acc);
-      }
-      __syncwarp();
-      if (st + S < nst) {
-        if (lane == 0) issue_planes(st + S);
-        issue_entries(st + S);
-      }
+    slot_c = slot_c + 1 == NS ? 0 : slot_c + 1;
+    STAGQ_ISSUE_BATCH();  // batch b + D refills the slot read one batch ago
+
+    const float s = transposed_reduce<UP>(v, lane);
+    const int uu = lane / (32 / UP);
+    if ((lane & (32 / UP - 1)) == 0 && uu < valid) pw_out[uu * RG * KW] = s;
+    pr += UP * pr_step;
+    pw_out += UP * RG * KW;
+  }
+#undef STAGQ_ISSUE_BATCH
+  cp_async_wait_all();
+  __syncthreads();
+
+  // Per row: held-out entries add x_c (v - lo_M(g(r, c))); then the K-slice
+  // partials in order; one warp per row, lanes over the row's entries.
+  const int nwarps = nthreads >> 5;
+  for (int lr = warp; lr < rows; lr += nwarps) {
+    const int e0 = rp[lr], e1 = rp[lr + 1];
+    float cs = 0.f;
+    for (int e = e0 + lane; e < e1; e += 32) {
+      const uint32_t en = staged ? ents[e - e_base] : __ldg(a.m.entries + e);
+      const int col = (int)(en & 0xFFFFu);
+      const float lo = tab[pairs[lr * ps + (col >> P.group_shift)]].x;
+      cs = fmaf(__half2float(xh[col]), __half2float(__ushort_as_half((unsigned short)(en >> 16))) - lo, cs);
     }
-    // Nothing may still be landing in shared memory when the CTA exits.
-    cp_async_wait_all();
-    for (int st = max(0, nst - S); st < nst; ++st)
-      mbar_wait(&full[st % S], (uint32_t)(st / S) & 1u);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) cs += __shfl_xor_sync(kFull, cs, off);
+    if (lane == 0) {
+      float acc = 0.f;
+      for (int k = 0; k < KW; ++k) acc += partial[lr * KW + k];
+      acc += cs;
+      if (a.y_f32) reinterpret_cast<float*>(a.y)[r0 + lr] = acc;
+      else reinterpret_cast<__half*>(a.y)[r0 + lr] = __float2half_rn(acc);
+    }
   }
 }
 
@@ -529,11 +451,11 @@ __global__ void decode_levels_kernel(const DeviceMatrix m, uint8_t* u) {
 cudaError_t ensure_smem(const void* kern, int key, size_t smem) {
   constexpr int kMaxDev = 64;
   static std::mutex mu;
-  static size_t granted[kMaxDev][32] = {};
+  static size_t granted[kMaxDev][64] = {};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (dev < 0 || dev >= kMaxDev || key < 0 || key >= 32) return cudaErrorInvalidValue;
+  if (dev < 0 || dev >= kMaxDev || key < 0 || key >= 64) return cudaErrorInvalidValue;
   std::lock_guard<std::mutex> lock(mu);
   if (granted[dev][key] >= smem) return cudaSuccess;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -541,9 +463,9 @@ cudaError_t ensure_smem(const void* kern, int key, size_t smem) {
   return err;
 }
 
-template <int M, int UP>
-cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const void* x, void* y, int y_f32,
-                           cudaStream_t stream) {
+template <int M, int UP, int D>
+cudaError_t launch_gemv_mud(const DeviceMatrix& m, const GemvPlan& plan, const void* x, void* y, int y_f32,
+                            cudaStream_t stream) {
   GemvKernelArgs a;
   a.m = m;
   a.plan = plan;
@@ -552,12 +474,12 @@ cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const vo
   a.y = y;
   a.y_f32 = y_f32;
   const SmemLayout L = smem_layout(plan, m.in, M);
-  auto kern = gemv_kernel<M, UP>;
-  cudaError_t err = ensure_smem(reinterpret_cast<const void*>(kern), M * 4 + UP, L.total);
+  auto kern = gemv_kernel<M, UP, D>;
+  cudaError_t err = ensure_smem(reinterpret_cast<const void*>(kern), ((M - 2) * 3 + (UP == 4 ? 2 : UP - 1)) * 4 + D - 1, L.total);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)plan.grid);
-  cfg.blockDim = dim3((unsigned)(32 * (plan.KW * plan.RG + 1)));
+  cfg.blockDim = dim3((unsigned)(32 * plan.KW * plan.RG));
   cfg.dynamicSmemBytes = L.total;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -566,6 +488,18 @@ cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const vo
   cfg.attrs = attr;
   cfg.numAttrs = plan.pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+template <int M, int UP>
+cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const void* x, void* y, int y_f32,
+                           cudaStream_t stream) {
+  switch (plan.depth) {
+    case 1: return launch_gemv_mud<M, UP, 1>(m, plan, x, y, y_f32, stream);
+    case 2: return launch_gemv_mud<M, UP, 2>(m, plan, x, y, y_f32, stream);
+    case 3: return launch_gemv_mud<M, UP, 3>(m, plan, x, y, y_f32, stream);
+    case 4: return launch_gemv_mud<M, UP, 4>(m, plan, x, y, y_f32, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 template <int M>
@@ -592,43 +526,35 @@ cudaError_t launch_decode_m(const DeviceMatrix& m, uint8_t* u, cudaStream_t stre
 
 uint32_t gemv_smem_bytes(const GemvPlan& plan, int in, int bits) { return smem_layout(plan, in, bits).total; }
 
-void stage_partition(int out, int in, int num_sms, int* grid, int* rows_per_stage) {
-  const int KW = (in / kChunk + 31) / 32;
-  const int RG = KW >= kMaxConsumerWarps ? 1 : kMaxConsumerWarps / KW;
-  const int up = RG * 2 <= kMaxStageRows ? 2 : 1;
+int gemv_grid(int out, int num_sms) {
   int g = out < num_sms ? out : num_sms;
   if ((out + g - 1) / g > kMaxRowsPerCta) g = (out + kMaxRowsPerCta - 1) / kMaxRowsPerCta;
-  *grid = g;
-  *rows_per_stage = RG * up;
+  return g;
 }
 
+int k_slices(int in) { return (in / kChunk + 31) / 32; }
+
 bool make_plan(const DeviceMatrix& m, int bits, GemvPlan* p) {
-  const int nchunk = m.in / kChunk;
-  p->KW = (nchunk + 31) / 32;
+  p->KW = k_slices(m.in);
   if (p->KW > kMaxConsumerWarps) return false;
-  p->RG = p->KW >= kMaxConsumerWarps ? 1 : kMaxConsumerWarps / p->KW;
-  int grid = 0, rs = 0;
-  stage_partition(m.out, m.in, m.num_sms, &grid, &rs);
-  p->grid = grid;
-  p->max_rows_per_cta = (m.out + grid - 1) / grid;
+  p->RG = kMaxConsumerWarps / p->KW;
+  p->grid = gemv_grid(m.out, m.num_sms);
+  p->max_rows_per_cta = (m.out + p->grid - 1) / p->grid;
   p->pair_stride = m.pair_stride;
-  p->ecap = m.ecap;
+  p->group_shift = 0;
+  while ((1 << p->group_shift) < m.group) ++p->group_shift;
   p->pdl = 1;
-  // Two rows per row group and stage if the ring can still hold >= 3 stages,
-  // else one; the ring then takes as many slots as shared memory allows.
-  for (int up = rs / p->RG; up >= 1; --up) {
-    p->up = up;
-    p->rows_per_stage = p->RG * up;
-    const int nst = (p->max_rows_per_cta + p->rows_per_stage - 1) / p->rows_per_stage;
-    int S = 0;
-    for (int t = 1; t <= nst; ++t) {
-      p->slots = t;
-      if (smem_layout(*p, m.in, bits).total > (uint32_t)m.smem_limit) break;
-      S = t;
+  // Stage the side record in shared memory when it fits beside a ring of at
+  // least two batches, else read it from global memory in the final pass.
+  for (int stage_ents = 1; stage_ents >= 0; --stage_ents) {
+    p->ent_cap = stage_ents ? m.max_cta_entries + 4 : 0;
+    for (int up = 4; up >= 1; up /= 2) {
+      p->up = up;
+      for (int d = kPrefetchGroups; d >= 2; --d) {
+        p->depth = d;
+        if (smem_layout(*p, m.in, bits).total <= (uint32_t)m.smem_limit) return true;
+      }
     }
-    if (S == 0) continue;
-    p->slots = S;
-    if (S >= (nst < 3 ? nst : 3) || up == 1) return true;
   }
   return false;
 }

@@ -20,8 +20,8 @@ int check_shape(int64_t out, int64_t in, int64_t group, int n_planes) {
   if (out <= 0 || in <= 0) return fail(STAGQ_EINVAL, "shape must be positive");
   if (in % STAGQ_IN_MULTIPLE) return fail(STAGQ_EINVAL, "in must be a multiple of 128");
   if (in > STAGQ_MAX_IN) return fail(STAGQ_EINVAL, "in exceeds STAGQ_MAX_IN");
-  if (group <= 0 || in % group || group % 64 != 0)
-    return fail(STAGQ_EINVAL, "group must divide in and be a multiple of 64");
+  if (group < 64 || in % group || (group & (group - 1)) != 0)
+    return fail(STAGQ_EINVAL, "group must be a power of two >= 64 that divides in");
   if (n_planes < 0 || n_planes > STAGQ_MAX_PLANES) return fail(STAGQ_EINVAL, "n_planes out of range");
   if (out > (int64_t)1 << 30) return fail(STAGQ_EINVAL, "out too large");
   return STAGQ_OK;
@@ -42,6 +42,9 @@ int validate_stream(const stagq_host_stream* s) {
   if (s->row_ptr[s->out] != s->nnz) return fail(STAGQ_EFORMAT, "row_ptr[out] != nnz");
   for (int64_t e = 0; e < s->nnz; ++e)
     if (s->col[e] >= s->in) return fail(STAGQ_EFORMAT, "side-record column >= in");
+  for (int64_t r = 0; r < s->out; ++r)
+    for (int64_t e = (int64_t)s->row_ptr[r] + 1; e < s->row_ptr[r + 1]; ++e)
+      if (s->col[e] <= s->col[e - 1]) return fail(STAGQ_EFORMAT, "side-record columns not increasing in a row");
   return STAGQ_OK;
 }
 
@@ -60,7 +63,6 @@ extern "C" const char* stagq_strerror(int status) {
     case STAGQ_ECUDA: return "CUDA error";
     case STAGQ_EIO: return "I/O error";
     case STAGQ_ENODEV: return "no usable sm_100 device";
-    case STAGQ_ETIMEOUT: return "kernel wait timed out";
     default: return "unknown status";
   }
 }
