@@ -41,6 +41,7 @@ extern "C" {
 #define STAGQ_ECUDA 4    /* a CUDA runtime call failed (detail in stagq_last_error) */
 #define STAGQ_EIO 5      /* file could not be read or written */
 #define STAGQ_ENODEV 6   /* no usable sm_100 device */
+#define STAGQ_ETIMEOUT 7 /* a GEMV kernel gave up waiting for its own copies (reported by stagq_check) */
 
 /* Limits of this implementation. */
 #define STAGQ_MAX_PLANES 4      /* stream depth N = 2 + n_planes <= 6 (the paper evaluates N = 6) */
@@ -211,7 +212,11 @@ int64_t stagq_bytes(stagq_handle h, int bits, int n);
 /*
  * Synchronise the handle's device and report any CUDA error raised by work
  * queued on it (the GEMV entry points are asynchronous and only report launch
- * errors). Returns STAGQ_OK or STAGQ_ECUDA.
+ * errors), then whether a GEMV on this handle gave up waiting for its own
+ * copies since the last check (every wait inside the kernel is bounded to
+ * 2 s; on expiry the kernel sets the handle's status word, lets its copies in
+ * flight land and returns, leaving y undefined). Clears the status word.
+ * Returns STAGQ_OK, STAGQ_ETIMEOUT or STAGQ_ECUDA.
  */
 int stagq_check(stagq_handle h);
 

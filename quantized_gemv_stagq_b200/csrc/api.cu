@@ -93,16 +93,30 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   const size_t base_bytes = (size_t)(out_ * in / 4), plane_bytes = (size_t)(out_ * in / 8);
   const size_t pair_row = (size_t)(in / s->group), pair_stride = align_up(pair_row, 16);
   const size_t pair_bytes = (size_t)out_ * pair_stride;
-  const size_t rp_bytes = (size_t)(out_ + 1) * 4, ent_bytes = (size_t)s->nnz * 4;
   const size_t tab_bytes = (size_t)(np + 1) * 256 * sizeof(float2);
+  // Side record cut per CTA of the GEMV grid (see DeviceMatrix::side).
+  const int grid = gemv_grid(s->out, s->in, prop.multiProcessorCount);
+  const int KW = k_slices(s->in), RG = row_groups(KW);
+  const int rows_cap = (int)((out_ + grid - 1) / grid);
+  const int class_rows = (rows_cap + RG - 1) / RG;
+  int64_t max_cta = 0;
+  for (int b = 0; b < grid; ++b) {
+    const int64_t ra = (int64_t)b * out_ / grid, rb = (int64_t)(b + 1) * out_ / grid;
+    const int64_t n = (int64_t)s->row_ptr[rb] - s->row_ptr[ra];
+    if (n > max_cta) max_cta = n;
+  }
+  const size_t side_ent_off = align_up((size_t)4 * RG * KW * ((size_t)class_rows + 1), 16);
+  const size_t side_stride = align_up(side_ent_off + 4 * (size_t)max_cta, 16);
+  if (side_stride > (size_t)INT32_MAX) return fail(STAGQ_EINVAL, "side record too large per CTA");
+  const size_t side_bytes = (size_t)grid * side_stride;
   size_t off = 0;
   const size_t o_base = off; off = align_up(off + base_bytes, 256);
   size_t o_plane[STAGQ_MAX_PLANES] = {};
   for (int k = 0; k < np; ++k) { o_plane[k] = off; off = align_up(off + plane_bytes, 256); }
   const size_t o_pair = off; off = align_up(off + pair_bytes, 256);
-  const size_t o_rp = off; off = align_up(off + rp_bytes, 256);
-  const size_t o_ent = off; off = align_up(off + ent_bytes + 16, 256);  // +16: 16-byte staged reads
+  const size_t o_side = off; off = align_up(off + side_bytes, 256);
   const size_t o_tab = off; off = align_up(off + tab_bytes, 256);
+  const size_t o_status = off; off = align_up(off + 4, 256);
   const size_t total = off;
 
   stagq_matrix* h = new (std::nothrow) stagq_matrix();
@@ -117,18 +131,32 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   h->d_bytes = total;
   uint8_t* d = static_cast<uint8_t*>(h->d_mem);
 
-  std::vector<uint32_t> ent((size_t)s->nnz);
-  for (int64_t i = 0; i < s->nnz; ++i) ent[i] = (uint32_t)s->col[i] | ((uint32_t)s->val[i] << 16);
   std::vector<float2> tabs;
   build_tables(s, tabs);
-  // most side-record entries in one CTA's row range
-  int32_t max_cta = 0;
+  std::vector<uint8_t> side(side_bytes, 0);
   {
-    const int grid = gemv_grid(s->out, prop.multiProcessorCount);
     for (int b = 0; b < grid; ++b) {
-      const int64_t ra = (int64_t)b * s->out / grid, rb = (int64_t)(b + 1) * s->out / grid;
-      const int64_t n = (int64_t)s->row_ptr[rb] - s->row_ptr[ra];
-      if (n > max_cta) max_cta = (int32_t)n;
+      const int64_t ra = (int64_t)b * out_ / grid, rb = (int64_t)(b + 1) * out_ / grid, n = rb - ra;
+      uint8_t* blk = &side[(size_t)b * side_stride];
+      int32_t* offs = reinterpret_cast<int32_t*>(blk);
+      uint32_t* ent = reinterpret_cast<uint32_t*>(blk + side_ent_off);
+      int32_t pos = 0;
+      for (int rg = 0; rg < RG; ++rg) {
+        const int64_t nm = n > rg ? (n - rg + RG - 1) / RG : 0;
+        for (int kw = 0; kw < KW; ++kw) {
+          int32_t* o = offs + ((size_t)rg * KW + kw) * ((size_t)class_rows + 1);
+          for (int64_t m = 0; m < nm; ++m) {
+            const int64_t r = ra + rg + (int64_t)RG * m;
+            o[m] = pos;
+            int64_t e = s->row_ptr[r];
+            const int64_t e1 = s->row_ptr[r + 1];
+            while (e < e1 && s->col[e] < (int64_t)kw * kSliceWeights) ++e;  // columns increase within a row
+            for (; e < e1 && s->col[e] < (int64_t)(kw + 1) * kSliceWeights; ++e)
+              ent[pos++] = (uint32_t)s->col[e] | ((uint32_t)s->val[e] << 16);
+          }
+          o[nm] = pos;
+        }
+      }
     }
   }
   std::vector<uint8_t> pairs(pair_bytes, 0);
@@ -138,8 +166,7 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   std::vector<Copy> copies = {{o_base, s->planes, base_bytes}};
   for (int k = 0; k < np; ++k) copies.push_back({o_plane[k], s->planes + base_bytes + (size_t)k * plane_bytes, plane_bytes});
   copies.push_back({o_pair, pairs.data(), pair_bytes});
-  copies.push_back({o_rp, s->row_ptr, rp_bytes});
-  if (ent_bytes) copies.push_back({o_ent, ent.data(), ent_bytes});
+  copies.push_back({o_side, side.data(), side_bytes});
   copies.push_back({o_tab, tabs.data(), tab_bytes});
   for (const Copy& c : copies) {
     e = cudaMemcpy(d + c.off, c.src, c.n, cudaMemcpyHostToDevice);
@@ -149,8 +176,11 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
       return cuda_fail(e, "cudaMemcpy of stream");
     }
   }
-  int smem_limit = 0;
-  e = cudaDeviceGetAttribute(&smem_limit, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+  e = cudaMemset(d + o_status, 0, 4);
+  int smem_limit = 0, smem_sm = 0, smem_reserved = 0;
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&smem_limit, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&smem_reserved, cudaDevAttrReservedSharedMemoryPerBlock, device);
   if (e != cudaSuccess) {
     cudaFree(h->d_mem);
     delete h;
@@ -163,11 +193,15 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   m.pair = d + o_pair;
   m.pair_stride = (int32_t)pair_stride;
   m.smem_limit = smem_limit;
-  m.row_ptr = reinterpret_cast<const int32_t*>(d + o_rp);
-  m.entries = reinterpret_cast<const uint32_t*>(d + o_ent);
+  m.side = d + o_side;
+  m.side_stride = (int32_t)side_stride;
+  m.side_ent_off = (int32_t)side_ent_off;
+  m.side_grid = grid;
   m.tables = reinterpret_cast<const float2*>(d + o_tab);
-  m.max_cta_entries = max_cta;
+  m.status = reinterpret_cast<uint32_t*>(d + o_status);
   m.num_sms = prop.multiProcessorCount;
+  m.smem_pair_budget = smem_sm / 2 - smem_reserved;
+  if (m.smem_pair_budget > smem_limit) m.smem_pair_budget = smem_limit;
   for (int b = 2; b <= 2 + np; ++b) h->plan_ok[b] = make_plan(m, b, &h->plan[b]);
   if (!h->plan_ok[2]) {
     cudaFree(h->d_mem);
@@ -274,6 +308,14 @@ extern "C" int stagq_check(stagq_handle h) {
   if (e != cudaSuccess) return cuda_fail(e, "work on the handle's device failed");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pending CUDA error");
+  uint32_t word = 0;
+  e = cudaMemcpy(&word, h->dm.status, 4, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (word) {
+    e = cudaMemset(h->dm.status, 0, 4);
+    if (e != cudaSuccess) return cuda_fail(e, "status reset");
+    return fail(STAGQ_ETIMEOUT, "a GEMV kernel gave up waiting for its copies (status " + std::to_string(word) + ")");
+  }
   return STAGQ_OK;
 }
 

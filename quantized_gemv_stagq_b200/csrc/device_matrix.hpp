@@ -6,10 +6,14 @@
 
 namespace stagq {
 
-constexpr int kMaxConsumerWarps = 16;   // warps per CTA
-constexpr int kMaxRowsPerCta = 2048;    // a CTA's row_ptr / slice offsets live in shared memory
-constexpr int kPrefetchGroups = 4;      // deepest cp.async prefetch (batches in flight per lane)
+constexpr int kMaxWarps = 16;           // warps per CTA (K slices x row groups)
+constexpr int kMaxSlots = 8;            // shared-memory ring slots
+constexpr int kMaxRowsPerCta = 2048;    // rows of one CTA
 constexpr int kSliceWeights = 2048;     // K weights per K slice (one warp: 32 lanes x 64)
+constexpr int kCtasPerSm = 2;           // GEMV CTAs per SM (<= 8 warps and <= half the SM's shared memory each)
+
+// Row groups of a CTA with KW K slices: up to 8 warps in all, at least one group.
+inline int row_groups(int KW) { return KW <= 4 ? 8 / KW : 1; }
 
 struct DeviceMatrix {
   int32_t out, in, group, n_planes;
@@ -18,30 +22,40 @@ struct DeviceMatrix {
   const uint8_t* plane[4];    // planes 3..6, out*in/8 bytes each (null when absent)
   const uint8_t* pair;        // 8-bit pairs, row stride pair_stride (in/group padded to 16)
   int32_t pair_stride;
-  const int32_t* row_ptr;     // [out+1]
-  const uint32_t* entries;    // [nnz]: column | (fp16 value << 16), then 16 bytes of padding
-  int32_t max_cta_entries;    // most side-record entries in one CTA's row range
+  // Side record cut per CTA of the GEMV grid (side_grid CTAs over the rows as
+  // gemv_grid splits them), side_stride bytes each. A CTA's rows fall in RG
+  // classes (local row mod RG); its entries are ordered by (class, K slice,
+  // row, column), and int32 offsets [RG][KW][class_rows + 1] give where each
+  // row of a class starts within its (class, K slice) run, plus the run's end.
+  // The entries (column | fp16 value << 16) start at side_ent_off.
+  const uint8_t* side;
+  int32_t side_stride, side_ent_off, side_grid;
   const float2* tables;       // [n_planes+1][256]: (lo_M, s_M * c_M) for M = 2..2+n_planes
+  uint32_t* status;           // nonzero once a kernel gave up waiting for its copies
   int num_sms;
   int smem_limit;             // opt-in shared memory per block
+  int smem_pair_budget;       // shared memory per block that still lets two blocks share an SM
 };
 
 // How one GEMV is laid out over the GPU (see gemv.cu).
 struct GemvPlan {
-  int grid;              // CTAs (one per SM unless rows per CTA would exceed kMaxRowsPerCta)
-  int KW, RG, up;        // K slices, row groups, rows per batch
-  int depth;             // batches each lane keeps in flight (2..kPrefetchGroups)
-  int ent_cap;           // side-record entries staged per CTA (0: read from global memory)
+  int grid;              // CTAs (= side_grid)
+  int KW, RG, NW;        // K slices, row groups, warps (KW * RG)
+  int up, br;            // rows per warp per block, rows per block (RG * up)
+  int ns;                // ring slots
+  int stage_side;        // the CTA's side record is copied into shared memory
+  int side_stride;
+  int rows_cap;          // most rows of one CTA
+  int class_rows;        // most rows of one row class (ceil(rows_cap / RG))
   int group_shift;       // log2(group)
   int pair_stride;
-  int max_rows_per_cta;
   int pdl;               // launch with programmatic dependent launch
 };
 
 // Plan for a GEMV at `bits`; returns false if the shape cannot be planned.
 bool make_plan(const DeviceMatrix& m, int bits, GemvPlan* plan);
 int k_slices(int in);
-int gemv_grid(int out, int num_sms);
+int gemv_grid(int out, int in, int num_sms);
 uint32_t gemv_smem_bytes(const GemvPlan& plan, int in, int bits);
 
 // y = W_hat^(bits) x for n = 1. y is fp16 (y_f32 = 0) or fp32.

@@ -4,29 +4,38 @@
 //   y_i = sum_groups [ s_M(g) * sum_{j in g} u_M,j x_j + lo_M(g) * sum_{j in g} x_j ]
 //         + sum_{held-out (i,c)} x_c (v_ic - lo_M(g(i,c)))
 // -- the affine map of Eq. (10) applied once per group, with u_M from Eq. (8),
-// and the side record of Eq. (4) fused into the epilogue (held-out digits are
-// zero, so the main stream decoded lo_M there and the correction is v - lo_M).
+// and the side record of Eq. (4) fused in (held-out digits are zero, so the
+// main stream decoded lo_M there and the correction is v - lo_M).
 //
 // How (design for B200; batch-one GEMV is bound by HBM, so no tensor cores):
-//  * one CTA per SM owns a contiguous, balanced range of rows; its warps are
-//    KW "K slices" (2048 weights of K each: 32 lanes x one 64-weight chunk)
-//    times RG row groups, and each warp walks its rows UP at a time;
-//  * the CTA's pair bytes and side-record entries are staged in shared memory
-//    once, up front; every lane streams its own chunk bytes -- 16 base bytes
-//    + 8 bytes per read plane (a p_M read never touches deeper planes) -- with
-//    cp.async into its own shared-memory ring, several batches ahead, so the
-//    loop has no barrier: cp.async.wait_group is the only ordering;
-//  * x is converted once per CTA to 16-bit fixed point with a power-of-two
-//    scale per 64-element chunk (|error| <= 2^-16 max|x_chunk|); each lane
-//    keeps its chunk's 64 activations in registers for every row;
-//  * a lane turns its chunk into code bytes / nibble composites (layout.cuh)
-//    and feeds them to dp2a integer dot products (exact in int32); the group
-//    affine is applied once per chunk in fp32 and a transposed shuffle reduces
-//    the batch's rows to one partial per (row, K slice) in shared memory;
-//  * a final pass per row adds the held-out entries, x_c (v - lo_M), and the
-//    KW partials in a fixed order and stores y -- deterministic, no atomics,
-//    no workspace, no second launch (the K split of Appendix G's atomic-add
-//    kernel becomes this reduction).
+//  * one CTA per SM owns a contiguous, balanced range of rows. It is cut into
+//    blocks of BR rows; a block's base rows, read-plane rows (a p_M read never
+//    touches deeper planes) and pair bytes are contiguous in HBM, so one
+//    thread moves a block into a shared-memory ring slot with 2 + (M - 2)
+//    bulk copies (cp.async.bulk, completion on the slot's mbarrier). The
+//    CTA's side record (per (row, K slice) offsets + entries, cut per CTA at
+//    load time) and the precision's pair table arrive the same way;
+//  * the CTA is small (<= 8 warps, <= 113 KB of shared memory, <= 128
+//    registers a thread) so the next GEMV's CTA fits beside it on the SM:
+//    with programmatic dependent launch its copies are in flight while this
+//    GEMV computes;
+//  * warps are KW "K slices" (2048 weights of K each: 32 lanes x one
+//    64-weight chunk) times RG row groups; in every block each warp takes UP
+//    rows, as straight-line code so their dot products interleave;
+//  * each lane turns its 64 activations into 16-bit fixed point with a
+//    power-of-two scale (|error| <= 2^-16 max|x_chunk|) and keeps them in
+//    registers; code bytes / nibble composites (layout.cuh) feed dp2a integer
+//    dot products (exact in int32); the group affine is applied once per chunk
+//    in fp32; the K slice's held-out entries add x~_c (v - lo_M) with the same
+//    fixed-point x~, so the result is exactly W_hat x~ up to fp32 rounding;
+//  * a transposed shuffle reduces the UP rows to one partial per (row, K
+//    slice); the warp that finishes a block last (a shared-memory counter)
+//    adds the block's KW partials in a fixed order, stores y and refills the
+//    slot -- deterministic, no atomics on data, no workspace, no second
+//    launch (the K split of Appendix G's atomic-add kernel becomes this);
+//  * every mbarrier wait is bounded in time; on expiry the kernel records it
+//    in the handle's status word, waits (bounded) for its own copies and
+//    returns.
 #include <cuda_fp16.h>
 
 #include <cstdint>
@@ -40,12 +49,54 @@ namespace {
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
+
 // ------------------------------------------------------------ PTX helpers
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ uint64_t global_timer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait until the phase of `bar` with the given parity has completed, for at
+// most `limit_ns`; false on expiry.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 15u) == 0 && global_timer() - t0 > limit_ns) return false;
+  }
+}
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+// dst, src and bytes are multiples of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
 __device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -165,24 +216,14 @@ struct GemvKernelArgs {
   int y_f32;
 };
 
-// Copies of 16 / 8 bytes that read `n` of them (0 or all) and zero-fill
-// the rest, so a predicate needs no branch. `src` must be a valid address.
-__device__ __forceinline__ void cp_async16z(uint32_t dst, const void* src, uint32_t n) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
-}
-__device__ __forceinline__ void cp_async8z(uint32_t dst, const void* src, uint32_t n) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // a copy that has not landed in 2 s never will
+constexpr uint64_t kDrainLimitNs = 100000000ull;   // after a failure: wait for own copies, 0.1 s
 
 // Shared-memory carve-up, identical on host (plan) and device.
 struct SmemLayout {
-  uint32_t xq, xh, xscale, xsum, tab, rp, pairs, ents, partial, ring;
-  uint32_t warp_ring;  // bytes of one warp's ring
+  uint32_t bar, cnt, last, tab, xq, xscale, xsum, partial, side, ring;
+  uint32_t slot;                 // bytes of one ring slot
+  uint32_t plane_piece, pair_piece;  // offsets inside a slot (base rows at 0)
   uint32_t total;
 };
 
@@ -190,170 +231,220 @@ __host__ __device__ inline uint32_t align_up_u32(uint32_t v, uint32_t a) { retur
 
 __host__ __device__ inline SmemLayout smem_layout(const GemvPlan& p, int in, int M) {
   SmemLayout L;
-  const uint32_t nchunk = in / kChunk, R = p.max_rows_per_cta, W = p.KW * p.RG;
+  const uint32_t nchunk = in / kChunk, BR = p.br;
   uint32_t o = 0;
+  L.bar = o; o += 8 * (kMaxSlots + 1);  // full[slot] + side/table barrier
+  L.cnt = o; o += 4 * kMaxSlots;         // warps done with the slot's blocks so far
+  L.last = o; o += 4 * kMaxSlots;        // last block issued into the slot
+  o = align_up_u32(o, 16);
+  L.tab = o; o += 256 * 8;
   L.xq = o; o += 2 * in;
-  L.xh = o; o += 2 * in;
   L.xscale = o; o += 4 * nchunk;
   L.xsum = o; o += 4 * nchunk;
   o = align_up_u32(o, 16);
-  L.tab = o; o += 256 * 8;
-  L.rp = o; o += 4 * (R + 1);
-  o = align_up_u32(o, 16);
-  L.pairs = o; o += R * p.pair_stride;
-  o = align_up_u32(o, 16);
-  L.ents = o; o += 4 * (p.ent_cap + 4);
-  L.partial = o; o += 4 * p.KW * R;
+  L.partial = o; o += 4u * p.ns * BR * p.KW;
+  o = align_up_u32(o, 128);
+  L.side = o; o += p.stage_side ? (uint32_t)p.side_stride : 0u;
   o = align_up_u32(o, 128);
   L.ring = o;
-  L.warp_ring = (uint32_t)(p.depth + 1) * p.up * 32u * (16 + 8 * (M - 2));
-  o += W * L.warp_ring;
+  L.plane_piece = BR * (in / 4);
+  L.pair_piece = L.plane_piece + (uint32_t)(M - 2) * BR * (in / 8);
+  L.slot = align_up_u32(L.pair_piece + BR * p.pair_stride, 128);
+  o += p.ns * L.slot;
   L.total = o;
   return L;
 }
 
-template <int M, int UP, int D>
-__global__ void __launch_bounds__(kMaxConsumerWarps * 32, 1) gemv_kernel(const GemvKernelArgs a) {
-  constexpr int NS = D + 1;                         // ring slots: D in flight + the one read
-  constexpr uint32_t RB = 32u * (16 + 8 * (M - 2));  // one row: base | planes, over 32 lanes
-  constexpr uint32_t SLOT = UP * RB;
+// Dot products of NR rows of one block for this lane's chunk, with the group
+// affine: v[u] = s_M c_M sum(v x~) + lo_M sum(x~) over the chunk, and the
+// lane's lo_M per row (for the side record). Row u of the warp sits at
+// offsets off.b + u * step.b (base), off.p + u * step.p (first read plane;
+// plane k at + k * plane_stride) and off.g + u * step.g (pair byte) in the slot.
+struct RowOffsets {
+  uint32_t b, p, g;
+};
+
+template <int M, int NR>
+__device__ __forceinline__ void rows_dot(const uint32_t (&X)[32], float xs, float xsm, const uint8_t* sb,
+                                         RowOffsets off, RowOffsets step, uint32_t plane_stride, const float2* tab,
+                                         float (&v)[NR], float (&lo)[NR]) {
+#pragma unroll
+  for (int u = 0; u < NR; ++u) {
+    const uint4 b4 = *reinterpret_cast<const uint4*>(sb + off.b + u * step.b);
+    const uint32_t B[4] = {b4.x, b4.y, b4.z, b4.w};
+    uint2 Pw[M > 2 ? M - 2 : 1];
+#pragma unroll
+    for (int k = 0; k < M - 2; ++k)
+      Pw[k] = *reinterpret_cast<const uint2*>(sb + off.p + u * step.p + k * plane_stride);
+    const int tot = chunk_dot<M>(X, B, Pw);
+    const float2 lm = tab[sb[off.g + u * step.g]];
+    v[u] = fmaf(lm.y, (float)tot * xs, lm.x * xsm);
+    lo[u] = lm.x;
+  }
+}
+
+// Held-out entries of NR consecutive rows of the warp's row class in its K
+// slice: entries [o[0], o[NR]) of the CTA's side record, row u owning
+// [o[u], o[u+1]). Adds x~_c (v - lo_M) to v[u]; lo_M comes from the lane
+// that owns column c (same K slice).
+template <int NR>
+__device__ __forceinline__ void side_record(const int (&o)[NR + 1], const uint32_t* ents, const int16_t* xq,
+                                            const float* xscale, int lane, const float (&lo)[NR], float (&v)[NR]) {
+  for (int j0 = o[0]; j0 < o[NR]; j0 += 32) {
+    const int j = j0 + lane;
+    const bool ok = j < o[NR];
+    const uint32_t en = ents[ok ? j : o[0]];
+    const int col = (int)(en & 0xFFFFu);
+    const int src = (col >> 6) & 31;
+    int u = 0;
+#pragma unroll
+    for (int i = 1; i < NR; ++i) u += j >= o[i];
+    float l = __shfl_sync(kFull, lo[0], src);
+#pragma unroll
+    for (int i = 1; i < NR; ++i) {
+      const float li = __shfl_sync(kFull, lo[i], src);
+      l = u == i ? li : l;
+    }
+    const float xv = (float)xq[col] * xscale[col >> 6];
+    const float cs = ok ? xv * (__half2float(__ushort_as_half((unsigned short)(en >> 16))) - l) : 0.f;
+#pragma unroll
+    for (int i = 0; i < NR; ++i) v[i] += u == i ? cs : 0.f;
+  }
+}
+
+template <int M, int UP>
+__global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKernelArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const GemvPlan& P = a.plan;
   const int in = a.m.in;
   const int nchunk = in / kChunk;
   const SmemLayout L = smem_layout(P, in, M);
+  const uint32_t sbase = smem_addr(smem);
+  float2* tab = reinterpret_cast<float2*>(smem + L.tab);
   int16_t* xq = reinterpret_cast<int16_t*>(smem + L.xq);
-  __half* xh = reinterpret_cast<__half*>(smem + L.xh);
   float* xscale = reinterpret_cast<float*>(smem + L.xscale);
   float* xsum = reinterpret_cast<float*>(smem + L.xsum);
-  float2* tab = reinterpret_cast<float2*>(smem + L.tab);
-  int* rp = reinterpret_cast<int*>(smem + L.rp);                // [rows + 1] row_ptr
-  uint8_t* pairs = smem + L.pairs;                              // [rows][pair_stride]
-  uint32_t* ents = reinterpret_cast<uint32_t*>(smem + L.ents);  // staged side record
-  float* partial = reinterpret_cast<float*>(smem + L.partial);  // [rows][KW]
+  float* partial = reinterpret_cast<float*>(smem + L.partial);  // [slot][BR][KW]
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + L.cnt);
+  int* last = reinterpret_cast<int*>(smem + L.last);
+  const uint32_t full0 = sbase + L.bar, side_bar = sbase + L.bar + 8 * kMaxSlots;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthreads = blockDim.x;
-  const int KW = P.KW, RG = P.RG, ps = P.pair_stride;
+  const int KW = P.KW, RG = P.RG, NW = P.NW, NS = P.ns, BR = P.br, ps = P.pair_stride;
   const int kw = warp % KW, rg = warp / KW;
   const int c = kw * 32 + lane;  // this lane's 64-weight chunk
   const bool active = c < nchunk;
-  const int gidx = (c * kChunk) >> P.group_shift;
+  const int cc = active ? c : 0;  // reads of inactive lanes stay inside the row
   const int r0 = (int)((int64_t)blockIdx.x * a.m.out / gridDim.x);
   const int rows = (int)((int64_t)(blockIdx.x + 1) * a.m.out / gridDim.x) - r0;
-  const int rows_rg = rows > rg ? (rows - rg + RG - 1) / RG : 0;  // rows of this row group
-  const int nb = (rows_rg + UP - 1) / UP;                         // batches
-  const uint32_t ring = smem_addr(smem + L.ring) + (uint32_t)warp * L.warp_ring;  // shared address
-  const uint8_t* const ring_g = smem + L.ring + (size_t)warp * L.warp_ring;       // same, generic
+  const int nblk = (rows + BR - 1) / BR;
+  const int rb = in / 4, rp = in / 8;
+  const uint8_t* side_g = a.m.side + (int64_t)blockIdx.x * a.m.side_stride;
+  const uint8_t* side = P.stage_side ? smem + L.side : side_g;
+  // (row class rg, K slice kw) run offsets: row m of the class starts at seg[m]
+  const int32_t* seg = reinterpret_cast<const int32_t*>(side) + (rg * KW + kw) * (P.class_rows + 1);
+  const uint32_t* ents = reinterpret_cast<const uint32_t*>(side + a.m.side_ent_off);
 
-  // Issue state: the next row (index mi within the row group) to prefetch.
-  const int64_t stride_b = (int64_t)RG * (in / 4), stride_p = (int64_t)RG * (in / 8);
-  const uint8_t* ib = a.m.base + (int64_t)(r0 + rg) * (in / 4) + c * kBaseChunkBytes;
-  const uint8_t* ip[M > 2 ? M - 2 : 1];
+  // Block b of the CTA's rows -> slot b % NS (one thread).
+  auto issue_block = [&](int b, int slot) {
+    const int lr0 = b * BR;
+    const int nr = min(BR, rows - lr0);
+    const uint32_t dst = sbase + L.ring + slot * L.slot, bar = full0 + 8 * slot;
+    mbar_arrive_expect_tx(bar, (uint32_t)nr * (rb + (M - 2) * rp + ps));
+    bulk_load(dst, a.m.base + (int64_t)(r0 + lr0) * rb, nr * rb, bar);
 #pragma unroll
-  for (int k = 0; k < M - 2; ++k) ip[k] = a.m.plane[k] + (int64_t)(r0 + rg) * (in / 8) + c * kPlaneChunkBytes;
-  const uint8_t* const safe = a.m.base;  // a valid address for zero-byte copies
-  int left = active ? rows_rg : 0;        // rows still to prefetch
-  uint32_t slot_i = 0;
+    for (int k = 0; k < M - 2; ++k)
+      bulk_load(dst + L.plane_piece + k * BR * rp, a.m.plane[k] + (int64_t)(r0 + lr0) * rp, nr * rp, bar);
+    bulk_load(dst + L.pair_piece, a.m.pair + (int64_t)(r0 + lr0) * ps, nr * ps, bar);
+    last[slot] = b;
+  };
 
-#define STAGQ_ISSUE_BATCH()                                                                    \
-  {                                                                                            \
-    uint32_t rec = ring + slot_i * SLOT + lane * 16;                                           \
-    _Pragma("unroll") for (int u = 0; u < UP; ++u) {                                           \
-      const bool ok = u < left;                                                                \
-      cp_async16z(rec, ok ? ib : safe, ok ? 16u : 0u);                                         \
-      _Pragma("unroll") for (int k = 0; k < M - 2; ++k)                                        \
-        cp_async8z(rec - lane * 8 + 512 + k * 256, ok ? ip[k] : safe, ok ? 8u : 0u);           \
-      ib += stride_b;                                                                          \
-      _Pragma("unroll") for (int k = 0; k < M - 2; ++k) ip[k] += stride_p;                     \
-      rec += RB;                                                                               \
-    }                                                                                          \
-    left -= UP;                                                                                \
-    slot_i = slot_i + 1 == NS ? 0 : slot_i + 1;                                                \
-    cp_async_commit();                                                                         \
-  }
-
-  // Copy order (cp.async groups): this CTA's pair bytes, the weights of
-  // batches 0..D-1, then its side record -- so batch b can start as soon as
-  // the pair bytes and its own weights have landed.
-  {
-    const uint32_t pdst = smem_addr(pairs);
-    const uint8_t* psrc = a.m.pair + (int64_t)r0 * ps;
-    for (int i = tid * 16; i < rows * ps; i += nthreads * 16) cp_async16z(pdst + i, psrc + i, 16u);
-    cp_async_commit();
-  }
-#pragma unroll
-  for (int b = 0; b < D; ++b) STAGQ_ISSUE_BATCH();
-  grid_launch_dependents();
-  if (tid < 256) tab[tid] = a.table[tid];
-  for (int i = tid; i <= rows; i += nthreads) rp[i] = __ldg(a.m.row_ptr + r0 + i);
-  const int e_begin = __ldg(a.m.row_ptr + r0), e_end = __ldg(a.m.row_ptr + r0 + rows);
-  const int e_base = e_begin & ~3;  // staged from a 16-byte boundary
-  const bool staged = (e_end - e_base) <= P.ent_cap;
-  {
-    if (staged) {
-      const uint32_t edst = smem_addr(ents);
-      const uint32_t* esrc = a.m.entries + e_base;
-      const int n16 = (e_end - e_base + 3) >> 2;  // 16-byte chunks; the entries array is padded
-      for (int i = tid; i < n16; i += nthreads) cp_async16z(edst + 16 * i, esrc + 4 * i, 16u);
+  // Thread 0 sets up the barriers and starts the copies that do not depend
+  // on the previous kernel: the pair table, the side record and block 0. The
+  // other blocks follow once this CTA's x loads are on their way, so that x
+  // does not queue behind them. (Every thread passes the barrier after the x
+  // conversion before it waits on an mbarrier.)
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      cnt[s] = 0;
+      last[s] = -1;
     }
-    cp_async_commit();
+    mbar_init(side_bar, 1);
+    fence_barrier_init();
+    mbar_arrive_expect_tx(side_bar, 256 * 8 + (P.stage_side ? (uint32_t)a.m.side_stride : 0u));
+    bulk_load(sbase + L.tab, a.table, 256 * 8, side_bar);
+    if (P.stage_side) bulk_load(sbase + L.side, side_g, (uint32_t)a.m.side_stride, side_bar);
+    issue_block(0, 0);
   }
-  grid_dependency_wait();  // x may come from the previous kernel
+  grid_launch_dependents();
+  grid_dependency_wait();  // x may come from the previous kernel; y may be read by it
+
+  // x -> 16-bit fixed point, once per CTA: a task is a quarter chunk (16
+  // values) and the 4 tasks of a chunk sit in adjacent lanes. Scale 2^e with
+  // max|x| 2^e in [2^14, 2^15) per chunk, so the largest entries convert
+  // exactly; rounding to nearest even goes through the 1.5 * 2^23 shifter (the
+  // low 16 bits of the sum are the two's-complement integer).
   {
-    // x -> 16-bit fixed point; a task is 8 values, 8 tasks form a 64-value chunk.
-    const int n8 = in / 8;
-    for (int i0 = warp * 32; i0 < n8; i0 += nthreads) {
-      const int i = i0 + lane;
-      const bool v = i < n8;
-      uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-      if (v) raw = __ldg(reinterpret_cast<const uint4*>(a.x) + i);
-      const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
-      float f[8];
+    constexpr float kShift = 12582912.0f;
+    constexpr int kBatch = 4;
+    const int ntask = 4 * nchunk;
+    const uint4* x4 = reinterpret_cast<const uint4*>(a.x);
+    for (int t0 = 0; t0 < ntask; t0 += kBatch * nthreads) {
+      uint4 raw[kBatch][2];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 t = __half22float2(h2[k]);
-        f[2 * k] = t.x;
-        f[2 * k + 1] = t.y;
+      for (int q = 0; q < kBatch; ++q) {
+        const int t = t0 + q * nthreads + tid;
+        raw[q][0] = raw[q][1] = make_uint4(0u, 0u, 0u, 0u);
+        if (t < ntask) {
+          raw[q][0] = __ldg(x4 + 2 * t);
+          raw[q][1] = __ldg(x4 + 2 * t + 1);
+        }
       }
-      float mx = 0.f, sm = 0.f;
+      if (t0 == 0 && tid == 0)
+        for (int b = 1; b < NS && b < nblk; ++b) issue_block(b, b);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        mx = fmaxf(mx, fabsf(f[k]));
-        sm += f[k];
-      }
+      for (int q = 0; q < kBatch; ++q) {
+        const int tw = t0 + q * nthreads + warp * 32;  // first task of this warp
+        if (tw >= ntask) break;                         // warp-uniform
+        const int t = tw + lane;
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(raw[q]);
+        __half2 m2 = __habs2(*reinterpret_cast<const __half2*>(&w[0]));
 #pragma unroll
-      for (int off = 1; off < 8; off <<= 1) {
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
-        sm += __shfl_xor_sync(kFull, sm, off);
-      }
-      // e with max|x| 2^e in [2^14, 2^15): the largest entries convert exactly
-      const int e = mx > 0.f ? 14 - (((__float_as_int(mx) >> 23) & 0xFF) - 127) : 0;
-      const float sc = __int_as_float((127 + e) << 23);
-      uint32_t packed[4];
+        for (int k = 1; k < 8; ++k) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __half2*>(&w[k])));
+        float mx = fmaxf(__low2float(m2), __high2float(m2));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+        const int e = mx > 0.f ? 14 - ((int)((__float_as_uint(mx) >> 23) & 0xFF) - 127) : 0;
+        const float sc = __int_as_float((127 + e) << 23);
+        uint32_t Q[8];
+        int sumq = 0;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int lo16 = __float2int_rn(f[2 * k] * sc);
-        const int hi16 = __float2int_rn(f[2 * k + 1] * sc);
-        packed[k] = (uint32_t)(lo16 & 0xFFFF) | ((uint32_t)hi16 << 16);
-      }
-      if (v) {
-        reinterpret_cast<uint4*>(xh)[i] = raw;
-        reinterpret_cast<uint4*>(xq)[i] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        if ((i & 7) == 0) {
-          xscale[i >> 3] = __int_as_float((127 - e) << 23);
-          xsum[i >> 3] = sm;
+        for (int k = 0; k < 8; ++k) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+          Q[k] = __byte_perm(__float_as_uint(fmaf(f.x, sc, kShift)), __float_as_uint(fmaf(f.y, sc, kShift)), 0x5410);
+          sumq = dp2a_lo(Q[k], 0x0101u, sumq);
+        }
+        sumq += __shfl_xor_sync(kFull, sumq, 1);
+        sumq += __shfl_xor_sync(kFull, sumq, 2);
+        if (t < ntask) {
+          uint4* dst = reinterpret_cast<uint4*>(xq) + 2 * t;
+          dst[0] = make_uint4(Q[0], Q[1], Q[2], Q[3]);
+          dst[1] = make_uint4(Q[4], Q[5], Q[6], Q[7]);
+          if ((t & 3) == 0) {
+            const float xs_c = __int_as_float((127 - e) << 23);
+            xscale[t >> 2] = xs_c;
+            xsum[t >> 2] = xs_c * (float)sumq;
+          }
         }
       }
     }
   }
-  // Pair bytes are group 0: with D + 1 newer groups allowed pending it has landed.
-  cp_async_wait_group<D + 1>();
   __syncthreads();
-
   uint32_t X[32];
   float xs, xsm;
   {
-    const uint4* src = reinterpret_cast<const uint4*>(xq + (active ? c : 0) * kChunk);
+    const uint4* src = reinterpret_cast<const uint4*>(xq) + cc * 8;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const uint4 t = src[k];
@@ -362,68 +453,86 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32, 1) gemv_kernel(const G
       X[4 * k + 2] = t.z;
       X[4 * k + 3] = t.w;
     }
-    xs = active ? xscale[c] : 0.f;
-    xsm = active ? xsum[c] : 0.f;
+    xs = active ? xscale[cc] : 0.f;
+    xsm = active ? xsum[cc] : 0.f;
   }
 
-  uint32_t slot_c = 0;
-  const uint8_t* pr = pairs + rg * ps + gidx;  // pair byte of the row being consumed
-  const int pr_step = RG * ps;
-  float* pw_out = partial + rg * KW + kw;
-  for (int b = 0; b < nb; ++b) {
-    // Groups so far: pairs, batches 0..D-1, side record, then one refill per
-    // iteration. Batch b < D is group b + 1, batch b >= D group b + 2.
-    if (b < D) cp_async_wait_group<D>();
-    else cp_async_wait_group<D - 1>();
-    const uint8_t* rec = ring_g + slot_c * SLOT + lane * 16;
-    const int valid = rows_rg - UP * b;  // rows of this batch that exist
-    float v[UP];
-#pragma unroll
-    for (int u = 0; u < UP; ++u) {
-      const uint4 b4 = *reinterpret_cast<const uint4*>(rec + u * RB);
-      const uint32_t B[4] = {b4.x, b4.y, b4.z, b4.w};
-      uint2 Pw[M > 2 ? M - 2 : 1];
-#pragma unroll
-      for (int k = 0; k < M - 2; ++k)
-        Pw[k] = *reinterpret_cast<const uint2*>(rec - lane * 8 + u * RB + 512 + k * 256);
-      const int tot = chunk_dot<M>(X, B, Pw);
-      const float2 lm = tab[u < valid ? pr[u * pr_step] : 0];
-      v[u] = fmaf(lm.y, (float)tot * xs, lm.x * xsm);
-    }
-    slot_c = slot_c + 1 == NS ? 0 : slot_c + 1;
-    STAGQ_ISSUE_BATCH();  // batch b + D refills the slot read one batch ago
+  // Where this warp's rows sit in a slot (row u of the warp = block row rg + RG u).
+  const RowOffsets off = {(uint32_t)(rg * rb + cc * 16), (uint32_t)(L.plane_piece + rg * rp + cc * 8),
+                          (uint32_t)(L.pair_piece + rg * ps + ((cc * kChunk) >> P.group_shift))};
+  const RowOffsets step = {(uint32_t)(RG * rb), (uint32_t)(RG * rp), (uint32_t)(RG * ps)};
+  const uint32_t plane_stride = BR * rp;
 
-    const float s = transposed_reduce<UP>(v, lane);
-    const int uu = lane / (32 / UP);
-    if ((lane & (32 / UP - 1)) == 0 && uu < valid) pw_out[uu * RG * KW] = s;
-    pr += UP * pr_step;
-    pw_out += UP * RG * KW;
-  }
-#undef STAGQ_ISSUE_BATCH
-  cp_async_wait_all();
-  __syncthreads();
-
-  // Per row: held-out entries add x_c (v - lo_M(g(r, c))); then the K-slice
-  // partials in order; one warp per row, lanes over the row's entries.
-  const int nwarps = nthreads >> 5;
-  for (int lr = warp; lr < rows; lr += nwarps) {
-    const int e0 = rp[lr], e1 = rp[lr + 1];
-    float cs = 0.f;
-    for (int e = e0 + lane; e < e1; e += 32) {
-      const uint32_t en = staged ? ents[e - e_base] : __ldg(a.m.entries + e);
-      const int col = (int)(en & 0xFFFFu);
-      const float lo = tab[pairs[lr * ps + (col >> P.group_shift)]].x;
-      cs = fmaf(__half2float(xh[col]), __half2float(__ushort_as_half((unsigned short)(en >> 16))) - lo, cs);
+  bool ok = mbar_wait(side_bar, 0, kWaitLimitNs);
+  const uint8_t* ring_g = smem + L.ring;
+  int slot = 0;
+  uint32_t phase = 0, round = 0;
+  for (int b = 0; ok && b < nblk; ++b) {
+    if (!mbar_wait(full0 + 8 * slot, phase, kWaitLimitNs)) {
+      ok = false;
+      break;
     }
+    const uint8_t* sb = ring_g + slot * L.slot;
+    const int nr = min(BR, rows - b * BR);
+    float* pout = partial + (slot * BR + rg) * KW + kw;
+    const int32_t* o = seg + UP * b;  // this block's rows of the class
+    // my rows in this block; a short block runs as a full one with the
+    // missing rows masked, unless fewer than half of them are there
+    const int mine = nr == BR ? UP : (nr > rg ? (nr - rg + RG - 1) / RG : 0);
+    if (mine == UP || 2 * mine > UP) {
+      float v[UP], lo[UP];
+      rows_dot<M, UP>(X, xs, xsm, sb, off, step, plane_stride, tab, v, lo);
+      int ob[UP + 1];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) cs += __shfl_xor_sync(kFull, cs, off);
+      for (int i = 0; i <= UP; ++i) ob[i] = o[i < mine ? i : mine];
+      side_record<UP>(ob, ents, xq, xscale, lane, lo, v);
+      const float s = transposed_reduce<UP>(v, lane);
+      const int uu = lane / (32 / UP);
+      if ((lane & (32 / UP - 1)) == 0 && uu < mine) pout[uu * RG * KW] = s;
+    } else {
+      for (int u = 0; u < mine; ++u) {
+        float v[1], lo[1];
+        const RowOffsets ou = {off.b + u * step.b, off.p + u * step.p, off.g + u * step.g};
+        rows_dot<M, 1>(X, xs, xsm, sb, ou, step, plane_stride, tab, v, lo);
+        const int ob[2] = {o[u], o[u + 1]};
+        side_record<1>(ob, ents, xq, xscale, lane, lo, v);
+        const float s = transposed_reduce<1>(v, lane);
+        if (lane == 0) pout[u * RG * KW] = s;
+      }
+    }
+    // Done with the slot: the warp that finishes it last stores the block's
+    // rows of y and refills the slot.
+    __syncwarp();
+    uint32_t done = 0;
     if (lane == 0) {
-      float acc = 0.f;
-      for (int k = 0; k < KW; ++k) acc += partial[lr * KW + k];
-      acc += cs;
-      if (a.y_f32) reinterpret_cast<float*>(a.y)[r0 + lr] = acc;
-      else reinterpret_cast<__half*>(a.y)[r0 + lr] = __float2half_rn(acc);
+      __threadfence_block();
+      done = atomicAdd(cnt + slot, 1u) + 1u;
     }
+    done = __shfl_sync(kFull, done, 0);
+    if (done == (uint32_t)NW * (round + 1)) {
+      __threadfence_block();
+      if (lane < nr) {
+        const float* pr = partial + (slot * BR + lane) * KW;
+        float acc = 0.f;
+        for (int k = 0; k < KW; ++k) acc += pr[k];
+        if (a.y_f32) reinterpret_cast<float*>(a.y)[r0 + b * BR + lane] = acc;
+        else reinterpret_cast<__half*>(a.y)[r0 + b * BR + lane] = __float2half_rn(acc);
+      }
+      __syncwarp();
+      if (lane == 0 && b + NS < nblk) issue_block(b + NS, slot);
+    }
+    if (++slot == NS) {
+      slot = 0;
+      phase ^= 1u;
+      ++round;
+    }
+  }
+  if (!ok && lane == 0) atomicOr(a.m.status, 1u);
+  if (__syncthreads_or(!ok) && tid == 0) {
+    // Gave up: let this CTA's copies in flight land before it exits.
+    mbar_wait(side_bar, 0, kDrainLimitNs);
+    for (int s = 0; s < NS; ++s)
+      if (last[s] >= 0) mbar_wait(full0 + 8 * s, (uint32_t)(last[s] / NS) & 1u, kDrainLimitNs);
   }
 }
 
@@ -463,9 +572,9 @@ cudaError_t ensure_smem(const void* kern, int key, size_t smem) {
   return err;
 }
 
-template <int M, int UP, int D>
-cudaError_t launch_gemv_mud(const DeviceMatrix& m, const GemvPlan& plan, const void* x, void* y, int y_f32,
-                            cudaStream_t stream) {
+template <int M, int UP>
+cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const void* x, void* y, int y_f32,
+                           cudaStream_t stream) {
   GemvKernelArgs a;
   a.m = m;
   a.plan = plan;
@@ -474,12 +583,12 @@ cudaError_t launch_gemv_mud(const DeviceMatrix& m, const GemvPlan& plan, const v
   a.y = y;
   a.y_f32 = y_f32;
   const SmemLayout L = smem_layout(plan, m.in, M);
-  auto kern = gemv_kernel<M, UP, D>;
-  cudaError_t err = ensure_smem(reinterpret_cast<const void*>(kern), ((M - 2) * 3 + (UP == 4 ? 2 : UP - 1)) * 4 + D - 1, L.total);
+  auto kern = gemv_kernel<M, UP>;
+  cudaError_t err = ensure_smem(reinterpret_cast<const void*>(kern), (M - 2) * 3 + (UP == 4 ? 2 : UP - 1), L.total);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)plan.grid);
-  cfg.blockDim = dim3((unsigned)(32 * plan.KW * plan.RG));
+  cfg.blockDim = dim3((unsigned)(32 * plan.NW));
   cfg.dynamicSmemBytes = L.total;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -488,18 +597,6 @@ cudaError_t launch_gemv_mud(const DeviceMatrix& m, const GemvPlan& plan, const v
   cfg.attrs = attr;
   cfg.numAttrs = plan.pdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kern, a);
-}
-
-template <int M, int UP>
-cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const void* x, void* y, int y_f32,
-                           cudaStream_t stream) {
-  switch (plan.depth) {
-    case 1: return launch_gemv_mud<M, UP, 1>(m, plan, x, y, y_f32, stream);
-    case 2: return launch_gemv_mud<M, UP, 2>(m, plan, x, y, y_f32, stream);
-    case 3: return launch_gemv_mud<M, UP, 3>(m, plan, x, y, y_f32, stream);
-    case 4: return launch_gemv_mud<M, UP, 4>(m, plan, x, y, y_f32, stream);
-    default: return cudaErrorInvalidValue;
-  }
 }
 
 template <int M>
@@ -526,33 +623,63 @@ cudaError_t launch_decode_m(const DeviceMatrix& m, uint8_t* u, cudaStream_t stre
 
 uint32_t gemv_smem_bytes(const GemvPlan& plan, int in, int bits) { return smem_layout(plan, in, bits).total; }
 
-int gemv_grid(int out, int num_sms) {
-  int g = out < num_sms ? out : num_sms;
+int k_slices(int in) { return (in / kChunk + 31) / 32; }
+
+int gemv_grid(int out, int in, int num_sms) {
+  // two CTAs per SM while a CTA has <= 8 warps, else one
+  const int per_sm = k_slices(in) <= kMaxWarps / 2 ? kCtasPerSm : 1;
+  int g = out < per_sm * num_sms ? out : per_sm * num_sms;
   if ((out + g - 1) / g > kMaxRowsPerCta) g = (out + kMaxRowsPerCta - 1) / kMaxRowsPerCta;
   return g;
 }
 
-int k_slices(int in) { return (in / kChunk + 31) / 32; }
-
 bool make_plan(const DeviceMatrix& m, int bits, GemvPlan* p) {
-  p->KW = k_slices(m.in);
-  if (p->KW > kMaxConsumerWarps) return false;
-  p->RG = kMaxConsumerWarps / p->KW;
-  p->grid = gemv_grid(m.out, m.num_sms);
-  p->max_rows_per_cta = (m.out + p->grid - 1) / p->grid;
-  p->pair_stride = m.pair_stride;
-  p->group_shift = 0;
-  while ((1 << p->group_shift) < m.group) ++p->group_shift;
-  p->pdl = 1;
-  // Stage the side record in shared memory when it fits beside a ring of at
-  // least two batches, else read it from global memory in the final pass.
-  for (int stage_ents = 1; stage_ents >= 0; --stage_ents) {
-    p->ent_cap = stage_ents ? m.max_cta_entries + 4 : 0;
-    for (int up = 4; up >= 1; up /= 2) {
-      p->up = up;
-      for (int d = kPrefetchGroups; d >= 2; --d) {
-        p->depth = d;
-        if (smem_layout(*p, m.in, bits).total <= (uint32_t)m.smem_limit) return true;
+  GemvPlan q = {};
+  q.KW = k_slices(m.in);
+  if (q.KW < 1 || q.KW > kMaxWarps) return false;
+  q.RG = row_groups(q.KW);
+  q.NW = q.KW * q.RG;
+  q.grid = m.side_grid;
+  q.rows_cap = (m.out + q.grid - 1) / q.grid;
+  q.class_rows = (q.rows_cap + q.RG - 1) / q.RG;
+  q.pair_stride = m.pair_stride;
+  q.side_stride = m.side_stride;
+  q.group_shift = 0;
+  while ((1 << q.group_shift) < m.group) ++q.group_shift;
+  q.pdl = 1;
+  // Rows per warp per block: up to 4, but no more than the CTA's rows call for.
+  const int per_rg = (q.rows_cap + q.RG - 1) / q.RG;
+  const int up_max = per_rg >= 4 ? 4 : per_rg >= 2 ? 2 : 1;
+  // Shared memory: small enough for two CTAs per SM when the CTA has <= 8
+  // warps, else (or if nothing fits) the per-block maximum. Prefer the side
+  // record staged, then at least four slots (or one per block), then more
+  // rows per warp.
+  const int budgets[2] = {q.NW <= kMaxWarps / 2 ? m.smem_pair_budget : m.smem_limit, m.smem_limit};
+  for (int bi = 0; bi < 2; ++bi) {
+    for (int stage = 1; stage >= 0; --stage) {
+      bool have = false;
+      GemvPlan best = q;
+      for (int up = up_max; up >= 1; up /= 2) {
+        GemvPlan t = q;
+        t.up = up;
+        t.br = q.RG * up;
+        t.stage_side = stage;
+        const int nblk = (q.rows_cap + t.br - 1) / t.br;
+        t.ns = nblk < kMaxSlots ? nblk : kMaxSlots;
+        while (t.ns >= 1 && smem_layout(t, m.in, bits).total > (uint32_t)budgets[bi]) --t.ns;
+        if (t.ns < 1) continue;
+        if (t.ns >= (nblk < 4 ? nblk : 4)) {
+          *p = t;
+          return true;
+        }
+        if (!have || t.ns > best.ns) {
+          best = t;
+          have = true;
+        }
+      }
+      if (have) {
+        *p = best;
+        return true;
       }
     }
   }

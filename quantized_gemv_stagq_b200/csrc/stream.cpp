@@ -63,6 +63,7 @@ extern "C" const char* stagq_strerror(int status) {
     case STAGQ_ECUDA: return "CUDA error";
     case STAGQ_EIO: return "I/O error";
     case STAGQ_ENODEV: return "no usable sm_100 device";
+    case STAGQ_ETIMEOUT: return "kernel gave up waiting for its copies";
     default: return "unknown status";
   }
 }
