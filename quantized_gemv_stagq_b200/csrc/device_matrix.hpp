@@ -10,7 +10,7 @@ constexpr int kMaxWarps = 16;           // warps per CTA (K slices x row groups)
 constexpr int kMaxSlots = 8;            // shared-memory ring slots
 constexpr int kMaxRowsPerCta = 2048;    // rows of one CTA
 constexpr int kSliceWeights = 2048;     // K weights per K slice (one warp: 32 lanes x 64)
-constexpr int kCtasPerSm = 2;           // GEMV CTAs per SM (<= 8 warps and <= half the SM's shared memory each)
+constexpr int64_t kTwoCtaWeightsPerSm = 256 * 1024;  // from this many weights per SM on, two GEMV CTAs per SM
 
 // Row groups of a CTA with KW K slices: up to 8 warps in all, at least one group.
 inline int row_groups(int KW) { return KW <= 4 ? 8 / KW : 1; }

@@ -13,21 +13,23 @@
 //    touches deeper planes) and pair bytes are contiguous in HBM, so one
 //    thread moves a block into a shared-memory ring slot with 2 + (M - 2)
 //    bulk copies (cp.async.bulk, completion on the slot's mbarrier). The
-//    CTA's side record (per (row, K slice) offsets + entries, cut per CTA at
-//    load time) and the precision's pair table arrive the same way;
+//    CTA's side record (cut per CTA at load time) and the precision's pair
+//    table arrive the same way;
 //  * the CTA is small (<= 8 warps, <= 113 KB of shared memory, <= 128
 //    registers a thread) so the next GEMV's CTA fits beside it on the SM:
-//    with programmatic dependent launch its copies are in flight while this
-//    GEMV computes;
+//    with programmatic dependent launch it starts early and its copies are in
+//    flight while this GEMV computes;
 //  * warps are KW "K slices" (2048 weights of K each: 32 lanes x one
 //    64-weight chunk) times RG row groups; in every block each warp takes UP
 //    rows, as straight-line code so their dot products interleave;
-//  * each lane turns its 64 activations into 16-bit fixed point with a
-//    power-of-two scale (|error| <= 2^-16 max|x_chunk|) and keeps them in
-//    registers; code bytes / nibble composites (layout.cuh) feed dp2a integer
-//    dot products (exact in int32); the group affine is applied once per chunk
-//    in fp32; the K slice's held-out entries add x~_c (v - lo_M) with the same
-//    fixed-point x~, so the result is exactly W_hat x~ up to fp32 rounding;
+//  * x is converted once per CTA to 16-bit fixed point with a power-of-two
+//    scale per 64-element chunk (|error| <= 2^-16 max|x_chunk|); each lane
+//    keeps its chunk's 64 activations in registers; code bytes / nibble
+//    composites (layout.cuh) feed dp2a integer dot products (exact in int32)
+//    and the group affine is applied once per chunk in fp32;
+//  * the held-out entries of the warp's rows in its K slice add
+//    x~_c (v - lo_M) with the same fixed-point x~, so the result is exactly
+//    W_hat x~ up to fp32 rounding;
 //  * a transposed shuffle reduces the UP rows to one partial per (row, K
 //    slice); the warp that finishes a block last (a shared-memory counter)
 //    adds the block's KW partials in a fixed order, stores y and refills the
@@ -48,6 +50,15 @@ namespace stagq {
 namespace {
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
+
+// x~ in shared memory: chunk c (64 int16) is 8 pieces of 16 bytes, piece p
+// stored at slot (p + c) mod 8, so that 32 lanes reading piece p of their own
+// chunks hit 8 different 16-byte bank groups instead of one.
+__device__ __forceinline__ int xq_piece(int c, int p) { return c * 8 + ((p + c) & 7); }
+__device__ __forceinline__ int xq_elem(int col) {
+  const int c = col >> 6, e = col & 63;
+  return xq_piece(c, e >> 3) * 8 + (e & 7);
+}
 
 
 // ------------------------------------------------------------ PTX helpers
@@ -221,7 +232,7 @@ constexpr uint64_t kDrainLimitNs = 100000000ull;   // after a failure: wait for 
 
 // Shared-memory carve-up, identical on host (plan) and device.
 struct SmemLayout {
-  uint32_t bar, cnt, last, tab, xq, xscale, xsum, partial, side, ring;
+  uint32_t bar, cnt, last, tab, xq, xscale, xsum, lo, partial, side, ring;
   uint32_t slot;                 // bytes of one ring slot
   uint32_t plane_piece, pair_piece;  // offsets inside a slot (base rows at 0)
   uint32_t total;
@@ -242,6 +253,7 @@ __host__ __device__ inline SmemLayout smem_layout(const GemvPlan& p, int in, int
   L.xscale = o; o += 4 * nchunk;
   L.xsum = o; o += 4 * nchunk;
   o = align_up_u32(o, 16);
+  L.lo = o; o += 4u * 32 * p.up * p.NW;  // per warp: lo_M of each lane's group per row of a block
   L.partial = o; o += 4u * p.ns * BR * p.KW;
   o = align_up_u32(o, 128);
   L.side = o; o += p.stage_side ? (uint32_t)p.side_stride : 0u;
@@ -284,32 +296,27 @@ __device__ __forceinline__ void rows_dot(const uint32_t (&X)[32], float xs, floa
 }
 
 // Held-out entries of NR consecutive rows of the warp's row class in its K
-// slice: entries [o[0], o[NR]) of the CTA's side record, row u owning
-// [o[u], o[u+1]). Adds x~_c (v - lo_M) to v[u]; lo_M comes from the lane
-// that owns column c (same K slice).
+// slice: row u owns entries [o_lo, o_hi) of the CTA's side record, handled by
+// the 32 / NR lanes of group u (lane / (32 / NR)). Adds x~_c (v - lo_M) to
+// v[u]; lo_M of column c's group is read from lo_s[u][c's lane], where every
+// lane of the warp left its own lo_M per row.
 template <int NR>
-__device__ __forceinline__ void side_record(const int (&o)[NR + 1], const uint32_t* ents, const int16_t* xq,
-                                            const float* xscale, int lane, const float (&lo)[NR], float (&v)[NR]) {
-  for (int j0 = o[0]; j0 < o[NR]; j0 += 32) {
-    const int j = j0 + lane;
-    const bool ok = j < o[NR];
-    const uint32_t en = ents[ok ? j : o[0]];
-    const int col = (int)(en & 0xFFFFu);
-    const int src = (col >> 6) & 31;
-    int u = 0;
-#pragma unroll
-    for (int i = 1; i < NR; ++i) u += j >= o[i];
-    float l = __shfl_sync(kFull, lo[0], src);
-#pragma unroll
-    for (int i = 1; i < NR; ++i) {
-      const float li = __shfl_sync(kFull, lo[i], src);
-      l = u == i ? li : l;
+__device__ __forceinline__ void side_record(int o_lo, int o_hi, const uint32_t* ents, const int16_t* xq,
+                                            const float* xscale, const float* lo_s, int lane, float (&v)[NR]) {
+  constexpr int LPR = 32 / NR;  // lanes per row
+  const int ur = lane / LPR;
+  const float* lo_row = lo_s + ur * 32;
+  float cs = 0.f;
+  for (int j = o_lo + lane % LPR; __any_sync(kFull, j < o_hi); j += LPR) {
+    if (j < o_hi) {
+      const uint32_t en = ents[j];
+      const int col = (int)(en & 0xFFFFu);
+      const float xv = (float)xq[xq_elem(col)] * xscale[col >> 6];
+      cs = fmaf(xv, __half2float(__ushort_as_half((unsigned short)(en >> 16))) - lo_row[(col >> 6) & 31], cs);
     }
-    const float xv = (float)xq[col] * xscale[col >> 6];
-    const float cs = ok ? xv * (__half2float(__ushort_as_half((unsigned short)(en >> 16))) - l) : 0.f;
-#pragma unroll
-    for (int i = 0; i < NR; ++i) v[i] += u == i ? cs : 0.f;
   }
+#pragma unroll
+  for (int i = 0; i < NR; ++i) v[i] += ur == i ? cs : 0.f;
 }
 
 template <int M, int UP>
@@ -325,6 +332,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
   float* xscale = reinterpret_cast<float*>(smem + L.xscale);
   float* xsum = reinterpret_cast<float*>(smem + L.xsum);
   float* partial = reinterpret_cast<float*>(smem + L.partial);  // [slot][BR][KW]
+  float* lo_w = reinterpret_cast<float*>(smem + L.lo) + 32 * UP * (threadIdx.x >> 5);
   uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + L.cnt);
   int* last = reinterpret_cast<int*>(smem + L.last);
   const uint32_t full0 = sbase + L.bar, side_bar = sbase + L.bar + 8 * kMaxSlots;
@@ -428,9 +436,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
         sumq += __shfl_xor_sync(kFull, sumq, 1);
         sumq += __shfl_xor_sync(kFull, sumq, 2);
         if (t < ntask) {
-          uint4* dst = reinterpret_cast<uint4*>(xq) + 2 * t;
-          dst[0] = make_uint4(Q[0], Q[1], Q[2], Q[3]);
-          dst[1] = make_uint4(Q[4], Q[5], Q[6], Q[7]);
+          uint4* dst = reinterpret_cast<uint4*>(xq);
+          dst[xq_piece(t >> 2, 2 * (t & 3))] = make_uint4(Q[0], Q[1], Q[2], Q[3]);
+          dst[xq_piece(t >> 2, 2 * (t & 3) + 1)] = make_uint4(Q[4], Q[5], Q[6], Q[7]);
           if ((t & 3) == 0) {
             const float xs_c = __int_as_float((127 - e) << 23);
             xscale[t >> 2] = xs_c;
@@ -444,10 +452,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
   uint32_t X[32];
   float xs, xsm;
   {
-    const uint4* src = reinterpret_cast<const uint4*>(xq) + cc * 8;
+    const uint4* src = reinterpret_cast<const uint4*>(xq);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const uint4 t = src[k];
+      const uint4 t = src[xq_piece(cc, k)];
       X[4 * k] = t.x;
       X[4 * k + 1] = t.y;
       X[4 * k + 2] = t.z;
@@ -482,10 +490,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
     if (mine == UP || 2 * mine > UP) {
       float v[UP], lo[UP];
       rows_dot<M, UP>(X, xs, xsm, sb, off, step, plane_stride, tab, v, lo);
-      int ob[UP + 1];
 #pragma unroll
-      for (int i = 0; i <= UP; ++i) ob[i] = o[i < mine ? i : mine];
-      side_record<UP>(ob, ents, xq, xscale, lane, lo, v);
+      for (int u = 0; u < UP; ++u) lo_w[u * 32 + lane] = lo[u];
+      __syncwarp();
+      const int ur = lane / (32 / UP);
+      side_record<UP>(o[ur < mine ? ur : mine], o[ur + 1 < mine ? ur + 1 : mine], ents, xq, xscale, lo_w, lane, v);
       const float s = transposed_reduce<UP>(v, lane);
       const int uu = lane / (32 / UP);
       if ((lane & (32 / UP - 1)) == 0 && uu < mine) pout[uu * RG * KW] = s;
@@ -494,12 +503,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
         float v[1], lo[1];
         const RowOffsets ou = {off.b + u * step.b, off.p + u * step.p, off.g + u * step.g};
         rows_dot<M, 1>(X, xs, xsm, sb, ou, step, plane_stride, tab, v, lo);
-        const int ob[2] = {o[u], o[u + 1]};
-        side_record<1>(ob, ents, xq, xscale, lane, lo, v);
+        lo_w[lane] = lo[0];
+        __syncwarp();
+        side_record<1>(o[u], o[u + 1], ents, xq, xscale, lo_w, lane, v);
         const float s = transposed_reduce<1>(v, lane);
         if (lane == 0) pout[u * RG * KW] = s;
       }
     }
+    __syncwarp();  // lo_w is rewritten by the next block
     // Done with the slot: the warp that finishes it last stores the block's
     // rows of y and refills the slot.
     __syncwarp();
@@ -626,8 +637,11 @@ uint32_t gemv_smem_bytes(const GemvPlan& plan, int in, int bits) { return smem_l
 int k_slices(int in) { return (in / kChunk + 31) / 32; }
 
 int gemv_grid(int out, int in, int num_sms) {
-  // two CTAs per SM while a CTA has <= 8 warps, else one
-  const int per_sm = k_slices(in) <= kMaxWarps / 2 ? kCtasPerSm : 1;
+  // Large matrices: two CTAs per SM (while a CTA has <= 8 warps), so one
+  // computes while the other starts or finishes. Small ones: one CTA per SM,
+  // which leaves room for the next GEMV's CTA to start early beside it.
+  const bool two = k_slices(in) <= kMaxWarps / 2 && (int64_t)out * in >= kTwoCtaWeightsPerSm * (int64_t)num_sms;
+  const int per_sm = two ? 2 : 1;
   int g = out < per_sm * num_sms ? out : per_sm * num_sms;
   if ((out + g - 1) / g > kMaxRowsPerCta) g = (out + kMaxRowsPerCta - 1) / kMaxRowsPerCta;
   return g;
@@ -652,7 +666,7 @@ bool make_plan(const DeviceMatrix& m, int bits, GemvPlan* p) {
   const int up_max = per_rg >= 4 ? 4 : per_rg >= 2 ? 2 : 1;
   // Shared memory: small enough for two CTAs per SM when the CTA has <= 8
   // warps, else (or if nothing fits) the per-block maximum. Prefer the side
-  // record staged, then at least four slots (or one per block), then more
+  // record staged, then at least three slots (or one per block), then more
   // rows per warp.
   const int budgets[2] = {q.NW <= kMaxWarps / 2 ? m.smem_pair_budget : m.smem_limit, m.smem_limit};
   for (int bi = 0; bi < 2; ++bi) {
@@ -668,7 +682,7 @@ bool make_plan(const DeviceMatrix& m, int bits, GemvPlan* p) {
         t.ns = nblk < kMaxSlots ? nblk : kMaxSlots;
         while (t.ns >= 1 && smem_layout(t, m.in, bits).total > (uint32_t)budgets[bi]) --t.ns;
         if (t.ns < 1) continue;
-        if (t.ns >= (nblk < 4 ? nblk : 4)) {
+        if (t.ns >= (nblk < 3 ? nblk : 3)) {
           *p = t;
           return true;
         }
