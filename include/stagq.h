@@ -198,6 +198,30 @@ int stagq_gemv_ex(stagq_handle h, int bits, const void* x, int n, void* y, uint3
 int stagq_gemv_host(stagq_handle h, int bits, const void* x_host, int n, void* y_host,
                     void* cuda_stream);
 
+/*
+ * As stagq_gemv_host, but allocates nothing: x and y are staged through a
+ * statically reserved device array of STAGQ_NOALLOC_STAGE_BYTES (x in its
+ * first 256 KiB, y in the rest), where stagq_gemv_host would cudaMalloc a
+ * staging buffer on first use. For callers that must not allocate device
+ * memory while they run: under a fixed device-memory budget owned by another
+ * allocator, or in a phase where new allocations are forbidden. The paper has
+ * no counterpart; this is a property of this library's host interface.
+ *   - The array exists on every GPU that loads the library and is held until
+ *     the process exits.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current (cudaGetSymbolAddress); make that first call before
+ *     any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents
+ *     (nothing of it is read before being written). Calls that overlap on the
+ *     GPU race: issue them one at a time. The call returns after the copy of y
+ *     has completed.
+ * Errors: as stagq_gemv_host; STAGQ_EINVAL when n*out*2 bytes of y exceed
+ * STAGQ_NOALLOC_STAGE_BYTES - 256 KiB (x always fits: n*in*2 <= 256 KiB).
+ */
+#define STAGQ_NOALLOC_STAGE_BYTES (2u << 20)
+int stagq_gemv_host_noalloc(stagq_handle h, int bits, const void* x_host, int n, void* y_host,
+                            void* cuda_stream);
+
 /* Test hook: u_M per weight (device [out*in] uint8, row-major), decoded on the GPU. */
 int stagq_decode_levels(stagq_handle h, int bits, uint8_t* u_dev, void* cuda_stream);
 

@@ -59,6 +59,7 @@ _SIGNATURES = {
     "stagq_gemv_n": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _c_p]),
     "stagq_gemv_ex": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _u32, _c_p]),
     "stagq_gemv_host": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _c_p]),
+    "stagq_gemv_host_noalloc": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _c_p]),
     "stagq_decode_levels": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, _c_p]),
     "stagq_bytes": (_i64, [_c_p, ctypes.c_int, ctypes.c_int]),
     "stagq_info": (ctypes.c_int, [_c_p, ctypes.POINTER(_Info)]),
@@ -286,6 +287,15 @@ def stagq_gemv_host(m: Matrix, bits: int, x_host: np.ndarray, y_host: np.ndarray
     """Host buffers (pinned or pageable numpy arrays): copies in and out, synchronous."""
     _check(lib().stagq_gemv_host(m.handle, bits, x_host.ctypes.data, n, y_host.ctypes.data,
                                  _stream_ptr(stream)), "stagq_gemv_host")
+
+
+def stagq_gemv_host_noalloc(m: Matrix, bits: int, x_host: np.ndarray, y_host: np.ndarray, n: int = 1,
+                            stream=None) -> None:
+    """As stagq_gemv_host, staging through the library's static device array
+    instead of a device buffer allocated on first use (no device allocation).
+    Calls must not overlap on the GPU; see include/stagq.h."""
+    _check(lib().stagq_gemv_host_noalloc(m.handle, bits, x_host.ctypes.data, n, y_host.ctypes.data,
+                                         _stream_ptr(stream)), "stagq_gemv_host_noalloc")
 
 
 def stagq_decode_levels(m: Matrix, bits: int, u_dev, stream=None) -> None:

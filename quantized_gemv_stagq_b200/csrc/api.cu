@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <mutex>
 #include <cstring>
 #include <new>
 #include <string>
@@ -333,4 +334,75 @@ extern "C" void stagq_free(stagq_handle h) {
   if (h->d_mem) cudaFree(h->d_mem);
   if (h->d_stage) cudaFree(h->d_stage);
   delete h;
+}
+
+// ---------------------------------------------------------------------------
+// Host-buffer GEMV that allocates no device memory.
+//
+// stagq_gemv_host stages x and y in a device buffer that the handle allocates
+// with cudaMalloc on first use. Some callers must not allocate at that point:
+// code that runs under a fixed device-memory budget owned by another
+// allocator, or in a phase where any new allocation is forbidden. This
+// variant stages through kNoAllocStageBytes of statically reserved device
+// memory instead (x at offset 0, y at kNoAllocXBytes). Every GPU that loads
+// this library holds the array until the process exits.
+namespace stagq {
+namespace {
+
+constexpr size_t kNoAllocXBytes = (size_t)STAGQ_MAX_BATCH * STAGQ_MAX_IN * 2;       // 256 KiB: any x
+constexpr size_t kNoAllocStageBytes = (size_t)STAGQ_NOALLOC_STAGE_BYTES;            // x and y together
+
+static __device__ __align__(256) uint8_t g_noalloc_stage[kNoAllocStageBytes];
+
+// Device address of g_noalloc_stage on each device. In host code the array's
+// name is only a host-side stand-in, so the address is taken once per device
+// with that device current.
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+int noalloc_stage(int device, uint8_t** out) {
+  if (device < 0 || device >= kNoAllocMaxDevices) return fail(STAGQ_EINVAL, "device index out of range");
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[device]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_stage);
+    if (e != cudaSuccess || !p) return cuda_fail(e == cudaSuccess ? cudaErrorInvalidSymbol : e, "cudaGetSymbolAddress");
+    g_noalloc_ptr[device] = p;
+  }
+  *out = static_cast<uint8_t*>(g_noalloc_ptr[device]);
+  return STAGQ_OK;
+}
+
+}  // namespace
+}  // namespace stagq
+
+extern "C" int stagq_gemv_host_noalloc(stagq_handle h, int bits, const void* x_host, int n, void* y_host,
+                                       void* cuda_stream) {
+  int st = check_handle_bits(h, bits);
+  if (st) return st;
+  if (!x_host || !y_host) return fail(STAGQ_EINVAL, "null x or y");
+  if (n < 1 || n > STAGQ_MAX_BATCH) return fail(STAGQ_EINVAL, "n outside 1..STAGQ_MAX_BATCH");
+  const size_t xb = (size_t)n * h->dm.in * 2, yb = (size_t)n * h->dm.out * 2;
+  if (xb > kNoAllocXBytes || yb > kNoAllocStageBytes - kNoAllocXBytes)
+    return fail(STAGQ_EINVAL, "n * out * 2 exceeds the static staging area (STAGQ_NOALLOC_STAGE_BYTES - 256 KiB)");
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return fail(STAGQ_ECUDA, "cudaSetDevice failed");
+  uint8_t* stage = nullptr;
+  st = noalloc_stage(h->device, &stage);
+  if (st) return st;
+  uint8_t* dx = stage;
+  uint8_t* dy = stage + kNoAllocXBytes;
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  // x is overwritten in full and the kernel writes every element of y, so
+  // nothing left in the array by an earlier call is read.
+  cudaError_t e = cudaMemcpyAsync(dx, x_host, xb, cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "copy of x");
+  st = stagq_gemv_ex(h, bits, dx, n, dy, 0u, cuda_stream);
+  if (st) return st;
+  e = cudaMemcpyAsync(y_host, dy, yb, cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "copy of y");
+  e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  return STAGQ_OK;
 }
