@@ -17,8 +17,8 @@
 struct stagq_matrix {
   int device = -1;
   stagq::DeviceMatrix dm{};
-  stagq::GemvPlan plan[7]{};     // per precision (index = bits)
-  bool plan_ok[7]{};
+  stagq::GemvPlan plan[7][STAGQ_MAX_BATCH + 1]{};  // per precision (bits) and vector count
+  bool plan_ok[7][STAGQ_MAX_BATCH + 1]{};
   void* d_mem = nullptr;
   size_t d_bytes = 0;
   void* d_stage = nullptr;      // x / y staging for stagq_gemv_host
@@ -203,8 +203,9 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   m.num_sms = prop.multiProcessorCount;
   m.smem_pair_budget = smem_sm / 2 - smem_reserved;
   if (m.smem_pair_budget > smem_limit) m.smem_pair_budget = smem_limit;
-  for (int b = 2; b <= 2 + np; ++b) h->plan_ok[b] = make_plan(m, b, &h->plan[b]);
-  if (!h->plan_ok[2]) {
+  for (int b = 2; b <= 2 + np; ++b)
+    for (int nb = 1; nb <= STAGQ_MAX_BATCH; ++nb) h->plan_ok[b][nb] = make_plan(m, b, nb, &h->plan[b][nb]);
+  if (!h->plan_ok[2][1]) {
     cudaFree(h->d_mem);
     delete h;
     return fail(STAGQ_EINVAL, "shape cannot be planned on this device");
@@ -233,11 +234,16 @@ extern "C" int stagq_gemv_ex(stagq_handle h, int bits, const void* x, int n, voi
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   const int yf32 = (flags & STAGQ_Y_F32) ? 1 : 0;
   const size_t ysz = yf32 ? 4 : 2;
-  if (!h->plan_ok[bits]) return fail(STAGQ_EINVAL, "no launch plan for this precision");
-  for (int j = 0; j < n; ++j) {
+  if (h->plan_ok[bits][n]) {  // one launch: the weights are read once for all n vectors
+    cudaError_t e = launch_gemv(h->dm, h->plan[bits][n], bits, x, y, yf32, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMV launch");
+    return STAGQ_OK;
+  }
+  if (!h->plan_ok[bits][1]) return fail(STAGQ_EINVAL, "no launch plan for this precision");
+  for (int j = 0; j < n; ++j) {  // shapes whose n-vector plan does not fit: one launch per vector
     const void* xj = static_cast<const uint8_t*>(x) + (size_t)j * h->dm.in * 2;
     void* yj = static_cast<uint8_t*>(y) + (size_t)j * h->dm.out * ysz;
-    cudaError_t e = launch_gemv(h->dm, h->plan[bits], bits, xj, yj, yf32, stream);
+    cudaError_t e = launch_gemv(h->dm, h->plan[bits][1], bits, xj, yj, yf32, stream);
     if (e != cudaSuccess) return cuda_fail(e, "GEMV launch");
   }
   return STAGQ_OK;

@@ -50,15 +50,18 @@ struct GemvPlan {
   int group_shift;       // log2(group)
   int pair_stride;
   int pdl;               // launch with programmatic dependent launch
+  int nb;                // activation vectors per launch (1..4; the weights are read once)
 };
 
-// Plan for a GEMV at `bits`; returns false if the shape cannot be planned.
-bool make_plan(const DeviceMatrix& m, int bits, GemvPlan* plan);
+// Plan for a GEMV at `bits` with `nb` activation vectors; false if the shape
+// cannot be planned.
+bool make_plan(const DeviceMatrix& m, int bits, int nb, GemvPlan* plan);
 int k_slices(int in);
 int gemv_grid(int out, int in, int num_sms);
 uint32_t gemv_smem_bytes(const GemvPlan& plan, int in, int bits);
 
-// y = W_hat^(bits) x for n = 1. y is fp16 (y_f32 = 0) or fp32.
+// y = W_hat^(bits) x for plan.nb vectors (x [nb][in], y [nb][out]). y is fp16
+// (y_f32 = 0) or fp32.
 cudaError_t launch_gemv(const DeviceMatrix& m, const GemvPlan& plan, int bits, const void* x, void* y,
                         int y_f32, cudaStream_t stream);
 

@@ -249,12 +249,12 @@ __host__ __device__ inline SmemLayout smem_layout(const GemvPlan& p, int in, int
   L.last = o; o += 4 * kMaxSlots;        // last block issued into the slot
   o = align_up_u32(o, 16);
   L.tab = o; o += 256 * 8;
-  L.xq = o; o += 2 * in;
-  L.xscale = o; o += 4 * nchunk;
-  L.xsum = o; o += 4 * nchunk;
+  L.xq = o; o += 2u * in * p.nb;        // x~ of each of the nb vectors
+  L.xscale = o; o += 4u * nchunk * p.nb;
+  L.xsum = o; o += 4u * nchunk * p.nb;
   o = align_up_u32(o, 16);
   L.lo = o; o += 4u * 32 * p.up * p.NW;  // per warp: lo_M of each lane's group per row of a block
-  L.partial = o; o += 4u * p.ns * BR * p.KW;
+  L.partial = o; o += 4u * p.ns * BR * p.KW * p.nb;  // [slot][BR][KW][nb]
   o = align_up_u32(o, 128);
   L.side = o; o += p.stage_side ? (uint32_t)p.side_stride : 0u;
   o = align_up_u32(o, 128);
@@ -295,6 +295,50 @@ __device__ __forceinline__ void rows_dot(const uint32_t (&X)[32], float xs, floa
   }
 }
 
+// As rows_dot for NB activation vectors (NB > 1): the slot's code words are
+// read once and dotted with each vector's x~, which is taken from shared
+// memory vector by vector (x~ of vector j at xq + j * in, its chunk scales at
+// xscale / xsum + j * nchunk). v[j][u] is row u against vector j.
+template <int M, int NR, int NB>
+__device__ __forceinline__ void rows_dot_nb(const int16_t* xq, const float* xscale, const float* xsum, int in,
+                                            int nchunk, int cc, bool active, const uint8_t* sb, RowOffsets off,
+                                            RowOffsets step, uint32_t plane_stride, const float2* tab,
+                                            float (&v)[NB][NR], float (&lo)[NR]) {
+  uint32_t B[NR][4];
+  uint2 Pw[NR][M > 2 ? M - 2 : 1];
+  float2 lm[NR];
+#pragma unroll
+  for (int u = 0; u < NR; ++u) {
+    const uint4 b4 = *reinterpret_cast<const uint4*>(sb + off.b + u * step.b);
+    B[u][0] = b4.x; B[u][1] = b4.y; B[u][2] = b4.z; B[u][3] = b4.w;
+#pragma unroll
+    for (int k = 0; k < M - 2; ++k)
+      Pw[u][k] = *reinterpret_cast<const uint2*>(sb + off.p + u * step.p + k * plane_stride);
+    lm[u] = tab[sb[off.g + u * step.g]];
+    lo[u] = lm[u].x;
+  }
+#pragma unroll
+  for (int j = 0; j < NB; ++j) {
+    uint32_t X[32];
+    const uint4* src = reinterpret_cast<const uint4*>(xq + j * in);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint4 t = src[xq_piece(cc, k)];
+      X[4 * k] = t.x;
+      X[4 * k + 1] = t.y;
+      X[4 * k + 2] = t.z;
+      X[4 * k + 3] = t.w;
+    }
+    const float xs = active ? xscale[j * nchunk + cc] : 0.f;
+    const float xsm = active ? xsum[j * nchunk + cc] : 0.f;
+#pragma unroll
+    for (int u = 0; u < NR; ++u) {
+      const int tot = chunk_dot<M>(X, B[u], Pw[u]);
+      v[j][u] = fmaf(lm[u].y, (float)tot * xs, lm[u].x * xsm);
+    }
+  }
+}
+
 // Held-out entries of NR consecutive rows of the warp's row class in its K
 // slice: row u owns entries [o_lo, o_hi) of the CTA's side record, handled by
 // the 32 / NR lanes of group u (lane / (32 / NR)). Adds x~_c (v - lo_M) to
@@ -319,7 +363,66 @@ __device__ __forceinline__ void side_record(int o_lo, int o_hi, const uint32_t* 
   for (int i = 0; i < NR; ++i) v[i] += ur == i ? cs : 0.f;
 }
 
-template <int M, int UP>
+// As side_record for NB activation vectors: v[j][u] += x~_j,c (v - lo_M).
+template <int NR, int NB>
+__device__ __forceinline__ void side_record_nb(int o_lo, int o_hi, const uint32_t* ents, const int16_t* xq,
+                                               const float* xscale, int in, int nchunk, const float* lo_s, int lane,
+                                               float (&v)[NB][NR]) {
+  constexpr int LPR = 32 / NR;  // lanes per row
+  const int ur = lane / LPR;
+  const float* lo_row = lo_s + ur * 32;
+  float cs[NB];
+#pragma unroll
+  for (int j = 0; j < NB; ++j) cs[j] = 0.f;
+  for (int e = o_lo + lane % LPR; __any_sync(kFull, e < o_hi); e += LPR) {
+    if (e < o_hi) {
+      const uint32_t en = ents[e];
+      const int col = (int)(en & 0xFFFFu);
+      const float d = __half2float(__ushort_as_half((unsigned short)(en >> 16))) - lo_row[(col >> 6) & 31];
+      const int xe = xq_elem(col);
+#pragma unroll
+      for (int j = 0; j < NB; ++j) cs[j] = fmaf((float)xq[j * in + xe] * xscale[j * nchunk + (col >> 6)], d, cs[j]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < NB; ++j)
+#pragma unroll
+    for (int i = 0; i < NR; ++i) v[j][i] += ur == i ? cs[j] : 0.f;
+}
+
+// The UP rows (or, for a short block, `mine` rows one at a time) of one block
+// for this lane's chunk: dot products, side record, and the cross-lane sums
+// into pout[u * pstep + j] (row u, vector j).
+template <int M, int NR, int NB>
+__device__ __forceinline__ void block_rows(const uint32_t (&X)[32], float xs, float xsm, const int16_t* xq,
+                                           const float* xscale, const float* xsum, int in, int nchunk, int cc,
+                                           bool active, const uint8_t* sb, RowOffsets off, RowOffsets step,
+                                           uint32_t plane_stride, const float2* tab, int mine, const int32_t* o,
+                                           const uint32_t* ents, float* lo_w, int lane, float* pout, int pstep) {
+  float v[NB][NR], lo[NR];
+  if constexpr (NB == 1) {
+    rows_dot<M, NR>(X, xs, xsm, sb, off, step, plane_stride, tab, v[0], lo);
+  } else {
+    rows_dot_nb<M, NR, NB>(xq, xscale, xsum, in, nchunk, cc, active, sb, off, step, plane_stride, tab, v, lo);
+  }
+#pragma unroll
+  for (int u = 0; u < NR; ++u) lo_w[u * 32 + lane] = lo[u];
+  __syncwarp();
+  const int ur = lane / (32 / NR);
+  if constexpr (NB == 1) {
+    side_record<NR>(o[ur < mine ? ur : mine], o[ur + 1 < mine ? ur + 1 : mine], ents, xq, xscale, lo_w, lane, v[0]);
+  } else {
+    side_record_nb<NR, NB>(o[ur < mine ? ur : mine], o[ur + 1 < mine ? ur + 1 : mine], ents, xq, xscale, in, nchunk,
+                           lo_w, lane, v);
+  }
+#pragma unroll
+  for (int j = 0; j < NB; ++j) {
+    const float s = transposed_reduce<NR>(v[j], lane);
+    if ((lane & (32 / NR - 1)) == 0 && ur < mine) pout[ur * pstep + j] = s;
+  }
+}
+
+template <int M, int UP, int NB>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKernelArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const GemvPlan& P = a.plan;
@@ -396,7 +499,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
   {
     constexpr float kShift = 12582912.0f;
     constexpr int kBatch = 4;
-    const int ntask = 4 * nchunk;
+    const int tpv = 4 * nchunk;  // tasks per vector
+    const int ntask = tpv * NB;
     const uint4* x4 = reinterpret_cast<const uint4*>(a.x);
     for (int t0 = 0; t0 < ntask; t0 += kBatch * nthreads) {
       uint4 raw[kBatch][2];
@@ -404,7 +508,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
       for (int q = 0; q < kBatch; ++q) {
         const int t = t0 + q * nthreads + tid;
         raw[q][0] = raw[q][1] = make_uint4(0u, 0u, 0u, 0u);
-        if (t < ntask) {
+        if (t < ntask) {  // x is [NB][in]: task t of the flat list reads 16 values from 16 t on
           raw[q][0] = __ldg(x4 + 2 * t);
           raw[q][1] = __ldg(x4 + 2 * t + 1);
         }
@@ -436,22 +540,23 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
         sumq += __shfl_xor_sync(kFull, sumq, 1);
         sumq += __shfl_xor_sync(kFull, sumq, 2);
         if (t < ntask) {
-          uint4* dst = reinterpret_cast<uint4*>(xq);
-          dst[xq_piece(t >> 2, 2 * (t & 3))] = make_uint4(Q[0], Q[1], Q[2], Q[3]);
-          dst[xq_piece(t >> 2, 2 * (t & 3) + 1)] = make_uint4(Q[4], Q[5], Q[6], Q[7]);
-          if ((t & 3) == 0) {
+          const int j = t / tpv, tt = t - j * tpv;  // vector, task within it
+          uint4* dst = reinterpret_cast<uint4*>(xq + j * in);
+          dst[xq_piece(tt >> 2, 2 * (tt & 3))] = make_uint4(Q[0], Q[1], Q[2], Q[3]);
+          dst[xq_piece(tt >> 2, 2 * (tt & 3) + 1)] = make_uint4(Q[4], Q[5], Q[6], Q[7]);
+          if ((tt & 3) == 0) {
             const float xs_c = __int_as_float((127 - e) << 23);
-            xscale[t >> 2] = xs_c;
-            xsum[t >> 2] = xs_c * (float)sumq;
+            xscale[j * nchunk + (tt >> 2)] = xs_c;
+            xsum[j * nchunk + (tt >> 2)] = xs_c * (float)sumq;
           }
         }
       }
     }
   }
   __syncthreads();
-  uint32_t X[32];
-  float xs, xsm;
-  {
+  uint32_t X[32];  // one vector: this lane's x~ stays in registers (more vectors: read per block)
+  float xs = 0.f, xsm = 0.f;
+  if constexpr (NB == 1) {
     const uint4* src = reinterpret_cast<const uint4*>(xq);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
@@ -482,32 +587,21 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
     }
     const uint8_t* sb = ring_g + slot * L.slot;
     const int nr = min(BR, rows - b * BR);
-    float* pout = partial + (slot * BR + rg) * KW + kw;
+    float* pout = partial + ((slot * BR + rg) * KW + kw) * NB;
+    const int pstep = RG * KW * NB;
     const int32_t* o = seg + UP * b;  // this block's rows of the class
     // my rows in this block; a short block runs as a full one with the
     // missing rows masked, unless fewer than half of them are there
     const int mine = nr == BR ? UP : (nr > rg ? (nr - rg + RG - 1) / RG : 0);
     if (mine == UP || 2 * mine > UP) {
-      float v[UP], lo[UP];
-      rows_dot<M, UP>(X, xs, xsm, sb, off, step, plane_stride, tab, v, lo);
-#pragma unroll
-      for (int u = 0; u < UP; ++u) lo_w[u * 32 + lane] = lo[u];
-      __syncwarp();
-      const int ur = lane / (32 / UP);
-      side_record<UP>(o[ur < mine ? ur : mine], o[ur + 1 < mine ? ur + 1 : mine], ents, xq, xscale, lo_w, lane, v);
-      const float s = transposed_reduce<UP>(v, lane);
-      const int uu = lane / (32 / UP);
-      if ((lane & (32 / UP - 1)) == 0 && uu < mine) pout[uu * RG * KW] = s;
+      block_rows<M, UP, NB>(X, xs, xsm, xq, xscale, xsum, in, nchunk, cc, active, sb, off, step, plane_stride, tab,
+                            mine, o, ents, lo_w, lane, pout, pstep);
     } else {
       for (int u = 0; u < mine; ++u) {
-        float v[1], lo[1];
         const RowOffsets ou = {off.b + u * step.b, off.p + u * step.p, off.g + u * step.g};
-        rows_dot<M, 1>(X, xs, xsm, sb, ou, step, plane_stride, tab, v, lo);
-        lo_w[lane] = lo[0];
-        __syncwarp();
-        side_record<1>(o[u], o[u + 1], ents, xq, xscale, lo_w, lane, v);
-        const float s = transposed_reduce<1>(v, lane);
-        if (lane == 0) pout[u * RG * KW] = s;
+        block_rows<M, 1, NB>(X, xs, xsm, xq, xscale, xsum, in, nchunk, cc, active, sb, ou, step, plane_stride, tab,
+                             1, o + u, ents, lo_w, lane, pout + u * pstep, pstep);
+        __syncwarp();  // lo_w is rewritten by the next row
       }
     }
     __syncwarp();  // lo_w is rewritten by the next block
@@ -523,11 +617,15 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
     if (done == (uint32_t)NW * (round + 1)) {
       __threadfence_block();
       if (lane < nr) {
-        const float* pr = partial + (slot * BR + lane) * KW;
-        float acc = 0.f;
-        for (int k = 0; k < KW; ++k) acc += pr[k];
-        if (a.y_f32) reinterpret_cast<float*>(a.y)[r0 + b * BR + lane] = acc;
-        else reinterpret_cast<__half*>(a.y)[r0 + b * BR + lane] = __float2half_rn(acc);
+        const float* pr = partial + (slot * BR + lane) * KW * NB;
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+          float acc = 0.f;
+          for (int k = 0; k < KW; ++k) acc += pr[k * NB + j];
+          const int64_t yi = (int64_t)j * a.m.out + r0 + b * BR + lane;
+          if (a.y_f32) reinterpret_cast<float*>(a.y)[yi] = acc;
+          else reinterpret_cast<__half*>(a.y)[yi] = __float2half_rn(acc);
+        }
       }
       __syncwarp();
       if (lane == 0 && b + NS < nblk) issue_block(b + NS, slot);
@@ -571,7 +669,7 @@ __global__ void decode_levels_kernel(const DeviceMatrix m, uint8_t* u) {
 cudaError_t ensure_smem(const void* kern, int key, size_t smem) {
   constexpr int kMaxDev = 64;
   static std::mutex mu;
-  static size_t granted[kMaxDev][64] = {};
+  static size_t granted[kMaxDev][64] = {};  // key < 60: (M - 2, rows per warp, vectors)
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
@@ -583,7 +681,7 @@ cudaError_t ensure_smem(const void* kern, int key, size_t smem) {
   return err;
 }
 
-template <int M, int UP>
+template <int M, int UP, int NB>
 cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const void* x, void* y, int y_f32,
                            cudaStream_t stream) {
   GemvKernelArgs a;
@@ -594,8 +692,9 @@ cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const vo
   a.y = y;
   a.y_f32 = y_f32;
   const SmemLayout L = smem_layout(plan, m.in, M);
-  auto kern = gemv_kernel<M, UP>;
-  cudaError_t err = ensure_smem(reinterpret_cast<const void*>(kern), (M - 2) * 3 + (UP == 4 ? 2 : UP - 1), L.total);
+  auto kern = gemv_kernel<M, UP, NB>;
+  const int key = ((M - 2) * 3 + (UP == 4 ? 2 : UP - 1)) * 4 + (NB - 1);
+  cudaError_t err = ensure_smem(reinterpret_cast<const void*>(kern), key, L.total);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)plan.grid);
@@ -613,11 +712,34 @@ cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const vo
 template <int M>
 cudaError_t launch_gemv_m(const DeviceMatrix& m, const GemvPlan& plan, const void* x, void* y, int y_f32,
                           cudaStream_t stream) {
-  switch (plan.up) {
-    case 1: return launch_gemv_mu<M, 1>(m, plan, x, y, y_f32, stream);
-    case 2: return launch_gemv_mu<M, 2>(m, plan, x, y, y_f32, stream);
-    case 4: return launch_gemv_mu<M, 4>(m, plan, x, y, y_f32, stream);
-    default: return cudaErrorInvalidValue;
+  // Instances the planner can select (see make_plan): more vectors or deeper
+  // reads take fewer rows per warp, so that the registers do not spill.
+  if (plan.nb == 1) {
+    if (plan.up == 1) return launch_gemv_mu<M, 1, 1>(m, plan, x, y, y_f32, stream);
+    if (plan.up == 2) return launch_gemv_mu<M, 2, 1>(m, plan, x, y, y_f32, stream);
+    if (plan.up == 4) return launch_gemv_mu<M, 4, 1>(m, plan, x, y, y_f32, stream);
+    return cudaErrorInvalidValue;
+  }
+  if constexpr (M >= 5) {
+    if (plan.up != 1) return cudaErrorInvalidValue;
+    switch (plan.nb) {
+      case 2: return launch_gemv_mu<M, 1, 2>(m, plan, x, y, y_f32, stream);
+      case 3: return launch_gemv_mu<M, 1, 3>(m, plan, x, y, y_f32, stream);
+      case 4: return launch_gemv_mu<M, 1, 4>(m, plan, x, y, y_f32, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  } else {
+    const int k = (plan.up == 4 ? 2 : plan.up - 1) * 4 + plan.nb;
+    switch (k) {
+      case 2: return launch_gemv_mu<M, 1, 2>(m, plan, x, y, y_f32, stream);
+      case 3: return launch_gemv_mu<M, 1, 3>(m, plan, x, y, y_f32, stream);
+      case 4: return launch_gemv_mu<M, 1, 4>(m, plan, x, y, y_f32, stream);
+      case 6: return launch_gemv_mu<M, 2, 2>(m, plan, x, y, y_f32, stream);
+      case 7: return launch_gemv_mu<M, 2, 3>(m, plan, x, y, y_f32, stream);
+      case 8: return launch_gemv_mu<M, 2, 4>(m, plan, x, y, y_f32, stream);
+      case 10: return launch_gemv_mu<M, 4, 2>(m, plan, x, y, y_f32, stream);
+      default: return cudaErrorInvalidValue;
+    }
   }
 }
 
@@ -647,8 +769,10 @@ int gemv_grid(int out, int in, int num_sms) {
   return g;
 }
 
-bool make_plan(const DeviceMatrix& m, int bits, GemvPlan* p) {
+bool make_plan(const DeviceMatrix& m, int bits, int nb, GemvPlan* p) {
   GemvPlan q = {};
+  if (nb < 1 || nb > 4) return false;
+  q.nb = nb;
   q.KW = k_slices(m.in);
   if (q.KW < 1 || q.KW > kMaxWarps) return false;
   q.RG = row_groups(q.KW);
@@ -663,7 +787,10 @@ bool make_plan(const DeviceMatrix& m, int bits, GemvPlan* p) {
   q.pdl = 1;
   // Rows per warp per block: up to 4, but no more than the CTA's rows call for.
   const int per_rg = (q.rows_cap + q.RG - 1) / q.RG;
-  const int up_max = per_rg >= 4 ? 4 : per_rg >= 2 ? 2 : 1;
+  int up_max = per_rg >= 4 ? 4 : per_rg >= 2 ? 2 : 1;
+  // registers: rows x vectors x planes (the instances launch_gemv_m provides)
+  if (nb >= 2 && bits >= 5) up_max = 1;
+  else if (nb >= 3 && up_max > 2) up_max = 2;
   // Shared memory: small enough for two CTAs per SM when the CTA has <= 8
   // warps, else (or if nothing fits) the per-block maximum. Prefer the side
   // record staged, then at least three slots (or one per block), then more

@@ -79,6 +79,27 @@ def test_gemv_matches_oracle(case):
     m.free()
 
 
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}x{c[1]}g{c[2]}p{c[3]}d{c[4]}")
+def test_batched_gemv_matches_oracle(case):
+    """n = 2..4 activation vectors in one launch (the weights are read once):
+    every column against the oracle, at every precision of the stream."""
+    out, inp, g, npl, dens, mode, seed = case
+    F = O.encode(synth.weights(out, inp, seed), g, npl, dens, mode)
+    m = _load(F)
+    for n in (2, 3, 4):
+        x = synth.activations(n, inp, seed + 200 + n)
+        for M in range(2, 3 + npl):
+            ref = O.gemv(F, M, x)
+            got = _gemv(m, M, x, f32=True)
+            for j in range(n):
+                check_close(got[j], ref[j], f"n{n} col{j} p{M}")
+            # each column equals the single-vector launch of that column (same kernel arithmetic)
+            one = _gemv(m, M, x[n - 1:n], f32=True)
+            check_close(got[n - 1:n], one, f"n{n} last col vs n1 p{M}")
+    Q.stagq_check(m)
+    m.free()
+
+
 def test_gemv_activation_edge_cases():
     out, inp = 256, 2048
     F = O.encode(synth.weights(out, inp, 11), 128, 2, 0.005, "fast")
@@ -177,10 +198,14 @@ def test_full_size_llama_sampled_rows(name, shape):
                     np.concatenate([P.val[P.row_ptr[r]:P.row_ptr[r + 1]] for r in rows]))
     eq = fields_equal(F, Psub)
     assert all(eq.values()), eq
-    x = synth.activations(1, inp, seed=7)
+    x = synth.activations(4, inp, seed=7)
     for M in (2, 3, 4):
-        y = _gemv(m, M, x, f32=False)[0]
-        check_close(y[rows].astype(np.float64), O.gemv(F, M, x)[0], f"{name} p{M}")
+        y = _gemv(m, M, x[:1], f32=False)[0]
+        check_close(y[rows].astype(np.float64), O.gemv(F, M, x[:1])[0], f"{name} p{M}")
         assert np.all(np.isfinite(y))
+        y4 = _gemv(m, M, x, f32=False)  # batch 4 in one launch
+        ref4 = O.gemv(F, M, x)
+        for j in range(4):
+            check_close(y4[j][rows].astype(np.float64), ref4[j], f"{name} p{M} n4 col{j}")
     Q.stagq_check(m)
     m.free()
