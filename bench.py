@@ -13,6 +13,16 @@ device time, in GB/s. Per-GEMV microseconds for every shape and precision are
 in ``per_gemv``.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl stagq|reference]
+                  [--workload llama31_8b_linears_b1 | phi4_olmo2_linears_b1 | precision_sweep | llama31_8b_stack]
+
+The default workload is the Llama-3.1-8B layer above. The others print one
+JSON line each with per-GEMV (or per-token) times:
+  phi4_olmo2_linears_b1  Phi-4 and OLMo-2-7B linears at 2/3/4 bits, batch 1;
+  precision_sweep        14336x4096 and 4096x14336 with base + 4 planes, read at
+                         2..6 bits, group 64 and 128, side record 0 / 0.1 / 1 %;
+  llama31_8b_stack       32 layers x 7 linears (6.98e9 weights) resident on the
+                         GPU, per-token GEMV time at batch 1 and 4, 2/3/4 bits
+                         read from one stored stream.
 """
 from __future__ import annotations
 
@@ -46,6 +56,10 @@ def _args():
     p.add_argument("--impl", default="stagq", choices=["stagq", "reference"])
     p.add_argument("--copies", type=int, default=6, help="device copies of the layer rotated over")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--workload", default=WORKLOAD,
+                   choices=[WORKLOAD, "phi4_olmo2_linears_b1", "precision_sweep", "llama31_8b_stack"])
+    p.add_argument("--stack-distinct", type=int, default=4,
+                   help="llama31_8b_stack: distinct encoded layers (the 32 resident layers cycle over them)")
     return p.parse_args()
 
 
@@ -206,6 +220,157 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------ GPU arm
+
+def time_gemv(Q, torch, mats, bits, x, y, n, stream, reps=24, repeats=5):
+    """Device time of one GEMV (µs): a CUDA graph of `reps` launches rotating
+    over the device copies in `mats` (so reads come from HBM), replayed
+    `repeats` times between CUDA events; median over 3 such measurements."""
+    C = len(mats)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        Q.stagq_gemv_n(mats[0], bits, x, n, y, stream=stream)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=stream):
+        for r in range(reps):
+            Q.stagq_gemv_n(mats[(r + 1) % C], bits, x, n, y, stream=stream)
+    g.replay()
+    torch.cuda.synchronize()
+    out = []
+    for _ in range(3):
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a0.record(stream)
+            for _ in range(repeats):
+                g.replay()
+            a1.record(stream)
+        torch.cuda.synchronize()
+        out.append(a0.elapsed_time(a1) * 1e3 / (repeats * reps))
+    del g
+    return statistics.median(out)
+
+
+def copies_for(Q, stored_bytes, l2, minimum=3):
+    """Device copies so that one pass over them is at least 4x the L2 size."""
+    return max(minimum, int(4 * l2 // max(stored_bytes, 1)) + 1)
+
+
+def _extra_line(args, workload, results, extra_cfg, clocks, peak, peak_kind, value, unit, gemvs):
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": 1, "steps": None, "warmup": None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int32 dot (u8 codes x i16 x) + fp32", "data": "synthetic",
+        "config": dict({"workload": workload}, **extra_cfg), "results": results,
+        "peak": {"hbm_gbs": peak, "kind": peak_kind}, "gpu_launches": gemvs, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_extra(args):
+    """The other measured workloads (one JSON line each)."""
+    import torch
+    import quantized_gemv_stagq_b200 as Q
+    from quantized_gemv_stagq_b200 import synth
+    torch.cuda.set_device(0)
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    peak, peak_kind = _peaks()
+    stream = torch.cuda.Stream()
+    clocks = ClockSampler(0)
+    clocks.start()
+    results = {}
+    launches = 0
+
+    def per_gemv(shapes, bits_list, group, n_planes, density, batch=1, tag=""):
+        nonlocal launches
+        for name, (out, inp) in shapes:
+            S = Q.stagq_pack(Q.stagq_encode(synth.weights(out, inp, seed=out + 3 * inp), group, n_planes,
+                                            density, "fast"))
+            m0 = Q.stagq_load(S, 0)
+            C = copies_for(Q, m0.device_bytes, l2)
+            mats = [m0] + [Q.stagq_load(S, 0) for _ in range(C - 1)]
+            x = torch.from_numpy(synth.activations(batch, inp, seed=inp)).cuda()
+            y = torch.empty(batch, out, dtype=torch.float16, device="cuda")
+            for b in bits_list:
+                us = time_gemv(Q, torch, mats, b, x, y, batch, stream)
+                launches += 24 * 5 * 3
+                nb = Q.stagq_bytes(m0, b, batch)
+                results[f"{tag}{name} {out}x{inp} p{b}"] = {"us": round(us, 3), "bytes": nb,
+                                                           "gbs": round(nb / us / 1e3, 1),
+                                                           "frac": round(nb / us / 1e3 / peak, 4)}
+            for m in mats:
+                m.free()
+            del S
+
+    if args.workload == "phi4_olmo2_linears_b1":
+        shapes = [("phi4." + k, v) for k, v in synth.PHI4_LINEARS.items()] + \
+                 [("olmo2." + k, v) for k, v in synth.OLMO2_7B_LINEARS.items()]
+        per_gemv(shapes, BITS, GROUP, N_PLANES, DENSITY)
+        cfg = {"linears_out_x_in": {k: list(v) for k, v in shapes}, "bits": list(BITS), "group": GROUP,
+               "n_planes": N_PLANES, "side_record_density": DENSITY, "batch": 1}
+    elif args.workload == "precision_sweep":
+        shapes = [("gate", (14336, 4096)), ("down", (4096, 14336))]
+        for g in (64, 128):
+            for d in (0.0, 0.001, 0.01):
+                per_gemv(shapes, (2, 3, 4, 5, 6), g, 4, d, tag=f"g{g} d{d} ")
+        cfg = {"shapes_out_x_in": [list(v) for _, v in shapes], "bits": [2, 3, 4, 5, 6], "n_planes": 4,
+               "groups": [64, 128], "side_record_densities": [0.0, 0.001, 0.01], "batch": 1}
+    else:  # llama31_8b_stack
+        layers, K = 32, max(1, args.stack_distinct)
+        shapes = _layer_shapes()
+        enc = []
+        for li in range(K):
+            enc.append([Q.stagq_pack(Q.stagq_encode(synth.weights(o, i, seed=1000 * li + j), GROUP, N_PLANES,
+                                                    DENSITY, "fast")) for j, (_, (o, i)) in enumerate(shapes)])
+        stack = [[Q.stagq_load(enc[li % K][j], 0) for j in range(len(shapes))] for li in range(layers)]
+        del enc
+        weights = layers * sum(o * i for _, (o, i) in shapes)
+        for batch in (1, 4):
+            xs = [torch.from_numpy(synth.activations(batch, i, seed=i + batch)).cuda() for _, (o, i) in shapes]
+            ys = [torch.empty(batch, o, dtype=torch.float16, device="cuda") for _, (o, i) in shapes]
+            for b in BITS:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.stream(stream):
+                    for li in range(layers):
+                        for j in range(len(shapes)):
+                            Q.stagq_gemv_n(stack[li][j], b, xs[j], batch, ys[j], stream=stream)
+                torch.cuda.synchronize()
+                with torch.cuda.graph(g, stream=stream):
+                    for li in range(layers):
+                        for j in range(len(shapes)):
+                            Q.stagq_gemv_n(stack[li][j], b, xs[j], batch, ys[j], stream=stream)
+                for _ in range(3):
+                    g.replay()
+                torch.cuda.synchronize()
+                ts = []
+                for _ in range(5):
+                    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    with torch.cuda.stream(stream):
+                        a0.record(stream)
+                        g.replay()
+                        a1.record(stream)
+                    torch.cuda.synchronize()
+                    ts.append(a0.elapsed_time(a1) * 1e3)
+                launches += 8 * layers * len(shapes)
+                us = statistics.median(ts)
+                nb = sum(Q.stagq_bytes(stack[0][j], b, batch) for j in range(len(shapes))) * layers
+                results[f"p{b} batch{batch}"] = {"us_per_token_step": round(us, 1),
+                                                 "us_per_token": round(us / batch, 1), "bytes": nb,
+                                                 "gbs": round(nb / us / 1e3, 1), "frac": round(nb / us / 1e3 / peak, 4),
+                                                 "gemvs": layers * len(shapes)}
+                del g
+        stored = sum(m.device_bytes for L in stack for m in L)
+        for L in stack:
+            for m in L:
+                m.free()
+        cfg = {"layers": layers, "linears_out_x_in": {k: list(v) for k, v in shapes}, "weights": weights,
+               "distinct_encoded_layers": K, "stored_bytes": stored, "bits": list(BITS), "batches": [1, 4],
+               "group": GROUP, "n_planes": N_PLANES, "side_record_density": DENSITY,
+               "note": f"the 32 resident layers cycle over {K} distinct encodings (timing does not depend on "
+                       f"the weight values; {stored / 1e9:.2f} GB resident >> L2)"}
+    clk = clocks.stop()
+    vals = [r["gbs"] for r in results.values()]
+    value = round(statistics.median(vals), 1) if vals else None
+    _extra_line(args, args.workload, results, cfg, clk, peak, peak_kind, value, "GB/s", launches)
+
 
 def run_stagq(args):
     import torch
@@ -368,6 +533,8 @@ def main():
     args = _args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload != WORKLOAD:
+        run_extra(args)
     else:
         run_stagq(args)
 
