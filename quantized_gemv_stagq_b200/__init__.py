@@ -21,6 +21,8 @@ STAGQ_OK = 0
 STAGQ_PAIR_SEARCH = 0
 STAGQ_PAIR_FAST = 1
 STAGQ_Y_F32 = 1
+STAGQ_KERNEL_GENERAL = 2
+STAGQ_KERNEL_SINGLE = 4
 STAGQ_MAX_PLANES = 4
 STAGQ_MAX_BATCH = 4
 

@@ -14,8 +14,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libstagq.so")
 
-SOURCES = ["api.cu", "gemv.cu", "encoder.cpp", "stream.cpp"]
-HEADERS = ["layout.cuh", "device_matrix.hpp", "host_common.hpp", "stream.hpp"]
+SOURCES = ["api.cu", "gemv.cu", "gemv1.cu", "encoder.cpp", "stream.cpp"]
+HEADERS = ["layout.cuh", "kernel_common.cuh", "device_matrix.hpp", "host_common.hpp", "stream.hpp"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -19,6 +19,9 @@ struct stagq_matrix {
   stagq::DeviceMatrix dm{};
   stagq::GemvPlan plan[7][STAGQ_MAX_BATCH + 1]{};  // per precision (bits) and vector count
   bool plan_ok[7][STAGQ_MAX_BATCH + 1]{};
+  stagq::Gemv1Plan plan1[7]{};   // single-vector kernel, per precision
+  bool plan1_ok[7]{};
+  bool prefer1[7]{};             // the single-vector kernel serves n = 1 by default
   void* d_mem = nullptr;
   size_t d_bytes = 0;
   void* d_stage = nullptr;      // x / y staging for stagq_gemv_host
@@ -110,12 +113,26 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   const size_t side_stride = align_up(side_ent_off + 4 * (size_t)max_cta, 16);
   if (side_stride > (size_t)INT32_MAX) return fail(STAGQ_EINVAL, "side record too large per CTA");
   const size_t side_bytes = (size_t)grid * side_stride;
+  // The same record cut for the single-vector kernel: one CTA per SM, rows in order.
+  const int grid1 = gemv1_grid(s->out, prop.multiProcessorCount);
+  const int rows_cap1 = (int)((out_ + grid1 - 1) / grid1);
+  int64_t max_cta1 = 0;
+  for (int b = 0; b < grid1; ++b) {
+    const int64_t ra = (int64_t)b * out_ / grid1, rb = (int64_t)(b + 1) * out_ / grid1;
+    const int64_t n = (int64_t)s->row_ptr[rb] - s->row_ptr[ra];
+    if (n > max_cta1) max_cta1 = n;
+  }
+  const size_t side1_ent_off = align_up((size_t)4 * ((size_t)rows_cap1 + 1), 16);
+  const size_t side1_stride = align_up(side1_ent_off + 4 * (size_t)max_cta1, 16);
+  if (side1_stride > (size_t)INT32_MAX) return fail(STAGQ_EINVAL, "side record too large per CTA");
+  const size_t side1_bytes = (size_t)grid1 * side1_stride;
   size_t off = 0;
   const size_t o_base = off; off = align_up(off + base_bytes, 256);
   size_t o_plane[STAGQ_MAX_PLANES] = {};
   for (int k = 0; k < np; ++k) { o_plane[k] = off; off = align_up(off + plane_bytes, 256); }
   const size_t o_pair = off; off = align_up(off + pair_bytes, 256);
   const size_t o_side = off; off = align_up(off + side_bytes, 256);
+  const size_t o_side1 = off; off = align_up(off + side1_bytes, 256);
   const size_t o_tab = off; off = align_up(off + tab_bytes, 256);
   const size_t o_status = off; off = align_up(off + 4, 256);
   const size_t total = off;
@@ -160,6 +177,20 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
       }
     }
   }
+  std::vector<uint8_t> side1(side1_bytes, 0);
+  for (int b = 0; b < grid1; ++b) {
+    const int64_t ra = (int64_t)b * out_ / grid1, rb = (int64_t)(b + 1) * out_ / grid1, n = rb - ra;
+    uint8_t* blk = &side1[(size_t)b * side1_stride];
+    int32_t* offs = reinterpret_cast<int32_t*>(blk);
+    uint32_t* ent = reinterpret_cast<uint32_t*>(blk + side1_ent_off);
+    int32_t pos = 0;
+    for (int64_t r = 0; r < n; ++r) {
+      offs[r] = pos;
+      for (int64_t e = s->row_ptr[ra + r]; e < s->row_ptr[ra + r + 1]; ++e)
+        ent[pos++] = (uint32_t)xq_slot_of_column(s->col[e]) | ((uint32_t)s->val[e] << 16);
+    }
+    offs[n] = pos;
+  }
   std::vector<uint8_t> pairs(pair_bytes, 0);
   for (int64_t r = 0; r < out_; ++r) std::memcpy(&pairs[(size_t)r * pair_stride], s->pair_idx + (size_t)r * pair_row, pair_row);
 
@@ -168,6 +199,7 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   for (int k = 0; k < np; ++k) copies.push_back({o_plane[k], s->planes + base_bytes + (size_t)k * plane_bytes, plane_bytes});
   copies.push_back({o_pair, pairs.data(), pair_bytes});
   copies.push_back({o_side, side.data(), side_bytes});
+  copies.push_back({o_side1, side1.data(), side1_bytes});
   copies.push_back({o_tab, tabs.data(), tab_bytes});
   for (const Copy& c : copies) {
     e = cudaMemcpy(d + c.off, c.src, c.n, cudaMemcpyHostToDevice);
@@ -198,6 +230,11 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   m.side_stride = (int32_t)side_stride;
   m.side_ent_off = (int32_t)side_ent_off;
   m.side_grid = grid;
+  m.side1 = d + o_side1;
+  m.side1_stride = (int32_t)side1_stride;
+  m.side1_ent_off = (int32_t)side1_ent_off;
+  m.side1_grid = grid1;
+  m.side1_max = (int32_t)max_cta1;
   m.tables = reinterpret_cast<const float2*>(d + o_tab);
   m.status = reinterpret_cast<uint32_t*>(d + o_status);
   m.num_sms = prop.multiProcessorCount;
@@ -205,6 +242,16 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   if (m.smem_pair_budget > smem_limit) m.smem_pair_budget = smem_limit;
   for (int b = 2; b <= 2 + np; ++b)
     for (int nb = 1; nb <= STAGQ_MAX_BATCH; ++nb) h->plan_ok[b][nb] = make_plan(m, b, nb, &h->plan[b][nb]);
+  // The single-vector kernel serves n = 1 on large matrices (>= 2^25 weights:
+  // Llama-3.1-8B gate/up/down): there its faster block loop outweighs its
+  // extra once-per-launch phases (entry rows, side-record terms, row sums),
+  // measured over a whole layer's chain of GEMVs at 2, 3 and 4 bits. On
+  // smaller matrices those phases dominate and the general kernel is faster.
+  const bool large = (int64_t)s->out * s->in >= ((int64_t)1 << 25);
+  for (int b = 2; b <= 2 + np; ++b) {
+    h->plan1_ok[b] = make_plan1(m, b, &h->plan1[b]);
+    h->prefer1[b] = large;
+  }
   if (!h->plan_ok[2][1]) {
     cudaFree(h->d_mem);
     delete h;
@@ -228,12 +275,21 @@ extern "C" int stagq_gemv_ex(stagq_handle h, int bits, const void* x, int n, voi
   if (!x || !y) return fail(STAGQ_EINVAL, "null x or y");
   if (n < 1 || n > STAGQ_MAX_BATCH) return fail(STAGQ_EINVAL, "n outside 1..STAGQ_MAX_BATCH");
   if (reinterpret_cast<uintptr_t>(x) % 16) return fail(STAGQ_EINVAL, "x must be 16-byte aligned");
-  if (flags & ~STAGQ_Y_F32) return fail(STAGQ_EINVAL, "unknown flags");
+  if (flags & ~(STAGQ_Y_F32 | STAGQ_KERNEL_GENERAL | STAGQ_KERNEL_SINGLE)) return fail(STAGQ_EINVAL, "unknown flags");
+  const bool force_general = flags & STAGQ_KERNEL_GENERAL, force_single = flags & STAGQ_KERNEL_SINGLE;
+  if (force_general && force_single) return fail(STAGQ_EINVAL, "both kernels forced");
+  if (force_single && (n != 1 || !h->plan1_ok[bits]))
+    return fail(STAGQ_EINVAL, "the single-vector kernel serves n = 1 on shapes it can plan");
   DeviceGuard guard(h->device);
   if (!guard.ok) return fail(STAGQ_ECUDA, "cudaSetDevice failed");
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   const int yf32 = (flags & STAGQ_Y_F32) ? 1 : 0;
   const size_t ysz = yf32 ? 4 : 2;
+  if (force_single || (n == 1 && !force_general && h->plan1_ok[bits] && h->prefer1[bits])) {
+    cudaError_t e = launch_gemv1(h->dm, h->plan1[bits], bits, x, y, yf32, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "GEMV launch");
+    return STAGQ_OK;
+  }
   if (h->plan_ok[bits][n]) {  // one launch: the weights are read once for all n vectors
     cudaError_t e = launch_gemv(h->dm, h->plan[bits][n], bits, x, y, yf32, stream);
     if (e != cudaSuccess) return cuda_fail(e, "GEMV launch");

@@ -15,6 +15,17 @@ constexpr int64_t kTwoCtaWeightsPerSm = 256 * 1024;  // from this many weights p
 // Row groups of a CTA with KW K slices: up to 8 warps in all, at least one group.
 inline int row_groups(int KW) { return KW <= 4 ? 8 / KW : 1; }
 
+// Shared-memory order of the fixed-point activations x~ inside a GEMV CTA:
+// chunk c (64 int16) is 8 pieces of 16 bytes, piece p stored at piece slot
+// (p + c) mod 8, so that 32 lanes reading piece p of their own chunks hit 8
+// different 16-byte bank groups instead of one.
+__host__ __device__ inline int xq_piece_index(int c, int p) { return c * 8 + ((p + c) & 7); }
+// Element slot of column `col` (its chunk is slot >> 6, as for the column).
+__host__ __device__ inline int xq_slot_of_column(int col) {
+  const int c = col >> 6, e = col & 63;
+  return xq_piece_index(c, e >> 3) * 8 + (e & 7);
+}
+
 struct DeviceMatrix {
   int32_t out, in, group, n_planes;
   int64_t nnz;
@@ -30,6 +41,13 @@ struct DeviceMatrix {
   // The entries (column | fp16 value << 16) start at side_ent_off.
   const uint8_t* side;
   int32_t side_stride, side_ent_off, side_grid;
+  // The same side record cut for the single-vector kernel (gemv1.cu): per CTA
+  // of its grid (side1_grid CTAs, one per SM), side1_stride bytes: int32
+  // offsets [rows + 1] (where each local row's entries start, then the end),
+  // and from side1_ent_off the entries (xq_slot_of_column(column) | fp16 value
+  // << 16) in (row, column) order; side1_max entries at most per CTA.
+  const uint8_t* side1;
+  int32_t side1_stride, side1_ent_off, side1_grid, side1_max;
   const float2* tables;       // [n_planes+1][256]: (lo_M, s_M * c_M) for M = 2..2+n_planes
   uint32_t* status;           // nonzero once a kernel gave up waiting for its copies
   int num_sms;
@@ -52,6 +70,27 @@ struct GemvPlan {
   int pdl;               // launch with programmatic dependent launch
   int nb;                // activation vectors per launch (1..4; the weights are read once)
 };
+
+// Launch plan of the single-vector kernel (gemv1.cu).
+struct Gemv1Plan {
+  int grid;              // CTAs (= side1_grid, at most one per SM)
+  int KW, RG, NW;        // K slices, row groups, consumer warps (KW * RG); one producer warp more
+  int up, br;            // rows per warp per block, rows per block (RG * up)
+  int ns;                // ring slots
+  int rows_cap;          // most rows of one CTA
+  int stage_side;        // the CTA's side record is copied into shared memory
+  int side_stride, side_ent_off, side_max;
+  int group_shift;       // log2(group)
+  int pair_stride;
+  int pdl;               // launch with programmatic dependent launch
+};
+
+// Plan for the single-vector kernel at `bits`; false if it cannot be planned
+// (the general kernel then serves n = 1 too).
+bool make_plan1(const DeviceMatrix& m, int bits, Gemv1Plan* plan);
+int gemv1_grid(int out, int num_sms);
+cudaError_t launch_gemv1(const DeviceMatrix& m, const Gemv1Plan& plan, int bits, const void* x, void* y, int y_f32,
+                         cudaStream_t stream);
 
 // Plan for a GEMV at `bits` with `nb` activation vectors; false if the shape
 // cannot be planned.

@@ -44,152 +44,13 @@
 #include <mutex>
 
 #include "device_matrix.hpp"
+#include "kernel_common.cuh"
 #include "layout.cuh"
 
 namespace stagq {
 namespace {
 
-constexpr unsigned kFull = 0xFFFFFFFFu;
-
-// x~ in shared memory: chunk c (64 int16) is 8 pieces of 16 bytes, piece p
-// stored at slot (p + c) mod 8, so that 32 lanes reading piece p of their own
-// chunks hit 8 different 16-byte bank groups instead of one.
-__device__ __forceinline__ int xq_piece(int c, int p) { return c * 8 + ((p + c) & 7); }
-__device__ __forceinline__ int xq_elem(int col) {
-  const int c = col >> 6, e = col & 63;
-  return xq_piece(c, e >> 3) * 8 + (e & 7);
-}
-
-
-// ------------------------------------------------------------ PTX helpers
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t global_timer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_barrier_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Wait until the phase of `bar` with the given parity has completed, for at
-// most `limit_ns`; false on expiry.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 15u) == 0 && global_timer() - t0 > limit_ns) return false;
-  }
-}
-// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
-// dst, src and bytes are multiples of 16.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(bar)
-               : "memory");
-}
-__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void grid_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-__device__ __forceinline__ int dp2a_lo(uint32_t xpair, uint32_t codes, int acc) {
-  int d;
-  asm("dp2a.lo.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(xpair), "r"(codes), "r"(acc));
-  return d;
-}
-__device__ __forceinline__ int dp2a_hi(uint32_t xpair, uint32_t codes, int acc) {
-  int d;
-  asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(xpair), "r"(codes), "r"(acc));
-  return d;
-}
-
-// Four weights (i, s, j = 0..3) whose code bytes are `m`, against their
-// fixed-point activations X[8i+2s] (j = 0, 1) and X[8i+2s+1] (j = 2, 3).
-__device__ __forceinline__ int dot4(const uint32_t (&X)[32], int i, int s, uint32_t m, int acc) {
-  acc = dp2a_lo(X[8 * i + 2 * s], m, acc);
-  return dp2a_hi(X[8 * i + 2 * s + 1], m, acc);
-}
-
-// sum over one 64-weight chunk of v_t X_t with v = u_M (v = 2 u_3 at M = 3).
-// B: the 4 base words; P[k]: the 2 chunk words of plane k+3. Exact in int32.
-template <int M>
-__device__ __forceinline__ int chunk_dot(const uint32_t (&X)[32], const uint32_t (&B)[4], const uint2* P) {
-  if constexpr (M == 2) {
-    int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      a0 = dot4(X, i, 0, B[i] & 0x03030303u, a0);
-      a1 = dot4(X, i, 1, B[i] & 0x0C0C0C0Cu, a1);
-      a2 = dot4(X, i, 2, B[i] & 0x30303030u, a2);
-      a3 = dot4(X, i, 3, B[i] & 0xC0C0C0C0u, a3);
-    }
-    // slot s carries q * 4^s, so every product in a_s is a multiple of 4^s
-    return a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6);
-  } else {
-    int lo = 0, hi = 0;
-#pragma unroll
-    for (int w = 0; w < 2; ++w) {
-      const uint32_t p3 = w ? P[0].y : P[0].x;
-      uint32_t p4 = 0u;
-      if constexpr (M >= 4) p4 = w ? P[1].y : P[1].x;
-      uint32_t E0, O0, E1, O1;
-      nibble_words(B[2 * w], B[2 * w + 1], p3, p4, E0, O0, E1, O1);
-      const int i0 = 2 * w, i1 = 2 * w + 1;
-      lo = dot4(X, i0, 1, E0 & 0x0F0F0F0Fu, lo);
-      hi = dot4(X, i0, 3, E0 & 0xF0F0F0F0u, hi);
-      lo = dot4(X, i0, 0, O0 & 0x0F0F0F0Fu, lo);
-      hi = dot4(X, i0, 2, O0 & 0xF0F0F0F0u, hi);
-      lo = dot4(X, i1, 1, E1 & 0x0F0F0F0Fu, lo);
-      hi = dot4(X, i1, 3, E1 & 0xF0F0F0F0u, hi);
-      lo = dot4(X, i1, 0, O1 & 0x0F0F0F0Fu, lo);
-      hi = dot4(X, i1, 2, O1 & 0xF0F0F0F0u, hi);
-    }
-    const int nib = lo + (hi >> 4);  // high-nibble products are multiples of 16
-    if constexpr (M <= 4) {
-      return nib;
-    } else {
-      int a5 = 0, a6 = 0;
-#pragma unroll
-      for (int w = 0; w < 2; ++w) {
-        const uint32_t p5 = w ? P[2].y : P[2].x;
-        uint32_t p6 = 0u;
-        if constexpr (M >= 6) p6 = w ? P[3].y : P[3].x;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-#pragma unroll
-          for (int s = 0; s < 4; ++s) {
-            const int sh = 4 * h + s;
-            a5 = dot4(X, 2 * w + h, s, (p5 >> sh) & 0x01010101u, a5);
-            if constexpr (M >= 6) a6 = dot4(X, 2 * w + h, s, (p6 >> sh) & 0x01010101u, a6);
-          }
-        }
-      }
-      if constexpr (M == 5) return 2 * nib + a5;
-      else return 4 * nib + 2 * a5 + a6;
-    }
-  }
-}
+using namespace kernels;
 
 // Sum v[0..UP-1] over the 32 lanes; afterwards lanes [u*32/UP, (u+1)*32/UP)
 // hold the total of v[u]. UP - 1 + log2(32) - log2(UP) shuffles.
@@ -677,6 +538,10 @@ cudaError_t ensure_smem(const void* kern, int key, size_t smem) {
   std::lock_guard<std::mutex> lock(mu);
   if (granted[dev][key] >= smem) return cudaSuccess;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // The largest shared-memory carve-out, as the single-vector kernel asks:
+  // consecutive GEMVs of either kernel then run under one L1 / shared split
+  // and can share an SM without reconfiguring it.
+  if (err == cudaSuccess) err = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (err == cudaSuccess) granted[dev][key] = smem;
   return err;
 }

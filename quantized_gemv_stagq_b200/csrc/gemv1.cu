@@ -1,0 +1,543 @@
+// sm_100a kernel of the StagQ GEMV for one activation vector, y = W_hat^(M) x.
+//
+// What is computed (StagQ paper, arXiv 2610.05977): for every row i,
+//   y_i = sum_groups [ s_M(g) * sum_{j in g} u_M,j x_j + lo_M(g) * sum_{j in g} x_j ]
+//         + sum_{held-out (i,c)} x_c (v_ic - lo_M(g(i,c)))
+// -- the affine map of Eq. (10) applied once per group, with u_M from Eq. (8),
+// and the side record of Eq. (4) (held-out digits are zero, so the main
+// stream decoded lo_M there and the correction is v - lo_M).
+//
+// How (for B200; batch-one GEMV is bound by HBM and by the SM's integer issue
+// rate, so no tensor cores):
+//  * One CTA per SM owns a contiguous, balanced range of rows, cut into blocks
+//    of BR rows. Warp 0 is the producer: it moves each block's base rows and
+//    read-plane rows (a p_M read never touches deeper planes) into a shared-
+//    memory ring slot with 1 + (M - 2) bulk copies. Warps 1..NW are consumers:
+//    KW K slices (2048 weights: 32 lanes x one 64-weight chunk) x RG row
+//    groups; in every block a consumer takes UP rows of its group in its slice.
+//  * The CTA uses at most half of an SM (<= 9 warps x 96 registers, <= half the
+//    shared memory), so the next GEMV's CTA is resident beside it and fills its
+//    ring -- weights, pair table, the CTA's pair bytes and side record do not
+//    depend on earlier kernels -- before this one finishes.
+//  * x is converted once per CTA to 16-bit fixed point with a power-of-two
+//    scale per 64-element chunk (|error| <= 2^-16 max|x_chunk|); each lane keeps
+//    its chunk's 64 activations in registers; code bytes / nibble composites
+//    (layout.cuh) feed dp2a integer dot products (exact in int32) and the group
+//    affine is applied once per chunk in fp32.
+//  * Two shuffle stages leave 8 partial sums per (row, K slice) in shared
+//    memory, and the slot goes back to the producer.
+//  * The held-out entries are taken apart from the blocks, where they would
+//    add a chain of dependent shared-memory reads to every block: each entry's
+//    local row is written once after the x conversion; after its blocks, every
+//    warp computes the terms x~_c (v - lo_M) of an equal share of the CTA's
+//    entries, independently of each other, into shared memory.
+//  * Finally one thread per row adds its partials and its entries' terms in a
+//    fixed order and stores y: deterministic, no atomics on data, no
+//    workspace, one launch.
+//  * Every mbarrier wait is bounded in time; on expiry the kernel records it
+//    in the handle's status word, waits (bounded) for its own copies and
+//    returns.
+#include <cuda_fp16.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "device_matrix.hpp"
+#include "kernel_common.cuh"
+#include "layout.cuh"
+
+namespace stagq {
+namespace {
+
+using namespace kernels;
+
+constexpr int kRegs1 = 96;             // registers per thread: two 9-warp CTAs fit one SM
+constexpr int kParts1 = 8;             // partial sums per (row, K slice), each over 4 lanes
+
+struct Gemv1Args {
+  DeviceMatrix m;
+  Gemv1Plan plan;
+  const float2* table;  // (lo_M, s_M c_M) of this precision
+  const __half* x;
+  void* y;
+  int y_f32;
+};
+
+constexpr uint64_t kWaitLimit1Ns = 2000000000ull;  // a copy that has not landed in 2 s never will
+constexpr uint64_t kDrainLimit1Ns = 100000000ull;  // after a failure: wait for own copies, 0.1 s
+
+// Floats per row of K-slice partials: KW x 8 padded to an odd multiple of 4, so
+// that 8 threads reading consecutive rows with 16-byte loads hit 8 different
+// bank groups.
+__host__ __device__ inline int part_stride1(int KW) { return KW * kParts1 + 4; }
+
+struct Smem1 {
+  uint32_t full, empty, side_bar, flag, tab, xq, xscale, xsum, pairs, side, part, rowid, term, ring;
+  uint32_t slot;         // bytes of one ring slot
+  uint32_t plane_piece;  // offset of the first read plane inside a slot (base rows at 0)
+  uint32_t total;
+};
+
+__host__ __device__ inline uint32_t up16(uint32_t v) { return (v + 15u) & ~15u; }
+
+__host__ __device__ inline Smem1 smem1(const Gemv1Plan& p, int in, int M) {
+  Smem1 L;
+  const uint32_t nchunk = in / kChunk, BR = p.br, rc = (uint32_t)p.rows_cap, sm = (uint32_t)p.side_max;
+  uint32_t o = 0;
+  L.full = o; o += 8 * kMaxSlots;    // block landed in the slot (producer arrive + bytes)
+  L.empty = o; o += 8 * kMaxSlots;   // every consumer warp is done with the slot
+  L.side_bar = o; o += 8;            // pair table, pair bytes and side record landed
+  L.flag = o; o += 8;                // a wait gave up (any thread)
+  L.tab = o; o += 256 * 8;
+  L.xq = o; o += 2 * in;
+  L.xscale = o; o += 4 * nchunk;
+  L.xsum = o; o += 4 * nchunk;
+  o = up16(o);
+  L.pairs = o; o += up16(rc * (uint32_t)p.pair_stride);
+  L.side = o; o += p.stage_side ? (uint32_t)p.side_stride : 0u;
+  o = up16(o);
+  L.part = o; o += 4u * rc * (uint32_t)part_stride1(p.KW);
+  L.term = o; o += 4u * sm;          // x~_c (v - lo_M) of each held-out entry
+  L.rowid = o; o += up16(2u * sm);   // local row of each held-out entry
+  o = (o + 127u) & ~127u;
+  L.ring = o;
+  L.plane_piece = BR * (in / 4);
+  L.slot = (L.plane_piece + (uint32_t)(M - 2) * BR * (in / 8) + 127u) & ~127u;
+  o += p.ns * L.slot;
+  L.total = o;
+  return L;
+}
+
+__device__ __forceinline__ void mbar_arrive1(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Cross-lane sums of the UP rows of a block: afterwards lane l holds, for row
+// reduced_row1<UP>(l), the sum of its 4 lanes {l, l^8, l^16, l^24}; lanes with
+// keeps_partial1<UP>(l) store it (8 partials per row).
+template <int UP>
+__device__ __forceinline__ float partial_reduce1(const float (&v)[UP], int lane) {
+  const bool h16 = lane & 16, h8 = lane & 8;
+  if constexpr (UP == 4) {
+    const float s0 = (h16 ? v[2] : v[0]) + __shfl_xor_sync(kFull, h16 ? v[0] : v[2], 16);
+    const float s1 = (h16 ? v[3] : v[1]) + __shfl_xor_sync(kFull, h16 ? v[1] : v[3], 16);
+    return (h8 ? s1 : s0) + __shfl_xor_sync(kFull, h8 ? s0 : s1, 8);
+  } else if constexpr (UP == 2) {
+    const float s = (h16 ? v[1] : v[0]) + __shfl_xor_sync(kFull, h16 ? v[0] : v[1], 16);
+    return s + __shfl_xor_sync(kFull, s, 8);
+  } else {
+    const float s = v[0] + __shfl_xor_sync(kFull, v[0], 16);
+    return s + __shfl_xor_sync(kFull, s, 8);
+  }
+}
+template <int UP>
+__device__ __forceinline__ int reduced_row1(int lane) {
+  return UP == 4 ? ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1) : UP == 2 ? (lane >> 4) & 1 : 0;
+}
+template <int UP>
+__device__ __forceinline__ bool keeps_partial1(int lane) {
+  return UP == 4 ? true : UP == 2 ? (lane & 8) == 0 : lane < 8;
+}
+
+template <int M, int UP>
+__global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const Gemv1Plan& P = a.plan;
+  const int in = a.m.in;
+  const int nchunk = in / kChunk;
+  const Smem1 L = smem1(P, in, M);
+  const uint32_t sbase = smem_addr(smem);
+  const float2* tab = reinterpret_cast<const float2*>(smem + L.tab);
+  int16_t* xq = reinterpret_cast<int16_t*>(smem + L.xq);
+  float* xscale = reinterpret_cast<float*>(smem + L.xscale);
+  float* xsum = reinterpret_cast<float*>(smem + L.xsum);
+  float* part = reinterpret_cast<float*>(smem + L.part);  // [row][part_stride1(KW)]: [KW][8] used
+  float* term = reinterpret_cast<float*>(smem + L.term);
+  uint16_t* rowid = reinterpret_cast<uint16_t*>(smem + L.rowid);
+  volatile uint32_t* flag = reinterpret_cast<volatile uint32_t*>(smem + L.flag);
+  const uint32_t full0 = sbase + L.full, empty0 = sbase + L.empty, side_bar = sbase + L.side_bar;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthreads = blockDim.x;
+  const int KW = P.KW, NW = P.NW, NS = P.ns, BR = P.br, ps = P.pair_stride, gs = P.group_shift;
+  const int PST = part_stride1(KW);
+  const int r0 = (int)((int64_t)blockIdx.x * a.m.out / gridDim.x);
+  const int rows = (int)((int64_t)(blockIdx.x + 1) * a.m.out / gridDim.x) - r0;
+  const int nblk = (rows + BR - 1) / BR;
+  const int rb = in / 4, rp = in / 8;
+  const uint8_t* side_g = a.m.side1 + (int64_t)blockIdx.x * P.side_stride;
+  const uint8_t* pair_g = a.m.pair + (int64_t)r0 * ps;
+  const uint8_t* pairs = smem + L.pairs;
+  const uint8_t* side = P.stage_side ? smem + L.side : side_g;
+
+  int issued = 0;  // blocks issued so far (producer lane 0 = thread 0)
+  // Block b of the CTA's rows -> slot b % NS (producer lane 0).
+  auto issue_block = [&](int b, int slot) {
+    const int lr0 = b * BR;
+    const int nr = min(BR, rows - lr0);
+    const uint32_t dst = sbase + L.ring + slot * L.slot, bar = full0 + 8 * slot;
+    mbar_arrive_expect_tx(bar, (uint32_t)nr * (rb + (M - 2) * rp));
+    bulk_load(dst, a.m.base + (int64_t)(r0 + lr0) * rb, nr * rb, bar);
+#pragma unroll
+    for (int k = 0; k < M - 2; ++k)
+      bulk_load(dst + L.plane_piece + k * BR * rp, a.m.plane[k] + (int64_t)(r0 + lr0) * rp, nr * rp, bar);
+    issued = b + 1;
+  };
+
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, (uint32_t)NW);
+    }
+    mbar_init(side_bar, 1);
+    *flag = 0u;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    // Nothing of this depends on earlier kernels: fill the ring before
+    // waiting for them.
+    const uint32_t pb = (uint32_t)(rows * ps);
+    const uint32_t sb = P.stage_side ? (uint32_t)P.side_stride : 0u;
+    mbar_arrive_expect_tx(side_bar, 256 * 8 + pb + sb);
+    bulk_load(sbase + L.tab, a.table, 256 * 8, side_bar);
+    bulk_load(sbase + L.pairs, pair_g, pb, side_bar);
+    if (sb) bulk_load(sbase + L.side, side_g, sb, side_bar);
+    for (int b = 0; b < NS && b < nblk; ++b) issue_block(b, b);
+  }
+  grid_launch_dependents();
+  grid_dependency_wait();  // x may come from the previous kernel; y may be read by it
+
+  // x -> 16-bit fixed point, once per CTA (every warp): a task is a quarter
+  // chunk (16 values) and the 4 tasks of a chunk sit in adjacent lanes. Scale
+  // 2^e with max|x| 2^e in [2^14, 2^15) per chunk, so the largest entries
+  // convert exactly; rounding to nearest even goes through the 1.5 * 2^23
+  // shifter (the low 16 bits of the sum are the two's-complement integer).
+  {
+    constexpr float kShift = 12582912.0f;
+    constexpr int kBatch = 4;
+    const int ntask = 4 * nchunk;
+    const uint4* x4 = reinterpret_cast<const uint4*>(a.x);
+    for (int t0 = 0; t0 < ntask; t0 += kBatch * nthreads) {
+      uint4 raw[kBatch][2];
+#pragma unroll
+      for (int q = 0; q < kBatch; ++q) {
+        const int t = t0 + q * nthreads + tid;
+        raw[q][0] = raw[q][1] = make_uint4(0u, 0u, 0u, 0u);
+        if (t < ntask) {
+          raw[q][0] = __ldg(x4 + 2 * t);
+          raw[q][1] = __ldg(x4 + 2 * t + 1);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < kBatch; ++q) {
+        const int tw = t0 + q * nthreads + warp * 32;  // first task of this warp
+        if (tw >= ntask) break;                         // warp-uniform
+        const int t = tw + lane;
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(raw[q]);
+        __half2 m2 = __habs2(*reinterpret_cast<const __half2*>(&w[0]));
+#pragma unroll
+        for (int k = 1; k < 8; ++k) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __half2*>(&w[k])));
+        float mx = fmaxf(__low2float(m2), __high2float(m2));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+        const int e = mx > 0.f ? 14 - ((int)((__float_as_uint(mx) >> 23) & 0xFF) - 127) : 0;
+        const float sc = __int_as_float((127 + e) << 23);
+        uint32_t Q[8];
+        int sumq = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+          Q[k] = __byte_perm(__float_as_uint(fmaf(f.x, sc, kShift)), __float_as_uint(fmaf(f.y, sc, kShift)), 0x5410);
+          sumq = dp2a_lo(Q[k], 0x0101u, sumq);
+        }
+        sumq += __shfl_xor_sync(kFull, sumq, 1);
+        sumq += __shfl_xor_sync(kFull, sumq, 2);
+        if (t < ntask) {
+          uint4* dst = reinterpret_cast<uint4*>(xq);
+          dst[xq_piece(t >> 2, 2 * (t & 3))] = make_uint4(Q[0], Q[1], Q[2], Q[3]);
+          dst[xq_piece(t >> 2, 2 * (t & 3) + 1)] = make_uint4(Q[4], Q[5], Q[6], Q[7]);
+          if ((t & 3) == 0) {
+            const float xs_c = __int_as_float((127 - e) << 23);
+            xscale[t >> 2] = xs_c;
+            xsum[t >> 2] = xs_c * (float)sumq;
+          }
+        }
+      }
+    }
+  }
+  bool ok = __all_sync(kFull, mbar_wait(side_bar, 0, kWaitLimit1Ns));
+  const int32_t* offs = reinterpret_cast<const int32_t*>(side);
+  const uint32_t* ents = reinterpret_cast<const uint32_t*>(side + P.side_ent_off);
+  // local row of each held-out entry (a thread per row)
+  if (ok) {
+    for (int r = tid; r < rows; r += nthreads) {
+      const int j1 = offs[r + 1];
+      for (int j = offs[r]; j < j1; ++j) rowid[j] = (uint16_t)r;
+    }
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    for (int b = 0; ok && b + NS < nblk; ++b) {
+      if (!__all_sync(kFull, mbar_wait(empty0 + 8 * (b % NS), (uint32_t)(b / NS) & 1u, kWaitLimit1Ns))) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) issue_block(b + NS, b % NS);
+      __syncwarp();
+    }
+  } else if (ok) {
+    // ---------------------------------------------------------- consumers
+    const int cw = warp - 1;                 // consumer warp index
+    const int kw = cw % KW, rg = cw / KW, RG = P.RG;
+    const int c = kw * 32 + lane;            // this lane's 64-weight chunk
+    const bool active = c < nchunk;
+    const int cc = active ? c : 0;           // reads of inactive lanes stay inside the row
+    uint32_t X[32];
+    float xs, xsm;
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(xq);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint4 t = src[xq_piece(cc, k)];
+        X[4 * k] = t.x;
+        X[4 * k + 1] = t.y;
+        X[4 * k + 2] = t.z;
+        X[4 * k + 3] = t.w;
+      }
+      xs = active ? xscale[cc] : 0.f;
+      xsm = active ? xsum[cc] : 0.f;
+    }
+    // Where this warp's rows sit in a slot (row u of the warp = block row rg + RG u).
+    const uint32_t off_b = (uint32_t)(rg * rb + cc * kBaseChunkBytes);
+    const uint32_t off_p = L.plane_piece + (uint32_t)(rg * rp + cc * kPlaneChunkBytes);
+    const uint32_t step_b = (uint32_t)(RG * rb), step_p = (uint32_t)(RG * rp), plane_stride = (uint32_t)(BR * rp);
+    const int pcol = (cc * kChunk) >> gs;    // this lane's pair byte within a row
+    const int urow = reduced_row1<UP>(lane);
+    const bool keep = keeps_partial1<UP>(lane);
+    const uint8_t* ring = smem + L.ring;
+    int slot = 0;
+    uint32_t phase = 0;
+    for (int b = 0; b < nblk; ++b) {
+      if (!__all_sync(kFull, mbar_wait(full0 + 8 * slot, phase, kWaitLimit1Ns))) {
+        ok = false;
+        break;
+      }
+      const uint8_t* sb = ring + slot * L.slot;
+      const int lr = b * BR + rg;            // local row of this warp's row 0 in the block
+      uint32_t B[UP][4];
+      uint2 Pw[UP][M > 2 ? M - 2 : 1];
+      float2 lm[UP];
+#pragma unroll
+      for (int u = 0; u < UP; ++u) {
+        const uint4 b4 = *reinterpret_cast<const uint4*>(sb + off_b + u * step_b);
+        B[u][0] = b4.x; B[u][1] = b4.y; B[u][2] = b4.z; B[u][3] = b4.w;
+#pragma unroll
+        for (int k = 0; k < M - 2; ++k)
+          Pw[u][k] = *reinterpret_cast<const uint2*>(sb + off_p + u * step_p + k * plane_stride);
+        const int row = min(lr + RG * u, rows - 1);  // rows past the CTA's end read a valid pair byte
+        lm[u] = tab[pairs[row * ps + pcol]];
+      }
+      float v[UP];
+#pragma unroll
+      for (int u = 0; u < UP; ++u) {
+        const int tot = chunk_dot<M>(X, B[u], Pw[u]);
+        v[u] = fmaf(lm[u].y, (float)tot * xs, lm[u].x * xsm);
+      }
+      const float s = partial_reduce1<UP>(v, lane);
+      const int row = lr + RG * urow;
+      if (keep && row < rows) part[row * PST + kw * kParts1 + (lane & 7)] = s;
+      __syncwarp();  // every lane has read the slot before it is released
+      if (lane == 0) mbar_arrive1(empty0 + 8 * slot);
+      if (++slot == NS) {
+        slot = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ side record
+  // Warp w takes entries [E w / (NW + 1), E (w + 1) / (NW + 1)), lane l every
+  // 32nd from l, four at a time; each term lands in its own slot.
+  if (ok) {
+    const int nw = NW + 1, E = offs[rows];
+    const int j0 = (int)((int64_t)E * warp / nw), j1 = (int)((int64_t)E * (warp + 1) / nw);
+    for (int jb = j0 + lane; jb < j1; jb += 4 * 32) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int j = jb + 32 * k;
+        if (j < j1) {
+          const uint32_t en = ents[j];
+          const int e = (int)(en & 0xFFFFu);  // x~ slot; e >> 6 is the column's 64-chunk
+          const float lo = tab[pairs[(int)rowid[j] * ps + (e >> gs)]].x;
+          term[j] = (float)xq[e] * xscale[e >> 6] * (__half2float(__ushort_as_half((unsigned short)(en >> 16))) - lo);
+        }
+      }
+    }
+  }
+  if (!ok && lane == 0) *flag = 1u;
+  __syncthreads();
+
+  if (*flag == 0u) {
+    // ---------------------------------------------------------- y
+    for (int r = tid; r < rows; r += nthreads) {
+      // four interleaved sums (a fixed order), 16-byte loads of the partials
+      const float4* pr = reinterpret_cast<const float4*>(part + r * PST);
+      float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int k = 0; k < KW * kParts1 / 4; ++k) {
+        const float4 q = pr[k];
+        t.x += q.x; t.y += q.y; t.z += q.z; t.w += q.w;
+      }
+      const int e1 = offs[r + 1];
+      int j = offs[r];
+      for (; j + 3 < e1; j += 4) {
+        t.x += term[j]; t.y += term[j + 1]; t.z += term[j + 2]; t.w += term[j + 3];
+      }
+      for (; j < e1; ++j) t.x += term[j];
+      const float acc = (t.x + t.y) + (t.z + t.w);
+      if (a.y_f32) reinterpret_cast<float*>(a.y)[r0 + r] = acc;
+      else reinterpret_cast<__half*>(a.y)[r0 + r] = __float2half_rn(acc);
+    }
+  } else if (tid == 0) {
+    atomicOr(a.m.status, 1u);
+    // Gave up: let this CTA's copies in flight land before it exits.
+    mbar_wait(side_bar, 0, kDrainLimit1Ns);
+    for (int b = issued - 1; b >= 0 && b >= issued - NS; --b)
+      mbar_wait(full0 + 8 * (b % NS), (uint32_t)(b / NS) & 1u, kDrainLimit1Ns);
+  }
+}
+
+// Opt a kernel into `smem` bytes of dynamic shared memory (and the largest
+// shared-memory carve-out) on the current device, once per (device, kernel).
+cudaError_t ensure_smem1(const void* kern, int key, size_t smem) {
+  constexpr int kMaxDev = 64;
+  static std::mutex mu;
+  static size_t granted[kMaxDev][16] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDev || key < 0 || key >= 16) return cudaErrorInvalidValue;
+  std::lock_guard<std::mutex> lock(mu);
+  if (granted[dev][key] >= smem) return cudaSuccess;
+  err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err == cudaSuccess) err = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (err == cudaSuccess) granted[dev][key] = smem;
+  return err;
+}
+
+template <int M, int UP>
+cudaError_t launch1_mu(const DeviceMatrix& m, const Gemv1Plan& plan, const void* x, void* y, int y_f32,
+                       cudaStream_t stream) {
+  Gemv1Args a;
+  a.m = m;
+  a.plan = plan;
+  a.table = m.tables + 256 * (M - 2);
+  a.x = reinterpret_cast<const __half*>(x);
+  a.y = y;
+  a.y_f32 = y_f32;
+  const Smem1 L = smem1(plan, m.in, M);
+  auto kern = gemv1_kernel<M, UP>;
+  cudaError_t err = ensure_smem1(reinterpret_cast<const void*>(kern), (M - 2) * 3 + (UP == 4 ? 2 : UP - 1), L.total);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)plan.grid);
+  cfg.blockDim = dim3((unsigned)(32 * (plan.NW + 1)));
+  cfg.dynamicSmemBytes = L.total;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = plan.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+template <int M>
+cudaError_t launch1_m(const DeviceMatrix& m, const Gemv1Plan& plan, const void* x, void* y, int y_f32,
+                      cudaStream_t stream) {
+  switch (plan.up) {
+    case 1: return launch1_mu<M, 1>(m, plan, x, y, y_f32, stream);
+    case 2: return launch1_mu<M, 2>(m, plan, x, y, y_f32, stream);
+    case 4: return launch1_mu<M, 4>(m, plan, x, y, y_f32, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+int gemv1_grid(int out, int num_sms) {
+  int g = out < num_sms ? out : num_sms;
+  if ((out + g - 1) / g > kMaxRowsPerCta) g = (out + kMaxRowsPerCta - 1) / kMaxRowsPerCta;
+  return g;
+}
+
+bool make_plan1(const DeviceMatrix& m, int bits, Gemv1Plan* p) {
+  Gemv1Plan q = {};
+  q.KW = (m.in / kChunk + 31) / 32;
+  if (q.KW < 1 || q.KW > kMaxWarps) return false;
+  q.RG = row_groups(q.KW);
+  q.NW = q.KW * q.RG;
+  if (q.NW + 1 > 4 * (16384 / (32 * kRegs1))) return false;  // register file of the four sub-partitions
+  q.grid = m.side1_grid;
+  if (q.grid < 1) return false;
+  q.rows_cap = (m.out + q.grid - 1) / q.grid;
+  q.pair_stride = m.pair_stride;
+  q.side_stride = m.side1_stride;
+  q.side_ent_off = m.side1_ent_off;
+  q.side_max = m.side1_max;
+  q.group_shift = 0;
+  while ((1 << q.group_shift) < m.group) ++q.group_shift;
+  q.pdl = 1;
+  const int per_rg = (q.rows_cap + q.RG - 1) / q.RG;
+  const int up_max = per_rg >= 4 ? 4 : per_rg >= 2 ? 2 : 1;
+  // Shared memory: at most half an SM when two CTAs' warps fit the register
+  // file, so the next GEMV's CTA can be resident beside this one; else the
+  // per-block maximum. Prefer the side record staged, then at least three
+  // slots (or one per block), then more rows per warp.
+  const bool pairable = 2 * (q.NW + 1) <= 4 * (16384 / (32 * kRegs1));
+  const int budgets[2] = {pairable ? m.smem_pair_budget : m.smem_limit, m.smem_limit};
+  for (int bi = 0; bi < 2; ++bi) {
+    for (int stage = 1; stage >= 0; --stage) {
+      bool have = false;
+      Gemv1Plan best = q;
+      for (int up = up_max; up >= 1; up /= 2) {
+        Gemv1Plan t = q;
+        t.up = up;
+        t.br = q.RG * up;
+        t.stage_side = stage;
+        const int nblk = (q.rows_cap + t.br - 1) / t.br;
+        t.ns = nblk < kMaxSlots ? nblk : kMaxSlots;
+        while (t.ns >= 1 && smem1(t, m.in, bits).total > (uint32_t)budgets[bi]) --t.ns;
+        if (t.ns < 1) continue;
+        if (t.ns >= (nblk < 3 ? nblk : 3)) {
+          *p = t;
+          return true;
+        }
+        if (!have || t.ns > best.ns) {
+          best = t;
+          have = true;
+        }
+      }
+      if (have) {
+        *p = best;
+        return true;
+      }
+    }
+  }
+  return false;
+}
+
+cudaError_t launch_gemv1(const DeviceMatrix& m, const Gemv1Plan& plan, int bits, const void* x, void* y, int y_f32,
+                         cudaStream_t stream) {
+  switch (bits) {
+    case 2: return launch1_m<2>(m, plan, x, y, y_f32, stream);
+    case 3: return launch1_m<3>(m, plan, x, y, y_f32, stream);
+    case 4: return launch1_m<4>(m, plan, x, y, y_f32, stream);
+    case 5: return launch1_m<5>(m, plan, x, y, y_f32, stream);
+    case 6: return launch1_m<6>(m, plan, x, y, y_f32, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace stagq

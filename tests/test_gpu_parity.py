@@ -28,11 +28,11 @@ def _load(F):
     return Q.stagq_load(Q.stagq_pack(to_lib_fields(F)), 0)
 
 
-def _gemv(m, bits, x_np, f32=True):
+def _gemv(m, bits, x_np, f32=True, kernel=0):
     x = torch.from_numpy(np.ascontiguousarray(x_np)).cuda()
     n = x.shape[0]
     y = torch.empty(n, m.out, dtype=torch.float32 if f32 else torch.float16, device="cuda")
-    Q.stagq_gemv_ex(m, bits, x, y, n=n, flags=Q.STAGQ_Y_F32 if f32 else 0)
+    Q.stagq_gemv_ex(m, bits, x, y, n=n, flags=(Q.STAGQ_Y_F32 if f32 else 0) | kernel)
     torch.cuda.synchronize()
     return y.cpu().numpy()
 
@@ -73,8 +73,9 @@ def test_gemv_matches_oracle(case):
     x = synth.activations(1, inp, seed + 100)
     for M in range(2, 3 + npl):
         ref = O.gemv(F, M, x)
-        check_close(_gemv(m, M, x, f32=True), ref, f"fp32 y p{M}")
-        check_close(_gemv(m, M, x, f32=False).astype(np.float64), ref, f"fp16 y p{M}")
+        for kern in (Q.STAGQ_KERNEL_GENERAL, Q.STAGQ_KERNEL_SINGLE):  # both n = 1 kernels
+            check_close(_gemv(m, M, x, f32=True, kernel=kern), ref, f"fp32 y p{M} kernel {kern}")
+            check_close(_gemv(m, M, x, f32=False, kernel=kern).astype(np.float64), ref, f"fp16 y p{M} kernel {kern}")
     Q.stagq_check(m)
     m.free()
 
@@ -130,13 +131,15 @@ def test_gemv_is_deterministic_and_reentrant():
     x = torch.from_numpy(synth.activations(1, 4096, 22)).cuda()
     ys = []
     s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
-    for st in (s1, s2, s1):
-        y = torch.empty(1, 1024, dtype=torch.float32, device="cuda")
-        with torch.cuda.stream(st):
-            Q.stagq_gemv_ex(m, 3, x, y, flags=Q.STAGQ_Y_F32, stream=st)
-        ys.append(y)
-    torch.cuda.synchronize()
-    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2])
+    for kern in (Q.STAGQ_KERNEL_GENERAL, Q.STAGQ_KERNEL_SINGLE):
+        ys = []
+        for st in (s1, s2, s1):
+            y = torch.empty(1, 1024, dtype=torch.float32, device="cuda")
+            with torch.cuda.stream(st):
+                Q.stagq_gemv_ex(m, 3, x, y, flags=Q.STAGQ_Y_F32 | kern, stream=st)
+            ys.append(y)
+        torch.cuda.synchronize()
+        assert torch.equal(ys[0], ys[1]) and torch.equal(ys[1], ys[2]), f"kernel {kern}"
     m.free()
 
 
@@ -173,6 +176,12 @@ def test_bad_calls_return_errors():
         Q.stagq_gemv_n(m, 2, x, 0, y)
     with pytest.raises(Q.StagqError):
         Q.stagq_gemv_ex(m, 2, x, y, flags=8)
+    with pytest.raises(Q.StagqError):  # both kernels forced
+        Q.stagq_gemv_ex(m, 2, x, y, flags=Q.STAGQ_KERNEL_GENERAL | Q.STAGQ_KERNEL_SINGLE)
+    x4 = torch.zeros(4, 512, dtype=torch.float16, device="cuda")
+    y4 = torch.zeros(4, 64, dtype=torch.float16, device="cuda")
+    with pytest.raises(Q.StagqError):  # the single-vector kernel with n > 1
+        Q.stagq_gemv_ex(m, 2, x4, y4, n=4, flags=Q.STAGQ_KERNEL_SINGLE)
     m.free()
 
 
@@ -200,9 +209,10 @@ def test_full_size_llama_sampled_rows(name, shape):
     assert all(eq.values()), eq
     x = synth.activations(4, inp, seed=7)
     for M in (2, 3, 4):
-        y = _gemv(m, M, x[:1], f32=False)[0]
-        check_close(y[rows].astype(np.float64), O.gemv(F, M, x[:1])[0], f"{name} p{M}")
-        assert np.all(np.isfinite(y))
+        for kern in (0, Q.STAGQ_KERNEL_GENERAL, Q.STAGQ_KERNEL_SINGLE):
+            y = _gemv(m, M, x[:1], f32=False, kernel=kern)[0]
+            check_close(y[rows].astype(np.float64), O.gemv(F, M, x[:1])[0], f"{name} p{M} kernel {kern}")
+            assert np.all(np.isfinite(y))
         y4 = _gemv(m, M, x, f32=False)  # batch 4 in one launch
         ref4 = O.gemv(F, M, x)
         for j in range(4):
