@@ -45,7 +45,9 @@ WORKLOAD = "llama31_8b_linears_b1"
 BITS = (2, 3, 4)
 GROUP, N_PLANES, DENSITY = 128, 2, 0.005
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["quantized_gemv_stagq_b200/csrc/gemv.cu", "quantized_gemv_stagq_b200/csrc/layout.cuh"]
+KERNEL_SOURCES = ["quantized_gemv_stagq_b200/csrc/gemv.cu", "quantized_gemv_stagq_b200/csrc/gemv1.cu",
+                  "quantized_gemv_stagq_b200/csrc/kernel_common.cuh", "quantized_gemv_stagq_b200/csrc/layout.cuh"]
+LARGE_WEIGHTS = 1 << 25  # from this many weights on, n = 1 runs the single-vector kernel (gemv1)
 
 
 def _args():
@@ -145,6 +147,13 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
                 "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+def _kernel_of(key):
+    """Name of the kernel that serves the GEMV `name@pM` at n = 1."""
+    from quantized_gemv_stagq_b200 import synth
+    out, inp = synth.LLAMA31_8B_LINEARS[key.split("@")[0]]
+    return "gemv1_kernel" if out * inp >= LARGE_WEIGHTS else "gemv_kernel"
 
 
 def _layer_shapes():
@@ -517,7 +526,7 @@ def run_stagq(args):
                    "parallelism": "replicas" if world > 1 else "single"},
         "frac_of_hbm": round(value / world / peak, 4),
         "per_gemv": per, "us_per_precision_layer": step_us,
-        "roofline": {"bound": "hbm", "kernel": f"gemv_kernel {dom_key}", "achieved": dom["gbs"], "peak": peak,
+        "roofline": {"bound": "hbm", "kernel": f"{_kernel_of(dom_key)} {dom_key}", "achieved": dom["gbs"], "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dom["gbs"] / peak, 4),
                      "traffic": traffic, "algorithmic_bytes": dom["bytes"]},
         "cpu_baseline": cpu,
