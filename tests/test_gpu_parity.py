@@ -189,18 +189,16 @@ LLAMA = list(synth.LLAMA31_8B_LINEARS.items())
 SAMPLE_ROWS = 48
 
 
-@pytest.mark.parametrize("name,shape", [(n, s) for n, s in LLAMA if n in ("q_proj", "k_proj", "gate_proj", "down_proj")])
-def test_full_size_llama_sampled_rows(name, shape):
-    """The bench's workload and launch: library encoder -> GPU; oracle encodes
-    the same weights itself; fields and y agree on sampled rows."""
-    out, inp = shape
-    W = synth.weights(out, inp, seed=1000 + out + inp)
-    P = Q.stagq_encode(W, 128, 2, 0.005, "fast")
+def _sampled_rows_case(out, inp, group, n_planes, density, seed, bits_list, kernels, batch4=True):
+    """Library encoder -> GPU (as the bench does); the oracle encodes the same
+    weights itself on sampled rows; fields and y agree on those rows."""
+    W = synth.weights(out, inp, seed=seed)
+    P = Q.stagq_encode(W, group, n_planes, density, "fast")
     m = Q.stagq_load(Q.stagq_pack(P), 0)
-    rng = np.random.default_rng(out)
+    rng = np.random.default_rng(out + inp)
     rows = np.unique(np.concatenate([[0, out - 1], rng.choice(out, SAMPLE_ROWS, replace=False)]))
-    F = O.encode(W, 128, 2, 0.005, "fast", rows=rows)
-    Psub = Q.Fields(F.out, inp, 128, 2, P.q[rows], P.planes[:, rows], P.pair_idx[rows],
+    F = O.encode(W, group, n_planes, density, "fast", rows=rows)
+    Psub = Q.Fields(F.out, inp, group, n_planes, P.q[rows], P.planes[:, rows], P.pair_idx[rows],
                     P.cb_log2s, P.cb_lo_over_s,
                     np.concatenate([[0], np.cumsum(np.diff(P.row_ptr)[rows])]).astype(np.int32),
                     np.concatenate([P.col[P.row_ptr[r]:P.row_ptr[r + 1]] for r in rows]),
@@ -208,14 +206,46 @@ def test_full_size_llama_sampled_rows(name, shape):
     eq = fields_equal(F, Psub)
     assert all(eq.values()), eq
     x = synth.activations(4, inp, seed=7)
-    for M in (2, 3, 4):
-        for kern in (0, Q.STAGQ_KERNEL_GENERAL, Q.STAGQ_KERNEL_SINGLE):
+    for M in bits_list:
+        ref1 = O.gemv(F, M, x[:1])[0]
+        for kern in kernels:
             y = _gemv(m, M, x[:1], f32=False, kernel=kern)[0]
-            check_close(y[rows].astype(np.float64), O.gemv(F, M, x[:1])[0], f"{name} p{M} kernel {kern}")
+            check_close(y[rows].astype(np.float64), ref1, f"{out}x{inp} p{M} kernel {kern}")
             assert np.all(np.isfinite(y))
-        y4 = _gemv(m, M, x, f32=False)  # batch 4 in one launch
-        ref4 = O.gemv(F, M, x)
-        for j in range(4):
-            check_close(y4[j][rows].astype(np.float64), ref4[j], f"{name} p{M} n4 col{j}")
+        if batch4:
+            y4 = _gemv(m, M, x, f32=False)  # batch 4 in one launch
+            ref4 = O.gemv(F, M, x)
+            for j in range(4):
+                check_close(y4[j][rows].astype(np.float64), ref4[j], f"{out}x{inp} p{M} n4 col{j}")
     Q.stagq_check(m)
     m.free()
+
+
+
+
+def _kernels():
+    return (0, Q.STAGQ_KERNEL_GENERAL, Q.STAGQ_KERNEL_SINGLE)
+
+
+@pytest.mark.parametrize("name,shape", [(n, s) for n, s in LLAMA if n in ("q_proj", "k_proj", "gate_proj", "down_proj")])
+def test_full_size_llama_sampled_rows(name, shape):
+    """The bench's workload and launch at full Llama-3.1-8B shapes."""
+    out, inp = shape
+    _sampled_rows_case(out, inp, 128, 2, 0.005, 1000 + out + inp, (2, 3, 4), _kernels())
+
+
+OTHER = [("phi4." + k, v) for k, v in synth.PHI4_LINEARS.items()] + \
+        [("olmo2." + k, v) for k, v in synth.OLMO2_7B_LINEARS.items()]
+
+
+@pytest.mark.parametrize("name,shape", OTHER, ids=[n for n, _ in OTHER])
+def test_full_size_phi4_olmo2_sampled_rows(name, shape):
+    """The Phi-4 and OLMo-2-7B linears of the bench at full size, 2/3/4 bits."""
+    out, inp = shape
+    _sampled_rows_case(out, inp, 128, 2, 0.005, 2000 + out + inp, (2, 3, 4), (0,), batch4=False)
+
+
+@pytest.mark.parametrize("group,density", [(64, 0.0), (128, 0.001), (64, 0.01)])
+def test_full_size_sweep_sampled_rows(group, density):
+    """The precision/structure sweep: base + 4 planes read at 2..6 bits."""
+    _sampled_rows_case(14336, 4096, group, 4, density, 3000 + group, (2, 3, 4, 5, 6), _kernels(), batch4=False)
