@@ -17,7 +17,9 @@ in ``per_gemv``.
 
 The default workload is the Llama-3.1-8B layer above. The others print one
 JSON line each with per-GEMV (or per-token) times:
-  phi4_olmo2_linears_b1  Phi-4 and OLMo-2-7B linears at 2/3/4 bits, batch 1;
+  phi4_olmo2_linears_b1  Phi-4 and OLMo-2-7B linears at 2/3/4 bits, batch 1,
+                         each alone and as one layer's chain (q k v o gate up
+                         down, one CUDA graph);
   precision_sweep        14336x4096 and 4096x14336 with base + 4 planes, read at
                          2..6 bits, group 64 and 128, side record 0 / 0.1 / 1 %;
   llama31_8b_stack       32 layers x 7 linears (6.98e9 weights) resident on the
@@ -47,7 +49,7 @@ GROUP, N_PLANES, DENSITY = 128, 2, 0.005
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["quantized_gemv_stagq_b200/csrc/gemv.cu", "quantized_gemv_stagq_b200/csrc/gemv1.cu",
                   "quantized_gemv_stagq_b200/csrc/kernel_common.cuh", "quantized_gemv_stagq_b200/csrc/layout.cuh"]
-LARGE_WEIGHTS = 1 << 25  # from this many weights on, n = 1 runs the single-vector kernel (gemv1)
+LARGE_WEIGHTS = 1 << 24  # above this many weights, n = 1 runs the single-vector kernel (gemv1)
 
 
 def _args():
@@ -153,7 +155,7 @@ def _kernel_of(key):
     """Name of the kernel that serves the GEMV `name@pM` at n = 1."""
     from quantized_gemv_stagq_b200 import synth
     out, inp = synth.LLAMA31_8B_LINEARS[key.split("@")[0]]
-    return "gemv1_kernel" if out * inp >= LARGE_WEIGHTS else "gemv_kernel"
+    return "gemv1_kernel" if out * inp > LARGE_WEIGHTS else "gemv_kernel"
 
 
 def _layer_shapes():
@@ -309,10 +311,66 @@ def run_extra(args):
                 m.free()
             del S
 
+    def layer_chain(model, linears, bits_list, group, n_planes, density):
+        """One layer's linears in order as one CUDA graph (the chain a decode
+        step runs), rotating over enough device copies that reads come from
+        HBM; µs per layer."""
+        nonlocal launches
+        enc = {}
+        for _, (out, inp) in linears:
+            if (out, inp) not in enc:
+                enc[(out, inp)] = Q.stagq_pack(Q.stagq_encode(synth.weights(out, inp, seed=out + 3 * inp), group,
+                                                              n_planes, density, "fast"))
+        first = [Q.stagq_load(enc[v], 0) for _, v in linears]
+        C = copies_for(Q, sum(m.device_bytes for m in first), l2, minimum=2)
+        mats = [first] + [[Q.stagq_load(enc[v], 0) for _, v in linears] for _ in range(C - 1)]
+        xs = {inp: torch.from_numpy(synth.activations(1, inp, seed=inp)).cuda() for _, (_, inp) in linears}
+        ys = [torch.empty(1, out, dtype=torch.float16, device="cuda") for _, (out, _) in linears]
+        for b in bits_list:
+            def body(c):
+                for j, (_, (out, inp)) in enumerate(linears):
+                    Q.stagq_gemv(mats[c][j], b, xs[inp], ys[j], stream=stream)
+            with torch.cuda.stream(stream):
+                body(0)
+            torch.cuda.synchronize()
+            reps = 2 * C
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for r in range(reps):
+                    body(r % C)
+            g.replay()
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(3):
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    a0.record(stream)
+                    for _ in range(4):
+                        g.replay()
+                    a1.record(stream)
+                torch.cuda.synchronize()
+                ts.append(a0.elapsed_time(a1) * 1e3 / (4 * reps))
+            launches += len(linears) * (1 + 13 * reps)
+            us = statistics.median(ts)
+            nb = sum(Q.stagq_bytes(m, b, 1) for m in first)
+            results[f"{model} layer p{b}"] = {"us": round(us, 3), "bytes": nb, "gbs": round(nb / us / 1e3, 1),
+                                              "frac": round(nb / us / 1e3 / peak, 4), "gemvs": len(linears)}
+            del g
+        for L in mats:
+            for m in L:
+                m.free()
+
     if args.workload == "phi4_olmo2_linears_b1":
         shapes = [("phi4." + k, v) for k, v in synth.PHI4_LINEARS.items()] + \
                  [("olmo2." + k, v) for k, v in synth.OLMO2_7B_LINEARS.items()]
         per_gemv(shapes, BITS, GROUP, N_PLANES, DENSITY)
+        P, O = synth.PHI4_LINEARS, synth.OLMO2_7B_LINEARS
+        layer_chain("phi4", [("q", P["qo"]), ("k", P["kv"]), ("v", P["kv"]), ("o", P["qo"]),
+                             ("gate", P["gate_up"]), ("up", P["gate_up"]), ("down", P["down"])],
+                    BITS, GROUP, N_PLANES, DENSITY)
+        layer_chain("olmo2", [("q", O["qkvo"]), ("k", O["qkvo"]), ("v", O["qkvo"]), ("o", O["qkvo"]),
+                              ("gate", O["gate_up"]), ("up", O["gate_up"]), ("down", O["down"])],
+                    BITS, GROUP, N_PLANES, DENSITY)
         cfg = {"linears_out_x_in": {k: list(v) for k, v in shapes}, "bits": list(BITS), "group": GROUP,
                "n_planes": N_PLANES, "side_record_density": DENSITY, "batch": 1}
     elif args.workload == "precision_sweep":

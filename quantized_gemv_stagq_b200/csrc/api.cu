@@ -242,12 +242,13 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   if (m.smem_pair_budget > smem_limit) m.smem_pair_budget = smem_limit;
   for (int b = 2; b <= 2 + np; ++b)
     for (int nb = 1; nb <= STAGQ_MAX_BATCH; ++nb) h->plan_ok[b][nb] = make_plan(m, b, nb, &h->plan[b][nb]);
-  // The single-vector kernel serves n = 1 on large matrices (>= 2^25 weights:
-  // Llama-3.1-8B gate/up/down): there its faster block loop outweighs its
-  // extra once-per-launch phases (entry rows, side-record terms, row sums),
-  // measured over a whole layer's chain of GEMVs at 2, 3 and 4 bits. On
-  // smaller matrices those phases dominate and the general kernel is faster.
-  const bool large = (int64_t)s->out * s->in >= ((int64_t)1 << 25);
+  // The single-vector kernel serves n = 1 on matrices of more than 2^24
+  // weights (Llama-3.1-8B gate/up/down, Phi-4 and OLMo-2 q/o/gate/up/down):
+  // there its faster block loop outweighs its extra once-per-launch phases
+  // (entry rows, side-record terms, row sums), measured on chains of GEMVs at
+  // 2..6 bits. On smaller matrices those phases dominate and the general
+  // kernel is faster.
+  const bool large = (int64_t)s->out * s->in > ((int64_t)1 << 24);
   for (int b = 2; b <= 2 + np; ++b) {
     h->plan1_ok[b] = make_plan1(m, b, &h->plan1[b]);
     h->prefer1[b] = large;

@@ -15,10 +15,12 @@
 //    memory ring slot with 1 + (M - 2) bulk copies. Warps 1..NW are consumers:
 //    KW K slices (2048 weights: 32 lanes x one 64-weight chunk) x RG row
 //    groups; in every block a consumer takes UP rows of its group in its slice.
-//  * The CTA uses at most half of an SM (<= 9 warps x 96 registers, <= half the
-//    shared memory), so the next GEMV's CTA is resident beside it and fills its
-//    ring -- weights, pair table, the CTA's pair bytes and side record do not
-//    depend on earlier kernels -- before this one finishes.
+//  * The CTA uses at most half of an SM (<= 9 warps x 96 registers, <= half
+//    the shared memory) wherever its ring still fits, so the next GEMV's CTA
+//    is resident beside it and fills its ring -- weights, pair table, the
+//    CTA's pair bytes and side record do not depend on earlier kernels --
+//    before this one finishes. Where it does not fit, the CTA has 12 or more
+//    consumer warps and the SM to itself (make_plan1).
 //  * x is converted once per CTA to 16-bit fixed point with a power-of-two
 //    scale per 64-element chunk (|error| <= 2^-16 max|x_chunk|); each lane keeps
 //    its chunk's 64 activations in registers; code bytes / nibble composites
@@ -51,7 +53,7 @@ namespace {
 
 using namespace kernels;
 
-constexpr int kRegs1 = 96;             // registers per thread: two 9-warp CTAs fit one SM
+constexpr int kRegs1 = 96;             // registers per thread: two 9-warp CTAs fit one SM, or one of 20
 constexpr int kParts1 = 8;             // partial sums per (row, K slice), each over 4 lanes
 
 struct Gemv1Args {
@@ -472,13 +474,62 @@ int gemv1_grid(int out, int num_sms) {
   return g;
 }
 
+// Ring depth and shape (measured on B200 over the Llama-3.1-8B, Phi-4 and
+// OLMo-2 linears at 2..6 bits, alone and in a layer's chain of GEMVs):
+//  * A CTA that takes at most half of an SM (registers and shared memory)
+//    lets the next GEMV's CTA, whatever its kernel, start beside it; in a
+//    chain of different GEMVs that overlap is worth more than any ring shape,
+//    so such a plan is taken whenever one fits (side record staged, 2 or more
+//    rows per warp per block, 3 or more slots or all blocks).
+//  * About 60 KB of weights in flight per SM hide the HBM latency: the ring
+//    grows to that from 3 slots where the budget allows.
+//  * A CTA that cannot be that small gets the SM to itself, and then 12 or
+//    more consumer warps (the loop is bound by integer issue, and more warps
+//    hide its latencies).
+//  * Larger blocks (UP = 4) amortise the per-block waits and sums, as long as
+//    the CTA's rows still make about 5 blocks to pipeline.
+constexpr uint32_t kInflightTarget = 60u * 1024u;
+constexpr int kWideWarps = 12;
+constexpr int kMinBlocks = 5;
+
+// Plan for one (row groups, shared-memory budget): false if nothing fits.
+// `strict`: only plans with the side record staged and 2 or more rows per
+// warp per block.
+bool plan1_fit(const DeviceMatrix& m, int bits, const Gemv1Plan& q, uint32_t budget, bool strict, Gemv1Plan* out) {
+  const int nblk4 = (q.rows_cap + 4 * q.RG - 1) / (4 * q.RG);
+  const int nblk2 = (q.rows_cap + 2 * q.RG - 1) / (2 * q.RG);
+  const int up0 = (nblk4 >= kMinBlocks || nblk2 < kMinBlocks) ? 4 : 2;
+  for (int stage = 1; stage >= (strict ? 1 : 0); --stage) {
+    for (int up = up0; up >= (strict ? 2 : 1); up /= 2) {
+      Gemv1Plan t = q;
+      t.up = up;
+      t.br = q.RG * up;
+      t.stage_side = stage;
+      const int nblk = (q.rows_cap + t.br - 1) / t.br;
+      const int ns_min = nblk < 3 ? nblk : 3;
+      const int ns_max = nblk < kMaxSlots ? nblk : kMaxSlots;
+      t.ns = 0;
+      for (int ns = ns_min; ns <= ns_max; ++ns) {
+        t.ns = ns;
+        if (smem1(t, m.in, bits).total > budget) {
+          t.ns = ns - 1;
+          break;
+        }
+        if ((uint32_t)ns * smem1(t, m.in, bits).slot >= kInflightTarget) break;
+      }
+      if (t.ns < ns_min) continue;
+      *out = t;
+      return true;
+    }
+  }
+  return false;
+}
+
 bool make_plan1(const DeviceMatrix& m, int bits, Gemv1Plan* p) {
+  constexpr int kRegFileWarps = 4 * (16384 / (32 * kRegs1));  // warps the register file holds
   Gemv1Plan q = {};
   q.KW = (m.in / kChunk + 31) / 32;
   if (q.KW < 1 || q.KW > kMaxWarps) return false;
-  q.RG = row_groups(q.KW);
-  q.NW = q.KW * q.RG;
-  if (q.NW + 1 > 4 * (16384 / (32 * kRegs1))) return false;  // register file of the four sub-partitions
   q.grid = m.side1_grid;
   if (q.grid < 1) return false;
   q.rows_cap = (m.out + q.grid - 1) / q.grid;
@@ -489,41 +540,32 @@ bool make_plan1(const DeviceMatrix& m, int bits, Gemv1Plan* p) {
   q.group_shift = 0;
   while ((1 << q.group_shift) < m.group) ++q.group_shift;
   q.pdl = 1;
-  const int per_rg = (q.rows_cap + q.RG - 1) / q.RG;
-  const int up_max = per_rg >= 4 ? 4 : per_rg >= 2 ? 2 : 1;
-  // Shared memory: at most half an SM when two CTAs' warps fit the register
-  // file, so the next GEMV's CTA can be resident beside this one; else the
-  // per-block maximum. Prefer the side record staged, then at least three
-  // slots (or one per block), then more rows per warp.
-  const bool pairable = 2 * (q.NW + 1) <= 4 * (16384 / (32 * kRegs1));
-  const int budgets[2] = {pairable ? m.smem_pair_budget : m.smem_limit, m.smem_limit};
-  for (int bi = 0; bi < 2; ++bi) {
-    for (int stage = 1; stage >= 0; --stage) {
-      bool have = false;
-      Gemv1Plan best = q;
-      for (int up = up_max; up >= 1; up /= 2) {
-        Gemv1Plan t = q;
-        t.up = up;
-        t.br = q.RG * up;
-        t.stage_side = stage;
-        const int nblk = (q.rows_cap + t.br - 1) / t.br;
-        t.ns = nblk < kMaxSlots ? nblk : kMaxSlots;
-        while (t.ns >= 1 && smem1(t, m.in, bits).total > (uint32_t)budgets[bi]) --t.ns;
-        if (t.ns < 1) continue;
-        if (t.ns >= (nblk < 3 ? nblk : 3)) {
-          *p = t;
-          return true;
-        }
-        if (!have || t.ns > best.ns) {
-          best = t;
-          have = true;
-        }
-      }
-      if (have) {
-        *p = best;
-        return true;
-      }
+
+  // Row groups. Narrow: 8 consumer warps for rows of 1 or 2 K slices (RG =
+  // 8 / KW), one per K slice beyond. Wide: at least kWideWarps consumer warps
+  // where the register file holds them.
+  const int rg_narrow = row_groups(q.KW);
+  int rg_wide = (kWideWarps + q.KW - 1) / q.KW;
+  while (rg_wide > rg_narrow && q.KW * rg_wide + 1 > kRegFileWarps) --rg_wide;
+  if (rg_wide < rg_narrow) rg_wide = rg_narrow;
+  if (q.KW * rg_narrow + 1 > kRegFileWarps) return false;
+  Gemv1Plan t;
+
+  // Half an SM (registers and shared memory) when it fits, else the wide CTA
+  // alone on its SM.
+  if (2 * (q.KW * rg_narrow + 1) <= kRegFileWarps) {
+    q.RG = rg_narrow;
+    q.NW = q.KW * q.RG;
+    if (plan1_fit(m, bits, q, (uint32_t)m.smem_pair_budget, true, &t)) {
+      *p = t;
+      return true;
     }
+  }
+  q.RG = rg_wide;
+  q.NW = q.KW * q.RG;
+  if (plan1_fit(m, bits, q, (uint32_t)m.smem_limit, false, &t)) {
+    *p = t;
+    return true;
   }
   return false;
 }
