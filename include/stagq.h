@@ -48,7 +48,12 @@ extern "C" {
 #define STAGQ_MAX_BATCH 4       /* columns of x per call in stagq_gemv_n */
 #define STAGQ_MAX_IN 32768      /* K; side-record columns are stored as uint16 */
 #define STAGQ_IN_MULTIPLE 128   /* K must be a multiple of this (16-byte plane rows) */
-/* The group size of a loadable stream is a power of two, at least 64, dividing K. */
+/* The group size of a loadable stream is a power of two, at least this, dividing
+ * K. Groups of 16 and 32 are the paper's encoder settings (Table 6), and its
+ * kernel evaluation runs at 32 (Section 4.3, Table 5), where the 8-bit pair
+ * costs 0.25 bpw; the kernels then apply G = 64 / group affines per
+ * 64-weight chunk. */
+#define STAGQ_MIN_GROUP 16
 
 /* Pair search mode of the encoder (Section 3.1). */
 #define STAGQ_PAIR_SEARCH 0     /* argmin of Eq. (5) over all 256 codebook pairs */

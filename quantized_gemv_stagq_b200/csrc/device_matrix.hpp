@@ -25,6 +25,11 @@ __host__ __device__ inline int xq_slot_of_column(int col) {
   const int c = col >> 6, e = col & 63;
   return xq_piece_index(c, e >> 3) * 8 + (e & 7);
 }
+// The column whose element slot is `slot` (inverse of xq_slot_of_column).
+__host__ __device__ inline int column_of_xq_slot(int slot) {
+  const int c = slot >> 6, piece_slot = (slot >> 3) & 7;
+  return c * 64 + ((piece_slot - c) & 7) * 8 + (slot & 7);
+}
 
 struct DeviceMatrix {
   int32_t out, in, group, n_planes;

@@ -93,7 +93,7 @@ constexpr uint64_t kDrainLimitNs = 100000000ull;   // after a failure: wait for 
 
 // Shared-memory carve-up, identical on host (plan) and device.
 struct SmemLayout {
-  uint32_t bar, cnt, last, tab, xq, xscale, xsum, lo, partial, side, ring;
+  uint32_t bar, cnt, last, tab, xq, xscale, xsum, xsum16, lo, partial, side, ring;
   uint32_t slot;                 // bytes of one ring slot
   uint32_t plane_piece, pair_piece;  // offsets inside a slot (base rows at 0)
   uint32_t total;
@@ -113,8 +113,10 @@ __host__ __device__ inline SmemLayout smem_layout(const GemvPlan& p, int in, int
   L.xq = o; o += 2u * in * p.nb;        // x~ of each of the nb vectors
   L.xscale = o; o += 4u * nchunk * p.nb;
   L.xsum = o; o += 4u * nchunk * p.nb;
+  L.xsum16 = o; o += p.group_shift < 6 ? 16u * nchunk * p.nb : 0u;  // per 16 values, for groups < 64
   o = align_up_u32(o, 16);
-  L.lo = o; o += 4u * 32 * p.up * p.NW;  // per warp: lo_M of each lane's group per row of a block
+  // per warp: lo_M of each of a lane's groups per row of a block
+  L.lo = o; o += 4u * 32 * p.up * p.NW * (uint32_t)groups_per_chunk(p.group_shift);
   L.partial = o; o += 4u * p.ns * BR * p.KW * p.nb;  // [slot][BR][KW][nb]
   o = align_up_u32(o, 128);
   L.side = o; o += p.stage_side ? (uint32_t)p.side_stride : 0u;
@@ -129,18 +131,40 @@ __host__ __device__ inline SmemLayout smem_layout(const GemvPlan& p, int in, int
 }
 
 // Dot products of NR rows of one block for this lane's chunk, with the group
-// affine: v[u] = s_M c_M sum(v x~) + lo_M sum(x~) over the chunk, and the
-// lane's lo_M per row (for the side record). Row u of the warp sits at
-// offsets off.b + u * step.b (base), off.p + u * step.p (first read plane;
-// plane k at + k * plane_stride) and off.g + u * step.g (pair byte) in the slot.
+// affine: v[u] = sum over the chunk's G groups of s_M c_M sum(v x~) + lo_M
+// sum(x~) (xsg[g]: sum of x~ over group g), and the lane's lo_M per row and
+// group (for the side record). Row u of the warp sits at offsets off.b + u *
+// step.b (base), off.p + u * step.p (first read plane; plane k at + k *
+// plane_stride) and off.g + u * step.g (its G pair bytes) in the slot.
 struct RowOffsets {
   uint32_t b, p, g;
 };
 
-template <int M, int NR>
-__device__ __forceinline__ void rows_dot(const uint32_t (&X)[32], float xs, float xsm, const uint8_t* sb,
+// v = sum_g s_M c_M tot[g] xs + lo_M xsg[g] for the G pair bytes in `pairs`
+// (byte g = group g); lo[g] = lo_M of group g.
+template <int G>
+__device__ __forceinline__ float group_affine(const float2* tab, uint32_t pairs, const int (&tot)[G], float xs,
+                                              const float (&xsg)[G], float (&lo)[G]) {
+  if constexpr (G == 1) {
+    const float2 l = tab[pairs];
+    lo[0] = l.x;
+    return fmaf(l.y, (float)tot[0] * xs, l.x * xsg[0]);
+  } else {
+    float acc = 0.f;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float2 l = tab[(pairs >> (8 * g)) & 0xFFu];
+      lo[g] = l.x;
+      acc = fmaf(l.y, (float)tot[g] * xs, fmaf(l.x, xsg[g], acc));
+    }
+    return acc;
+  }
+}
+
+template <int M, int NR, int G>
+__device__ __forceinline__ void rows_dot(const uint32_t (&X)[32], float xs, const float (&xsg)[G], const uint8_t* sb,
                                          RowOffsets off, RowOffsets step, uint32_t plane_stride, const float2* tab,
-                                         float (&v)[NR], float (&lo)[NR]) {
+                                         float (&v)[NR], float (&lo)[NR][G]) {
 #pragma unroll
   for (int u = 0; u < NR; ++u) {
     const uint4 b4 = *reinterpret_cast<const uint4*>(sb + off.b + u * step.b);
@@ -149,25 +173,25 @@ __device__ __forceinline__ void rows_dot(const uint32_t (&X)[32], float xs, floa
 #pragma unroll
     for (int k = 0; k < M - 2; ++k)
       Pw[k] = *reinterpret_cast<const uint2*>(sb + off.p + u * step.p + k * plane_stride);
-    const int tot = chunk_dot<M>(X, B, Pw);
-    const float2 lm = tab[sb[off.g + u * step.g]];
-    v[u] = fmaf(lm.y, (float)tot * xs, lm.x * xsm);
-    lo[u] = lm.x;
+    int tot[G];
+    chunk_dot_g<M, G>(X, B, Pw, tot);
+    v[u] = group_affine<G>(tab, load_pairs<G>(sb + off.g + u * step.g), tot, xs, xsg, lo[u]);
   }
 }
 
 // As rows_dot for NB activation vectors (NB > 1): the slot's code words are
 // read once and dotted with each vector's x~, which is taken from shared
 // memory vector by vector (x~ of vector j at xq + j * in, its chunk scales at
-// xscale / xsum + j * nchunk). v[j][u] is row u against vector j.
-template <int M, int NR, int NB>
-__device__ __forceinline__ void rows_dot_nb(const int16_t* xq, const float* xscale, const float* xsum, int in,
-                                            int nchunk, int cc, bool active, const uint8_t* sb, RowOffsets off,
-                                            RowOffsets step, uint32_t plane_stride, const float2* tab,
-                                            float (&v)[NB][NR], float (&lo)[NR]) {
+// xscale / xsum + j * nchunk, its 16-value sums at xsum16 + 4 j nchunk). v[j][u]
+// is row u against vector j.
+template <int M, int NR, int NB, int G>
+__device__ __forceinline__ void rows_dot_nb(const int16_t* xq, const float* xscale, const float* xsum,
+                                            const float* xsum16, int in, int nchunk, int cc, bool active,
+                                            const uint8_t* sb, RowOffsets off, RowOffsets step, uint32_t plane_stride,
+                                            const float2* tab, float (&v)[NB][NR], float (&lo)[NR][G]) {
   uint32_t B[NR][4];
   uint2 Pw[NR][M > 2 ? M - 2 : 1];
-  float2 lm[NR];
+  uint32_t pr[NR];
 #pragma unroll
   for (int u = 0; u < NR; ++u) {
     const uint4 b4 = *reinterpret_cast<const uint4*>(sb + off.b + u * step.b);
@@ -175,8 +199,7 @@ __device__ __forceinline__ void rows_dot_nb(const int16_t* xq, const float* xsca
 #pragma unroll
     for (int k = 0; k < M - 2; ++k)
       Pw[u][k] = *reinterpret_cast<const uint2*>(sb + off.p + u * step.p + k * plane_stride);
-    lm[u] = tab[sb[off.g + u * step.g]];
-    lo[u] = lm[u].x;
+    pr[u] = load_pairs<G>(sb + off.g + u * step.g);
   }
 #pragma unroll
   for (int j = 0; j < NB; ++j) {
@@ -191,33 +214,53 @@ __device__ __forceinline__ void rows_dot_nb(const int16_t* xq, const float* xsca
       X[4 * k + 3] = t.w;
     }
     const float xs = active ? xscale[j * nchunk + cc] : 0.f;
-    const float xsm = active ? xsum[j * nchunk + cc] : 0.f;
+    float xsg[G];
+    if constexpr (G == 1) {
+      xsg[0] = active ? xsum[j * nchunk + cc] : 0.f;
+    } else {
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float t = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4 / G; ++q) t += xsum16[4 * (j * nchunk + cc) + (4 / G) * g + q];
+        xsg[g] = active ? t : 0.f;
+      }
+    }
 #pragma unroll
     for (int u = 0; u < NR; ++u) {
-      const int tot = chunk_dot<M>(X, B[u], Pw[u]);
-      v[j][u] = fmaf(lm[u].y, (float)tot * xs, lm[u].x * xsm);
+      int tot[G];
+      chunk_dot_g<M, G>(X, B[u], Pw[u], tot);
+      v[j][u] = group_affine<G>(tab, pr[u], tot, xs, xsg, lo[u]);
     }
   }
+}
+
+// Where lo_M of column `col`'s group sits among a row's per-lane lo values
+// (G per lane: lane (col >> 6) & 31, group (col >> gs) within its chunk).
+template <int G>
+__device__ __forceinline__ int lo_index(int col, int gs) {
+  if constexpr (G == 1) return (col >> 6) & 31;
+  else return ((col >> 6) & 31) * G + ((col >> gs) & (G - 1));
 }
 
 // Held-out entries of NR consecutive rows of the warp's row class in its K
 // slice: row u owns entries [o_lo, o_hi) of the CTA's side record, handled by
 // the 32 / NR lanes of group u (lane / (32 / NR)). Adds x~_c (v - lo_M) to
-// v[u]; lo_M of column c's group is read from lo_s[u][c's lane], where every
-// lane of the warp left its own lo_M per row.
-template <int NR>
+// v[u]; lo_M of column c's group is read from lo_s[u][c's lane][group], where
+// every lane of the warp left its own lo_M per row and group.
+template <int NR, int G>
 __device__ __forceinline__ void side_record(int o_lo, int o_hi, const uint32_t* ents, const int16_t* xq,
-                                            const float* xscale, const float* lo_s, int lane, float (&v)[NR]) {
+                                            const float* xscale, const float* lo_s, int lane, int gs, float (&v)[NR]) {
   constexpr int LPR = 32 / NR;  // lanes per row
   const int ur = lane / LPR;
-  const float* lo_row = lo_s + ur * 32;
+  const float* lo_row = lo_s + ur * 32 * G;
   float cs = 0.f;
   for (int j = o_lo + lane % LPR; __any_sync(kFull, j < o_hi); j += LPR) {
     if (j < o_hi) {
       const uint32_t en = ents[j];
       const int col = (int)(en & 0xFFFFu);
       const float xv = (float)xq[xq_elem(col)] * xscale[col >> 6];
-      cs = fmaf(xv, __half2float(__ushort_as_half((unsigned short)(en >> 16))) - lo_row[(col >> 6) & 31], cs);
+      cs = fmaf(xv, __half2float(__ushort_as_half((unsigned short)(en >> 16))) - lo_row[lo_index<G>(col, gs)], cs);
     }
   }
 #pragma unroll
@@ -225,13 +268,13 @@ __device__ __forceinline__ void side_record(int o_lo, int o_hi, const uint32_t* 
 }
 
 // As side_record for NB activation vectors: v[j][u] += x~_j,c (v - lo_M).
-template <int NR, int NB>
+template <int NR, int NB, int G>
 __device__ __forceinline__ void side_record_nb(int o_lo, int o_hi, const uint32_t* ents, const int16_t* xq,
                                                const float* xscale, int in, int nchunk, const float* lo_s, int lane,
-                                               float (&v)[NB][NR]) {
+                                               int gs, float (&v)[NB][NR]) {
   constexpr int LPR = 32 / NR;  // lanes per row
   const int ur = lane / LPR;
-  const float* lo_row = lo_s + ur * 32;
+  const float* lo_row = lo_s + ur * 32 * G;
   float cs[NB];
 #pragma unroll
   for (int j = 0; j < NB; ++j) cs[j] = 0.f;
@@ -239,7 +282,7 @@ __device__ __forceinline__ void side_record_nb(int o_lo, int o_hi, const uint32_
     if (e < o_hi) {
       const uint32_t en = ents[e];
       const int col = (int)(en & 0xFFFFu);
-      const float d = __half2float(__ushort_as_half((unsigned short)(en >> 16))) - lo_row[(col >> 6) & 31];
+      const float d = __half2float(__ushort_as_half((unsigned short)(en >> 16))) - lo_row[lo_index<G>(col, gs)];
       const int xe = xq_elem(col);
 #pragma unroll
       for (int j = 0; j < NB; ++j) cs[j] = fmaf((float)xq[j * in + xe] * xscale[j * nchunk + (col >> 6)], d, cs[j]);
@@ -254,27 +297,32 @@ __device__ __forceinline__ void side_record_nb(int o_lo, int o_hi, const uint32_
 // The UP rows (or, for a short block, `mine` rows one at a time) of one block
 // for this lane's chunk: dot products, side record, and the cross-lane sums
 // into pout[u * pstep + j] (row u, vector j).
-template <int M, int NR, int NB>
-__device__ __forceinline__ void block_rows(const uint32_t (&X)[32], float xs, float xsm, const int16_t* xq,
-                                           const float* xscale, const float* xsum, int in, int nchunk, int cc,
-                                           bool active, const uint8_t* sb, RowOffsets off, RowOffsets step,
-                                           uint32_t plane_stride, const float2* tab, int mine, const int32_t* o,
-                                           const uint32_t* ents, float* lo_w, int lane, float* pout, int pstep) {
-  float v[NB][NR], lo[NR];
+template <int M, int NR, int NB, int G>
+__device__ __forceinline__ void block_rows(const uint32_t (&X)[32], float xs, const float (&xsg)[G], const int16_t* xq,
+                                           const float* xscale, const float* xsum, const float* xsum16, int in,
+                                           int nchunk, int cc, bool active, const uint8_t* sb, RowOffsets off,
+                                           RowOffsets step, uint32_t plane_stride, const float2* tab, int mine,
+                                           const int32_t* o, const uint32_t* ents, float* lo_w, int lane, int gs,
+                                           float* pout, int pstep) {
+  float v[NB][NR], lo[NR][G];
   if constexpr (NB == 1) {
-    rows_dot<M, NR>(X, xs, xsm, sb, off, step, plane_stride, tab, v[0], lo);
+    rows_dot<M, NR, G>(X, xs, xsg, sb, off, step, plane_stride, tab, v[0], lo);
   } else {
-    rows_dot_nb<M, NR, NB>(xq, xscale, xsum, in, nchunk, cc, active, sb, off, step, plane_stride, tab, v, lo);
+    rows_dot_nb<M, NR, NB, G>(xq, xscale, xsum, xsum16, in, nchunk, cc, active, sb, off, step, plane_stride, tab, v,
+                              lo);
   }
 #pragma unroll
-  for (int u = 0; u < NR; ++u) lo_w[u * 32 + lane] = lo[u];
+  for (int u = 0; u < NR; ++u)
+#pragma unroll
+    for (int g = 0; g < G; ++g) lo_w[(u * 32 + lane) * G + g] = lo[u][g];
   __syncwarp();
   const int ur = lane / (32 / NR);
   if constexpr (NB == 1) {
-    side_record<NR>(o[ur < mine ? ur : mine], o[ur + 1 < mine ? ur + 1 : mine], ents, xq, xscale, lo_w, lane, v[0]);
+    side_record<NR, G>(o[ur < mine ? ur : mine], o[ur + 1 < mine ? ur + 1 : mine], ents, xq, xscale, lo_w, lane, gs,
+                       v[0]);
   } else {
-    side_record_nb<NR, NB>(o[ur < mine ? ur : mine], o[ur + 1 < mine ? ur + 1 : mine], ents, xq, xscale, in, nchunk,
-                           lo_w, lane, v);
+    side_record_nb<NR, NB, G>(o[ur < mine ? ur : mine], o[ur + 1 < mine ? ur + 1 : mine], ents, xq, xscale, in,
+                              nchunk, lo_w, lane, gs, v);
   }
 #pragma unroll
   for (int j = 0; j < NB; ++j) {
@@ -283,7 +331,7 @@ __device__ __forceinline__ void block_rows(const uint32_t (&X)[32], float xs, fl
   }
 }
 
-template <int M, int UP, int NB>
+template <int M, int UP, int NB, int G>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKernelArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const GemvPlan& P = a.plan;
@@ -295,8 +343,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
   int16_t* xq = reinterpret_cast<int16_t*>(smem + L.xq);
   float* xscale = reinterpret_cast<float*>(smem + L.xscale);
   float* xsum = reinterpret_cast<float*>(smem + L.xsum);
+  float* xsum16 = reinterpret_cast<float*>(smem + L.xsum16);
   float* partial = reinterpret_cast<float*>(smem + L.partial);  // [slot][BR][KW]
-  float* lo_w = reinterpret_cast<float*>(smem + L.lo) + 32 * UP * (threadIdx.x >> 5);
+  float* lo_w = reinterpret_cast<float*>(smem + L.lo) + 32 * UP * G * (threadIdx.x >> 5);
   uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + L.cnt);
   int* last = reinterpret_cast<int*>(smem + L.last);
   const uint32_t full0 = sbase + L.bar, side_bar = sbase + L.bar + 8 * kMaxSlots;
@@ -398,6 +447,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
           Q[k] = __byte_perm(__float_as_uint(fmaf(f.x, sc, kShift)), __float_as_uint(fmaf(f.y, sc, kShift)), 0x5410);
           sumq = dp2a_lo(Q[k], 0x0101u, sumq);
         }
+        const int sum16 = sumq;
         sumq += __shfl_xor_sync(kFull, sumq, 1);
         sumq += __shfl_xor_sync(kFull, sumq, 2);
         if (t < ntask) {
@@ -405,6 +455,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
           uint4* dst = reinterpret_cast<uint4*>(xq + j * in);
           dst[xq_piece(tt >> 2, 2 * (tt & 3))] = make_uint4(Q[0], Q[1], Q[2], Q[3]);
           dst[xq_piece(tt >> 2, 2 * (tt & 3) + 1)] = make_uint4(Q[4], Q[5], Q[6], Q[7]);
+          if constexpr (G > 1) xsum16[t] = __int_as_float((127 - e) << 23) * (float)sum16;  // t = 4 (j nchunk + c) + q
           if ((tt & 3) == 0) {
             const float xs_c = __int_as_float((127 - e) << 23);
             xscale[j * nchunk + (tt >> 2)] = xs_c;
@@ -416,7 +467,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
   }
   __syncthreads();
   uint32_t X[32];  // one vector: this lane's x~ stays in registers (more vectors: read per block)
-  float xs = 0.f, xsm = 0.f;
+  float xs = 0.f, xsg[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) xsg[g] = 0.f;
   if constexpr (NB == 1) {
     const uint4* src = reinterpret_cast<const uint4*>(xq);
 #pragma unroll
@@ -428,7 +481,17 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
       X[4 * k + 3] = t.w;
     }
     xs = active ? xscale[cc] : 0.f;
-    xsm = active ? xsum[cc] : 0.f;
+    if constexpr (G == 1) {
+      xsg[0] = active ? xsum[cc] : 0.f;
+    } else {
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float t = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4 / G; ++q) t += xsum16[4 * cc + (4 / G) * g + q];  // exact: multiples of one 2^-e
+        xsg[g] = active ? t : 0.f;
+      }
+    }
   }
 
   // Where this warp's rows sit in a slot (row u of the warp = block row rg + RG u).
@@ -455,13 +518,13 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
     // missing rows masked, unless fewer than half of them are there
     const int mine = nr == BR ? UP : (nr > rg ? (nr - rg + RG - 1) / RG : 0);
     if (mine == UP || 2 * mine > UP) {
-      block_rows<M, UP, NB>(X, xs, xsm, xq, xscale, xsum, in, nchunk, cc, active, sb, off, step, plane_stride, tab,
-                            mine, o, ents, lo_w, lane, pout, pstep);
+      block_rows<M, UP, NB, G>(X, xs, xsg, xq, xscale, xsum, xsum16, in, nchunk, cc, active, sb, off, step,
+                               plane_stride, tab, mine, o, ents, lo_w, lane, P.group_shift, pout, pstep);
     } else {
       for (int u = 0; u < mine; ++u) {
         const RowOffsets ou = {off.b + u * step.b, off.p + u * step.p, off.g + u * step.g};
-        block_rows<M, 1, NB>(X, xs, xsm, xq, xscale, xsum, in, nchunk, cc, active, sb, ou, step, plane_stride, tab,
-                             1, o + u, ents, lo_w, lane, pout + u * pstep, pstep);
+        block_rows<M, 1, NB, G>(X, xs, xsg, xq, xscale, xsum, xsum16, in, nchunk, cc, active, sb, ou, step,
+                                plane_stride, tab, 1, o + u, ents, lo_w, lane, P.group_shift, pout + u * pstep, pstep);
         __syncwarp();  // lo_w is rewritten by the next row
       }
     }
@@ -530,11 +593,11 @@ __global__ void decode_levels_kernel(const DeviceMatrix m, uint8_t* u) {
 cudaError_t ensure_smem(const void* kern, int key, size_t smem) {
   constexpr int kMaxDev = 64;
   static std::mutex mu;
-  static size_t granted[kMaxDev][64] = {};  // key < 60: (M - 2, rows per warp, vectors)
+  static size_t granted[kMaxDev][192] = {};  // key < 180: (M - 2, rows per warp, vectors, groups per chunk)
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (dev < 0 || dev >= kMaxDev || key < 0 || key >= 64) return cudaErrorInvalidValue;
+  if (dev < 0 || dev >= kMaxDev || key < 0 || key >= 192) return cudaErrorInvalidValue;
   std::lock_guard<std::mutex> lock(mu);
   if (granted[dev][key] >= smem) return cudaSuccess;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -546,7 +609,7 @@ cudaError_t ensure_smem(const void* kern, int key, size_t smem) {
   return err;
 }
 
-template <int M, int UP, int NB>
+template <int M, int UP, int NB, int G>
 cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const void* x, void* y, int y_f32,
                            cudaStream_t stream) {
   GemvKernelArgs a;
@@ -557,8 +620,8 @@ cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const vo
   a.y = y;
   a.y_f32 = y_f32;
   const SmemLayout L = smem_layout(plan, m.in, M);
-  auto kern = gemv_kernel<M, UP, NB>;
-  const int key = ((M - 2) * 3 + (UP == 4 ? 2 : UP - 1)) * 4 + (NB - 1);
+  auto kern = gemv_kernel<M, UP, NB, G>;
+  const int key = (((M - 2) * 3 + (UP == 4 ? 2 : UP - 1)) * 4 + (NB - 1)) * 3 + (G == 4 ? 2 : G - 1);
   cudaError_t err = ensure_smem(reinterpret_cast<const void*>(kern), key, L.total);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -578,31 +641,47 @@ template <int M>
 cudaError_t launch_gemv_m(const DeviceMatrix& m, const GemvPlan& plan, const void* x, void* y, int y_f32,
                           cudaStream_t stream) {
   // Instances the planner can select (see make_plan): more vectors or deeper
-  // reads take fewer rows per warp, so that the registers do not spill.
+  // reads take fewer rows per warp, so that the registers do not spill;
+  // groups below 64 weights take one row per warp.
+  const int G = groups_per_chunk(plan.group_shift);
+  if (G > 1) {
+    if (plan.up != 1) return cudaErrorInvalidValue;
+    switch (G * 8 + plan.nb) {
+      case 16 + 1: return launch_gemv_mu<M, 1, 1, 2>(m, plan, x, y, y_f32, stream);
+      case 16 + 2: return launch_gemv_mu<M, 1, 2, 2>(m, plan, x, y, y_f32, stream);
+      case 16 + 3: return launch_gemv_mu<M, 1, 3, 2>(m, plan, x, y, y_f32, stream);
+      case 16 + 4: return launch_gemv_mu<M, 1, 4, 2>(m, plan, x, y, y_f32, stream);
+      case 32 + 1: return launch_gemv_mu<M, 1, 1, 4>(m, plan, x, y, y_f32, stream);
+      case 32 + 2: return launch_gemv_mu<M, 1, 2, 4>(m, plan, x, y, y_f32, stream);
+      case 32 + 3: return launch_gemv_mu<M, 1, 3, 4>(m, plan, x, y, y_f32, stream);
+      case 32 + 4: return launch_gemv_mu<M, 1, 4, 4>(m, plan, x, y, y_f32, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   if (plan.nb == 1) {
-    if (plan.up == 1) return launch_gemv_mu<M, 1, 1>(m, plan, x, y, y_f32, stream);
-    if (plan.up == 2) return launch_gemv_mu<M, 2, 1>(m, plan, x, y, y_f32, stream);
-    if (plan.up == 4) return launch_gemv_mu<M, 4, 1>(m, plan, x, y, y_f32, stream);
+    if (plan.up == 1) return launch_gemv_mu<M, 1, 1, 1>(m, plan, x, y, y_f32, stream);
+    if (plan.up == 2) return launch_gemv_mu<M, 2, 1, 1>(m, plan, x, y, y_f32, stream);
+    if (plan.up == 4) return launch_gemv_mu<M, 4, 1, 1>(m, plan, x, y, y_f32, stream);
     return cudaErrorInvalidValue;
   }
   if constexpr (M >= 5) {
     if (plan.up != 1) return cudaErrorInvalidValue;
     switch (plan.nb) {
-      case 2: return launch_gemv_mu<M, 1, 2>(m, plan, x, y, y_f32, stream);
-      case 3: return launch_gemv_mu<M, 1, 3>(m, plan, x, y, y_f32, stream);
-      case 4: return launch_gemv_mu<M, 1, 4>(m, plan, x, y, y_f32, stream);
+      case 2: return launch_gemv_mu<M, 1, 2, 1>(m, plan, x, y, y_f32, stream);
+      case 3: return launch_gemv_mu<M, 1, 3, 1>(m, plan, x, y, y_f32, stream);
+      case 4: return launch_gemv_mu<M, 1, 4, 1>(m, plan, x, y, y_f32, stream);
       default: return cudaErrorInvalidValue;
     }
   } else {
     const int k = (plan.up == 4 ? 2 : plan.up - 1) * 4 + plan.nb;
     switch (k) {
-      case 2: return launch_gemv_mu<M, 1, 2>(m, plan, x, y, y_f32, stream);
-      case 3: return launch_gemv_mu<M, 1, 3>(m, plan, x, y, y_f32, stream);
-      case 4: return launch_gemv_mu<M, 1, 4>(m, plan, x, y, y_f32, stream);
-      case 6: return launch_gemv_mu<M, 2, 2>(m, plan, x, y, y_f32, stream);
-      case 7: return launch_gemv_mu<M, 2, 3>(m, plan, x, y, y_f32, stream);
-      case 8: return launch_gemv_mu<M, 2, 4>(m, plan, x, y, y_f32, stream);
-      case 10: return launch_gemv_mu<M, 4, 2>(m, plan, x, y, y_f32, stream);
+      case 2: return launch_gemv_mu<M, 1, 2, 1>(m, plan, x, y, y_f32, stream);
+      case 3: return launch_gemv_mu<M, 1, 3, 1>(m, plan, x, y, y_f32, stream);
+      case 4: return launch_gemv_mu<M, 1, 4, 1>(m, plan, x, y, y_f32, stream);
+      case 6: return launch_gemv_mu<M, 2, 2, 1>(m, plan, x, y, y_f32, stream);
+      case 7: return launch_gemv_mu<M, 2, 3, 1>(m, plan, x, y, y_f32, stream);
+      case 8: return launch_gemv_mu<M, 2, 4, 1>(m, plan, x, y, y_f32, stream);
+      case 10: return launch_gemv_mu<M, 4, 2, 1>(m, plan, x, y, y_f32, stream);
       default: return cudaErrorInvalidValue;
     }
   }
@@ -656,6 +735,7 @@ bool make_plan(const DeviceMatrix& m, int bits, int nb, GemvPlan* p) {
   // registers: rows x vectors x planes (the instances launch_gemv_m provides)
   if (nb >= 2 && bits >= 5) up_max = 1;
   else if (nb >= 3 && up_max > 2) up_max = 2;
+  if (q.group_shift < 6) up_max = 1;  // groups below 64 weights: G pairs and lo values per row
   // Shared memory: small enough for two CTAs per SM when the CTA has <= 8
   // warps, else (or if nothing fits) the per-block maximum. Prefer the side
   // record staged, then at least three slots (or one per block), then more

@@ -74,7 +74,7 @@ constexpr uint64_t kDrainLimit1Ns = 100000000ull;  // after a failure: wait for 
 __host__ __device__ inline int part_stride1(int KW) { return KW * kParts1 + 4; }
 
 struct Smem1 {
-  uint32_t full, empty, side_bar, flag, tab, xq, xscale, xsum, pairs, side, part, rowid, term, ring;
+  uint32_t full, empty, side_bar, flag, tab, xq, xscale, xsum, xsum16, pairs, side, part, rowid, term, ring;
   uint32_t slot;         // bytes of one ring slot
   uint32_t plane_piece;  // offset of the first read plane inside a slot (base rows at 0)
   uint32_t total;
@@ -94,6 +94,7 @@ __host__ __device__ inline Smem1 smem1(const Gemv1Plan& p, int in, int M) {
   L.xq = o; o += 2 * in;
   L.xscale = o; o += 4 * nchunk;
   L.xsum = o; o += 4 * nchunk;
+  L.xsum16 = o; o += p.group_shift < 6 ? 16 * nchunk : 0u;  // per 16 values, for groups < 64
   o = up16(o);
   L.pairs = o; o += up16(rc * (uint32_t)p.pair_stride);
   L.side = o; o += p.stage_side ? (uint32_t)p.side_stride : 0u;
@@ -141,7 +142,7 @@ __device__ __forceinline__ bool keeps_partial1(int lane) {
   return UP == 4 ? true : UP == 2 ? (lane & 8) == 0 : lane < 8;
 }
 
-template <int M, int UP>
+template <int M, int UP, int G>
 __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const Gemv1Plan& P = a.plan;
@@ -153,6 +154,7 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
   int16_t* xq = reinterpret_cast<int16_t*>(smem + L.xq);
   float* xscale = reinterpret_cast<float*>(smem + L.xscale);
   float* xsum = reinterpret_cast<float*>(smem + L.xsum);
+  float* xsum16 = reinterpret_cast<float*>(smem + L.xsum16);
   float* part = reinterpret_cast<float*>(smem + L.part);  // [row][part_stride1(KW)]: [KW][8] used
   float* term = reinterpret_cast<float*>(smem + L.term);
   uint16_t* rowid = reinterpret_cast<uint16_t*>(smem + L.rowid);
@@ -252,12 +254,14 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
           Q[k] = __byte_perm(__float_as_uint(fmaf(f.x, sc, kShift)), __float_as_uint(fmaf(f.y, sc, kShift)), 0x5410);
           sumq = dp2a_lo(Q[k], 0x0101u, sumq);
         }
+        const int sum16 = sumq;
         sumq += __shfl_xor_sync(kFull, sumq, 1);
         sumq += __shfl_xor_sync(kFull, sumq, 2);
         if (t < ntask) {
           uint4* dst = reinterpret_cast<uint4*>(xq);
           dst[xq_piece(t >> 2, 2 * (t & 3))] = make_uint4(Q[0], Q[1], Q[2], Q[3]);
           dst[xq_piece(t >> 2, 2 * (t & 3) + 1)] = make_uint4(Q[4], Q[5], Q[6], Q[7]);
+          if constexpr (G > 1) xsum16[t] = __int_as_float((127 - e) << 23) * (float)sum16;
           if ((t & 3) == 0) {
             const float xs_c = __int_as_float((127 - e) << 23);
             xscale[t >> 2] = xs_c;
@@ -298,6 +302,7 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
     const int cc = active ? c : 0;           // reads of inactive lanes stay inside the row
     uint32_t X[32];
     float xs, xsm;
+    float xsg[G];  // sum of x~ over each of the chunk's groups (G > 1)
     {
       const uint4* src = reinterpret_cast<const uint4*>(xq);
 #pragma unroll
@@ -310,6 +315,15 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
       }
       xs = active ? xscale[cc] : 0.f;
       xsm = active ? xsum[cc] : 0.f;
+      if constexpr (G > 1) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float t = 0.f;
+#pragma unroll
+          for (int q = 0; q < 4 / G; ++q) t += xsum16[4 * cc + (4 / G) * g + q];  // exact: multiples of one 2^-e
+          xsg[g] = active ? t : 0.f;
+        }
+      }
     }
     // Where this warp's rows sit in a slot (row u of the warp = block row rg + RG u).
     const uint32_t off_b = (uint32_t)(rg * rb + cc * kBaseChunkBytes);
@@ -331,6 +345,7 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
       uint32_t B[UP][4];
       uint2 Pw[UP][M > 2 ? M - 2 : 1];
       float2 lm[UP];
+      uint32_t pw[UP];  // G > 1: the row's G pair bytes of this chunk
 #pragma unroll
       for (int u = 0; u < UP; ++u) {
         const uint4 b4 = *reinterpret_cast<const uint4*>(sb + off_b + u * step_b);
@@ -339,13 +354,26 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
         for (int k = 0; k < M - 2; ++k)
           Pw[u][k] = *reinterpret_cast<const uint2*>(sb + off_p + u * step_p + k * plane_stride);
         const int row = min(lr + RG * u, rows - 1);  // rows past the CTA's end read a valid pair byte
-        lm[u] = tab[pairs[row * ps + pcol]];
+        if constexpr (G == 1) lm[u] = tab[pairs[row * ps + pcol]];
+        else pw[u] = load_pairs<G>(pairs + row * ps + pcol);
       }
       float v[UP];
 #pragma unroll
       for (int u = 0; u < UP; ++u) {
-        const int tot = chunk_dot<M>(X, B[u], Pw[u]);
-        v[u] = fmaf(lm[u].y, (float)tot * xs, lm[u].x * xsm);
+        if constexpr (G == 1) {
+          const int tot = chunk_dot<M>(X, B[u], Pw[u]);
+          v[u] = fmaf(lm[u].y, (float)tot * xs, lm[u].x * xsm);
+        } else {
+          int tot[G];
+          chunk_dot_g<M, G>(X, B[u], Pw[u], tot);
+          float acc = 0.f;
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float2 l = tab[(pw[u] >> (8 * g)) & 0xFFu];
+            acc = fmaf(l.y, (float)tot[g] * xs, fmaf(l.x, xsg[g], acc));
+          }
+          v[u] = acc;
+        }
       }
       const float s = partial_reduce1<UP>(v, lane);
       const int row = lr + RG * urow;
@@ -372,7 +400,8 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
         if (j < j1) {
           const uint32_t en = ents[j];
           const int e = (int)(en & 0xFFFFu);  // x~ slot; e >> 6 is the column's 64-chunk
-          const float lo = tab[pairs[(int)rowid[j] * ps + (e >> gs)]].x;
+          const int grp = G == 1 ? e >> gs : column_of_xq_slot(e) >> gs;  // the column's group
+          const float lo = tab[pairs[(int)rowid[j] * ps + grp]].x;
           term[j] = (float)xq[e] * xscale[e >> 6] * (__half2float(__ushort_as_half((unsigned short)(en >> 16))) - lo);
         }
       }
@@ -415,11 +444,11 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
 cudaError_t ensure_smem1(const void* kern, int key, size_t smem) {
   constexpr int kMaxDev = 64;
   static std::mutex mu;
-  static size_t granted[kMaxDev][16] = {};
+  static size_t granted[kMaxDev][64] = {};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (dev < 0 || dev >= kMaxDev || key < 0 || key >= 16) return cudaErrorInvalidValue;
+  if (dev < 0 || dev >= kMaxDev || key < 0 || key >= 64) return cudaErrorInvalidValue;
   std::lock_guard<std::mutex> lock(mu);
   if (granted[dev][key] >= smem) return cudaSuccess;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -428,7 +457,7 @@ cudaError_t ensure_smem1(const void* kern, int key, size_t smem) {
   return err;
 }
 
-template <int M, int UP>
+template <int M, int UP, int G>
 cudaError_t launch1_mu(const DeviceMatrix& m, const Gemv1Plan& plan, const void* x, void* y, int y_f32,
                        cudaStream_t stream) {
   Gemv1Args a;
@@ -439,8 +468,9 @@ cudaError_t launch1_mu(const DeviceMatrix& m, const Gemv1Plan& plan, const void*
   a.y = y;
   a.y_f32 = y_f32;
   const Smem1 L = smem1(plan, m.in, M);
-  auto kern = gemv1_kernel<M, UP>;
-  cudaError_t err = ensure_smem1(reinterpret_cast<const void*>(kern), (M - 2) * 3 + (UP == 4 ? 2 : UP - 1), L.total);
+  auto kern = gemv1_kernel<M, UP, G>;
+  const int key = ((M - 2) * 3 + (UP == 4 ? 2 : UP - 1)) * 3 + (G == 4 ? 2 : G - 1);
+  cudaError_t err = ensure_smem1(reinterpret_cast<const void*>(kern), key, L.total);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)plan.grid);
@@ -458,10 +488,14 @@ cudaError_t launch1_mu(const DeviceMatrix& m, const Gemv1Plan& plan, const void*
 template <int M>
 cudaError_t launch1_m(const DeviceMatrix& m, const Gemv1Plan& plan, const void* x, void* y, int y_f32,
                       cudaStream_t stream) {
-  switch (plan.up) {
-    case 1: return launch1_mu<M, 1>(m, plan, x, y, y_f32, stream);
-    case 2: return launch1_mu<M, 2>(m, plan, x, y, y_f32, stream);
-    case 4: return launch1_mu<M, 4>(m, plan, x, y, y_f32, stream);
+  switch (groups_per_chunk(plan.group_shift) * 8 + plan.up) {
+    case 8 + 1: return launch1_mu<M, 1, 1>(m, plan, x, y, y_f32, stream);
+    case 8 + 2: return launch1_mu<M, 2, 1>(m, plan, x, y, y_f32, stream);
+    case 8 + 4: return launch1_mu<M, 4, 1>(m, plan, x, y, y_f32, stream);
+    case 16 + 1: return launch1_mu<M, 1, 2>(m, plan, x, y, y_f32, stream);  // groups of 32
+    case 16 + 2: return launch1_mu<M, 2, 2>(m, plan, x, y, y_f32, stream);
+    case 32 + 1: return launch1_mu<M, 1, 4>(m, plan, x, y, y_f32, stream);  // groups of 16
+    case 32 + 2: return launch1_mu<M, 2, 4>(m, plan, x, y, y_f32, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -498,7 +532,8 @@ constexpr int kMinBlocks = 5;
 bool plan1_fit(const DeviceMatrix& m, int bits, const Gemv1Plan& q, uint32_t budget, bool strict, Gemv1Plan* out) {
   const int nblk4 = (q.rows_cap + 4 * q.RG - 1) / (4 * q.RG);
   const int nblk2 = (q.rows_cap + 2 * q.RG - 1) / (2 * q.RG);
-  const int up0 = (nblk4 >= kMinBlocks || nblk2 < kMinBlocks) ? 4 : 2;
+  // groups below 64 weights (several pairs per chunk): at most 2 rows per warp per block
+  const int up0 = q.group_shift < 6 ? 2 : (nblk4 >= kMinBlocks || nblk2 < kMinBlocks) ? 4 : 2;
   for (int stage = 1; stage >= (strict ? 1 : 0); --stage) {
     for (int up = up0; up >= (strict ? 2 : 1); up /= 2) {
       Gemv1Plan t = q;

@@ -91,23 +91,34 @@ __device__ __forceinline__ int dot4(const uint32_t (&X)[32], int i, int s, uint3
   return dp2a_hi(X[8 * i + 2 * s + 1], m, acc);
 }
 
-// sum over one 64-weight chunk of v_t X_t with v = u_M (v = 2 u_3 at M = 3).
-// B: the 4 base words; P[k]: the 2 chunk words of plane k+3. Exact in int32.
-template <int M>
-__device__ __forceinline__ int chunk_dot(const uint32_t (&X)[32], const uint32_t (&B)[4], const uint2* P) {
+// Sums of v_t X_t over the G groups of one 64-weight chunk, v = u_M (v = 2 u_3
+// at M = 3). G = 1, 2 or 4: a group is 64 / G weights, i.e. 4 / G consecutive
+// chunk words (word i holds weights 16 i .. 16 i + 15). B: the 4 base words;
+// P[k]: the 2 chunk words of plane k+3. Exact in int32.
+template <int M, int G>
+__device__ __forceinline__ void chunk_dot_g(const uint32_t (&X)[32], const uint32_t (&B)[4], const uint2* P,
+                                            int (&tot)[G]) {
+  static_assert(G == 1 || G == 2 || G == 4, "groups per chunk");
+  constexpr int WPG = 4 / G;  // chunk words per group
   if constexpr (M == 2) {
-    int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+    int a[G][4];
+#pragma unroll
+    for (int g = 0; g < G; ++g) a[g][0] = a[g][1] = a[g][2] = a[g][3] = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      a0 = dot4(X, i, 0, B[i] & 0x03030303u, a0);
-      a1 = dot4(X, i, 1, B[i] & 0x0C0C0C0Cu, a1);
-      a2 = dot4(X, i, 2, B[i] & 0x30303030u, a2);
-      a3 = dot4(X, i, 3, B[i] & 0xC0C0C0C0u, a3);
+      const int g = i / WPG;
+      a[g][0] = dot4(X, i, 0, B[i] & 0x03030303u, a[g][0]);
+      a[g][1] = dot4(X, i, 1, B[i] & 0x0C0C0C0Cu, a[g][1]);
+      a[g][2] = dot4(X, i, 2, B[i] & 0x30303030u, a[g][2]);
+      a[g][3] = dot4(X, i, 3, B[i] & 0xC0C0C0C0u, a[g][3]);
     }
-    // slot s carries q * 4^s, so every product in a_s is a multiple of 4^s
-    return a0 + (a1 >> 2) + (a2 >> 4) + (a3 >> 6);
+    // slot s carries q * 4^s, so every product in a[g][s] is a multiple of 4^s
+#pragma unroll
+    for (int g = 0; g < G; ++g) tot[g] = a[g][0] + (a[g][1] >> 2) + (a[g][2] >> 4) + (a[g][3] >> 6);
   } else {
-    int lo = 0, hi = 0;
+    int lo[G], hi[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) lo[g] = hi[g] = 0;
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
       const uint32_t p3 = w ? P[0].y : P[0].x;
@@ -115,21 +126,26 @@ __device__ __forceinline__ int chunk_dot(const uint32_t (&X)[32], const uint32_t
       if constexpr (M >= 4) p4 = w ? P[1].y : P[1].x;
       uint32_t E0, O0, E1, O1;
       nibble_words(B[2 * w], B[2 * w + 1], p3, p4, E0, O0, E1, O1);
-      const int i0 = 2 * w, i1 = 2 * w + 1;
-      lo = dot4(X, i0, 1, E0 & 0x0F0F0F0Fu, lo);
-      hi = dot4(X, i0, 3, E0 & 0xF0F0F0F0u, hi);
-      lo = dot4(X, i0, 0, O0 & 0x0F0F0F0Fu, lo);
-      hi = dot4(X, i0, 2, O0 & 0xF0F0F0F0u, hi);
-      lo = dot4(X, i1, 1, E1 & 0x0F0F0F0Fu, lo);
-      hi = dot4(X, i1, 3, E1 & 0xF0F0F0F0u, hi);
-      lo = dot4(X, i1, 0, O1 & 0x0F0F0F0Fu, lo);
-      hi = dot4(X, i1, 2, O1 & 0xF0F0F0F0u, hi);
+      const int i0 = 2 * w, i1 = 2 * w + 1, g0 = i0 / WPG, g1 = i1 / WPG;
+      lo[g0] = dot4(X, i0, 1, E0 & 0x0F0F0F0Fu, lo[g0]);
+      hi[g0] = dot4(X, i0, 3, E0 & 0xF0F0F0F0u, hi[g0]);
+      lo[g0] = dot4(X, i0, 0, O0 & 0x0F0F0F0Fu, lo[g0]);
+      hi[g0] = dot4(X, i0, 2, O0 & 0xF0F0F0F0u, hi[g0]);
+      lo[g1] = dot4(X, i1, 1, E1 & 0x0F0F0F0Fu, lo[g1]);
+      hi[g1] = dot4(X, i1, 3, E1 & 0xF0F0F0F0u, hi[g1]);
+      lo[g1] = dot4(X, i1, 0, O1 & 0x0F0F0F0Fu, lo[g1]);
+      hi[g1] = dot4(X, i1, 2, O1 & 0xF0F0F0F0u, hi[g1]);
     }
-    const int nib = lo + (hi >> 4);  // high-nibble products are multiples of 16
+    int nib[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) nib[g] = lo[g] + (hi[g] >> 4);  // high-nibble products are multiples of 16
     if constexpr (M <= 4) {
-      return nib;
+#pragma unroll
+      for (int g = 0; g < G; ++g) tot[g] = nib[g];
     } else {
-      int a5 = 0, a6 = 0;
+      int a5[G], a6[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) a5[g] = a6[g] = 0;
 #pragma unroll
       for (int w = 0; w < 2; ++w) {
         const uint32_t p5 = w ? P[2].y : P[2].x;
@@ -137,18 +153,41 @@ __device__ __forceinline__ int chunk_dot(const uint32_t (&X)[32], const uint32_t
         if constexpr (M >= 6) p6 = w ? P[3].y : P[3].x;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
+          const int g = (2 * w + h) / WPG;
 #pragma unroll
           for (int s = 0; s < 4; ++s) {
             const int sh = 4 * h + s;
-            a5 = dot4(X, 2 * w + h, s, (p5 >> sh) & 0x01010101u, a5);
-            if constexpr (M >= 6) a6 = dot4(X, 2 * w + h, s, (p6 >> sh) & 0x01010101u, a6);
+            a5[g] = dot4(X, 2 * w + h, s, (p5 >> sh) & 0x01010101u, a5[g]);
+            if constexpr (M >= 6) a6[g] = dot4(X, 2 * w + h, s, (p6 >> sh) & 0x01010101u, a6[g]);
           }
         }
       }
-      if constexpr (M == 5) return 2 * nib + a5;
-      else return 4 * nib + 2 * a5 + a6;
+#pragma unroll
+      for (int g = 0; g < G; ++g) tot[g] = M == 5 ? 2 * nib[g] + a5[g] : 4 * nib[g] + 2 * a5[g] + a6[g];
     }
   }
+}
+
+// The whole chunk as one group (groups of 64 weights or more).
+template <int M>
+__device__ __forceinline__ int chunk_dot(const uint32_t (&X)[32], const uint32_t (&B)[4], const uint2* P) {
+  int t[1];
+  chunk_dot_g<M, 1>(X, B, P, t);
+  return t[0];
+}
+
+// Groups per 64-weight chunk for a group size of 2^group_shift (>= 16).
+__host__ __device__ inline int groups_per_chunk(int group_shift) {
+  return group_shift >= 6 ? 1 : 1 << (6 - group_shift);
+}
+
+// G pair bytes of one row, starting at p (aligned to G bytes), as an integer
+// whose byte g is the pair of the chunk's group g.
+template <int G>
+__device__ __forceinline__ uint32_t load_pairs(const uint8_t* p) {
+  if constexpr (G == 1) return *p;
+  else if constexpr (G == 2) return *reinterpret_cast<const uint16_t*>(p);
+  else return *reinterpret_cast<const uint32_t*>(p);
 }
 
 }  // namespace kernels

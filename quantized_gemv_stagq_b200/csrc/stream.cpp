@@ -20,8 +20,8 @@ int check_shape(int64_t out, int64_t in, int64_t group, int n_planes) {
   if (out <= 0 || in <= 0) return fail(STAGQ_EINVAL, "shape must be positive");
   if (in % STAGQ_IN_MULTIPLE) return fail(STAGQ_EINVAL, "in must be a multiple of 128");
   if (in > STAGQ_MAX_IN) return fail(STAGQ_EINVAL, "in exceeds STAGQ_MAX_IN");
-  if (group < 64 || in % group || (group & (group - 1)) != 0)
-    return fail(STAGQ_EINVAL, "group must be a power of two >= 64 that divides in");
+  if (group < STAGQ_MIN_GROUP || in % group || (group & (group - 1)) != 0)
+    return fail(STAGQ_EINVAL, "group must be a power of two >= 16 that divides in");
   if (n_planes < 0 || n_planes > STAGQ_MAX_PLANES) return fail(STAGQ_EINVAL, "n_planes out of range");
   if (out > (int64_t)1 << 30) return fail(STAGQ_EINVAL, "out too large");
   return STAGQ_OK;

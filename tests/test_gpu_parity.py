@@ -49,6 +49,13 @@ SMALL = [
     (200, 4096, 128, 1, 0.02, "fast", 8),       # one plane
     (296, 4096, 128, 2, 0.6, "fast", 9),        # > 2048 record entries per stage (overflow path)
     (300, 32768, 128, 4, 0.005, "fast", 10),    # widest K: 16 K-warps, one-row stages at p6
+    # groups of 16 / 32 (the paper's encoder settings; its kernel runs at 32): 2 or 4 pairs per chunk
+    (512, 512, 32, 2, 0.005, "fast", 11),       # the tiny workload at g = 32 (0.25 bpw pair)
+    (96, 2048, 16, 4, 0.01, "fast", 12),        # g = 16, deep stream, p2..p6
+    (37, 640, 32, 3, 0.02, "fast", 13),         # g = 32, ragged K, fewer rows than SMs
+    (300, 5120, 16, 2, 0.005, "fast", 14),      # g = 16, K = 2.5 warp tiles
+    (64, 768, 16, 2, 1.0, "fast", 15),          # g = 16, everything held out
+    (48, 256, 16, 2, 0.02, "search", 16),       # g = 16, searched pairs
 ]
 
 
@@ -245,7 +252,7 @@ def test_full_size_phi4_olmo2_sampled_rows(name, shape):
     _sampled_rows_case(out, inp, 128, 2, 0.005, 2000 + out + inp, (2, 3, 4), (0,), batch4=False)
 
 
-@pytest.mark.parametrize("group,density", [(64, 0.0), (128, 0.001), (64, 0.01)])
+@pytest.mark.parametrize("group,density", [(64, 0.0), (128, 0.001), (64, 0.01), (32, 0.005), (16, 0.005)])
 def test_full_size_sweep_sampled_rows(group, density):
     """The precision/structure sweep: base + 4 planes read at 2..6 bits."""
     _sampled_rows_case(14336, 4096, group, 4, density, 3000 + group, (2, 3, 4, 5, 6), _kernels(), batch4=False)

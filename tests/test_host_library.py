@@ -56,7 +56,7 @@ def test_encoder_handles_constant_and_zero_groups():
         assert all(eq.values()), (mode, eq)
 
 
-@pytest.mark.parametrize("npl,g", [(0, 64), (1, 128), (2, 128), (3, 64), (4, 64)])
+@pytest.mark.parametrize("npl,g", [(0, 64), (1, 128), (2, 128), (3, 64), (4, 64), (2, 16), (3, 32)])
 def test_packed_levels_reread_on_host_equal_oracle_levels(npl, g):
     W = synth.weights(24, 640, seed=npl)
     F = O.encode(W, group=g, n_planes=npl, density=0.01, mode="fast")
@@ -102,6 +102,9 @@ def test_error_paths_return_status_codes():
     W = synth.weights(8, 192, seed=1)
     with pytest.raises(Q.StagqError) as e:   # in not a multiple of 128
         Q.stagq_pack(Q.stagq_encode(W, group=64, n_planes=2, density=0.0, mode="fast"))
+    assert e.value.status == 1
+    with pytest.raises(Q.StagqError) as e:   # group below 16
+        Q.stagq_pack(Q.stagq_encode(synth.weights(8, 256, seed=1), group=8, n_planes=2, density=0.0, mode="fast"))
     assert e.value.status == 1
     S = _stream()
     with pytest.raises(Q.StagqError) as e:
