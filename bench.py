@@ -21,7 +21,8 @@ JSON line each with per-GEMV (or per-token) times:
                          each alone and as one layer's chain (q k v o gate up
                          down, one CUDA graph);
   precision_sweep        14336x4096 and 4096x14336 with base + 4 planes, read at
-                         2..6 bits, group 64 and 128, side record 0 / 0.1 / 1 %;
+                         2..6 bits, group 16, 32, 64 and 128, side record
+                         0 / 0.1 / 1 %;
   llama31_8b_stack       32 layers x 7 linears (6.98e9 weights) resident on the
                          GPU, per-token GEMV time at batch 1 and 4, 2/3/4 bits
                          read from one stored stream.
@@ -375,11 +376,11 @@ def run_extra(args):
                "n_planes": N_PLANES, "side_record_density": DENSITY, "batch": 1}
     elif args.workload == "precision_sweep":
         shapes = [("gate", (14336, 4096)), ("down", (4096, 14336))]
-        for g in (64, 128):
+        for g in (16, 32, 64, 128):
             for d in (0.0, 0.001, 0.01):
                 per_gemv(shapes, (2, 3, 4, 5, 6), g, 4, d, tag=f"g{g} d{d} ")
         cfg = {"shapes_out_x_in": [list(v) for _, v in shapes], "bits": [2, 3, 4, 5, 6], "n_planes": 4,
-               "groups": [64, 128], "side_record_densities": [0.0, 0.001, 0.01], "batch": 1}
+               "groups": [16, 32, 64, 128], "side_record_densities": [0.0, 0.001, 0.01], "batch": 1}
     else:  # llama31_8b_stack
         layers, K = 32, max(1, args.stack_distinct)
         shapes = _layer_shapes()
