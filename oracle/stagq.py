@@ -10,8 +10,10 @@ binding) never does, and it shares no code with them.
 It covers three things:
 
 * the encoder of Sections 3.1-3.6 (+ Appendices B and E) for synthetic
-  weights: side record, clipping, initial pair, uniform codebooks, per-group
-  pair choice by Eq. (5)-(6), nearest-rounding base, sign planes (Eq. (7));
+  weights: side record (the workloads' global top-|w| density, or the
+  paper's pre-grid ratio guard plus the post-grid guard), clipping, initial
+  pair, uniform codebooks, per-group pair choice by Eq. (5)-(6),
+  nearest-rounding base, sign planes (Eq. (7));
 * the decoder: composite integer Eq. (8), affine map Eq. (10) (with the
   additive form Eq. (9) kept as a cross-check), complete reconstruction
   Eq. (4);
@@ -60,7 +62,8 @@ class Fields:
     cb_lo_over_s: np.ndarray    # float16 [16]
     row_ptr: np.ndarray         # int64 [out + 1]  (side record, CSR)
     col: np.ndarray             # int64 [nnz], sorted inside each row
-    val: np.ndarray             # float16 [nnz], the recorded value P
+    val: np.ndarray             # float16 [nnz]: the recorded value (pre-grid) or residual (post-grid)
+    post: np.ndarray = None     # bool [nnz]: entry held out by the post-grid guard (None: none)
 
     @property
     def depth(self) -> int:
@@ -70,6 +73,10 @@ class Fields:
     @property
     def nnz(self) -> int:
         return int(self.col.shape[0])
+
+    @property
+    def post_flags(self) -> np.ndarray:
+        return np.zeros(self.nnz, dtype=bool) if self.post is None else np.asarray(self.post, dtype=bool)
 
 
 # --------------------------------------------------------------------------
@@ -196,6 +203,46 @@ def select_side_record(W: np.ndarray, density: float) -> np.ndarray:
     mask[above] = True
     mask[tied[: k - above.size]] = True
     return mask.reshape(out, inp)
+
+
+def select_ratio_guard(W: np.ndarray, group: int, T: float) -> np.ndarray:
+    """Section 3.5, pre-grid guard under the ratio criterion: in each group,
+    the largest-|w| entry is held out when its magnitude exceeds T times the
+    second largest magnitude of the group (T = 4 on Llama-3.1-8B, Table 6).
+
+    Reading: "largest" is the first index of the maximum |w|; the second
+    largest is the maximum over the group's other entries, so two equal
+    largest magnitudes hold nothing out. Returns a bool mask [out, inp].
+    """
+    out, inp = W.shape
+    ng = inp // group
+    A = np.abs(W.astype(np.float64)).reshape(out, ng, group)
+    j1 = np.argmax(A, axis=2)                                    # first maximum
+    a1 = np.take_along_axis(A, j1[:, :, None], axis=2)[:, :, 0]
+    others = A.copy()
+    np.put_along_axis(others, j1[:, :, None], -np.inf, axis=2)
+    a2 = others.max(axis=2) if group > 1 else np.zeros_like(a1)
+    take = a1 > T * a2
+    mask = np.zeros((out, ng, group), dtype=bool)
+    np.put_along_axis(mask, j1[:, :, None], take[:, :, None], axis=2)
+    return mask.reshape(out, inp)
+
+
+def select_post_guard(W: np.ndarray, W2: np.ndarray, held: np.ndarray) -> np.ndarray:
+    """Appendix E, post-grid guard of a ratio-criterion matrix: after the grid
+    is fixed, the one position per output row with the largest
+    activation-weighted two-bit error E_c (W - W_hat^(2))^2.
+
+    Reading: E_c = 1 as in Eq. (5) (x ~ N(0,1), no calibration set); ties go
+    to the smallest column; positions already held out by the pre-grid guard
+    are not candidates, and a row with none takes nothing. Returns a bool mask.
+    """
+    err = (W.astype(np.float64) - W2) ** 2
+    err = np.where(held, -np.inf, err)
+    mask = np.zeros(W.shape, dtype=bool)
+    rows = np.flatnonzero(~np.all(held, axis=1))
+    mask[rows, np.argmax(err[rows], axis=1)] = True
+    return mask
 
 
 def clip_held_out(W: np.ndarray, mask: np.ndarray, group: int):
@@ -351,11 +398,15 @@ def choose_pairs(Vc: np.ndarray, group: int, N: int, lo_tab, s_tab, empty,
 
 def encode(W: np.ndarray, group: int = 128, n_planes: int = 2,
            density: float = 0.005, mode: str = "search", rows=None,
-           row_block: int = 512) -> Fields:
+           row_block: int = 512, guard: str = "density", ratio_T: float = 4.0,
+           post_guard: bool = True) -> Fields:
     """Figure 3's encoder for synthetic weights (no AWQ scale: with x ~ N(0,1)
-    every channel scale is equal; no post-grid guard):
+    every channel scale is equal):
 
-    1. side record: top-|w| entries (``select_side_record``), P = fp16 value;
+    1. side record: with ``guard="density"`` the top-|w| entries
+       (``select_side_record``, the workloads' reading); with ``guard="ratio"``
+       the pre-grid ratio guard of Section 3.5 (``select_ratio_guard``, T =
+       ``ratio_T``); P = fp16 value;
     2. clip held-out entries inward for the fit (``clip_held_out``);
     3. initial pairs (Appendix B), 4. uniform codebooks (Appendix E),
     5. pair per group (Eq. (5) search, or the labelled fast rule),
@@ -363,6 +414,13 @@ def encode(W: np.ndarray, group: int = 128, n_planes: int = 2,
        store zero digits (Reading: the planes skip them, Section 3.6, and the
        paper gives no stored value -- zeros make the main stream decode to
        lo_M there, which Eq. (4) then masks).
+
+    8. with ``guard="ratio"`` and ``post_guard``, the post-grid guard
+       (``select_post_guard``): per row the position with the largest two-bit
+       error. Its base digit stays; its planes are zero; it records the fp16
+       residual r = fp16(w - W_hat^(2)), and Eq. (4) takes P = W_hat^(2) + r
+       there (Section 3, Eq. (4): the two-bit reconstruction plus the
+       residual, the same for every M).
 
     Steps 1-4 look at the whole matrix (global record, per-matrix codebooks).
     With ``rows`` given, steps 5-7 run only for those rows and the returned
@@ -378,7 +436,13 @@ def encode(W: np.ndarray, group: int = 128, n_planes: int = 2,
     N = 2 + n_planes
     ng = inp // group
 
-    mask = select_side_record(W, density)
+    if guard == "density":
+        mask = select_side_record(W, density)
+    elif guard == "ratio":
+        mask = select_ratio_guard(W, group, ratio_T)
+    else:
+        raise ValueError("guard must be 'density' or 'ratio'")
+    with_post = guard == "ratio" and post_guard
     Vc, empty = clip_held_out(W, mask, group)
     lo0, s0, flat = initial_pairs(Vc, group)
     cb_log2s, cb_lo_over_s = fit_codebooks(lo0, s0, empty | flat)
@@ -389,6 +453,8 @@ def encode(W: np.ndarray, group: int = 128, n_planes: int = 2,
     pair_idx = np.empty((n, ng), dtype=np.uint8)
     q = np.empty((n, inp), dtype=np.uint8)
     planes = np.empty((n_planes, n, inp), dtype=np.uint8)
+    post = np.zeros((n, inp), dtype=bool)
+    resid = np.zeros((n, inp), dtype=np.float16)
     for b0 in range(0, n, row_block):
         rb = rows[b0:b0 + row_block]
         sl = slice(b0, b0 + rb.size)
@@ -397,22 +463,31 @@ def encode(W: np.ndarray, group: int = 128, n_planes: int = 2,
                                     cb_lo_over_s=cb_lo_over_s, flat=flat[rb])
         lo_w = np.repeat(lo_tab[pair_idx[sl].astype(np.int64)], group, axis=1)
         s_w = np.repeat(s_tab[pair_idx[sl].astype(np.int64)], group, axis=1)
-        qb, bits, _ = encode_digits(W[rb].astype(np.float64), lo_w, s_w, N)
+        Wb = W[rb].astype(np.float64)
+        qb, bits, _ = encode_digits(Wb, lo_w, s_w, N)
         m = mask[rb]
-        q[sl] = np.where(m, 0, qb)
+        pb = np.zeros_like(m)
+        if with_post:
+            W2 = lo_w + s_w * qb                          # Eq. (10) at M = 2: lo + s q
+            pb = select_post_guard(W[rb], W2, m)
+            resid[sl] = np.where(pb, Wb - W2, 0.0).astype(np.float16)
+        post[sl] = pb
+        q[sl] = np.where(m, 0, qb)                        # post-grid positions keep their base digit
         for k in range(n_planes):
-            planes[k, sl] = np.where(m, 0, bits[k])
+            planes[k, sl] = np.where(m | pb, 0, bits[k])
 
-    sub = mask[rows]
+    sub = mask[rows] | post
     r_idx, cols = np.nonzero(sub)                         # row-major order
     row_ptr = np.zeros(n + 1, dtype=np.int64)
     np.add.at(row_ptr, r_idx + 1, 1)
     row_ptr = np.cumsum(row_ptr)
-    val = W[rows[r_idx], cols].astype(np.float16)
+    is_post = post[r_idx, cols]
+    val = np.where(is_post, resid[r_idx, cols], W[rows[r_idx], cols]).astype(np.float16)
     return Fields(out=n, inp=inp, group=group, n_planes=n_planes, q=q,
                   planes=planes, pair_idx=pair_idx,
                   cb_log2s=cb_log2s, cb_lo_over_s=cb_lo_over_s,
-                  row_ptr=row_ptr, col=cols.astype(np.int64), val=val)
+                  row_ptr=row_ptr, col=cols.astype(np.int64), val=val,
+                  post=is_post if with_post else None)
 
 
 # --------------------------------------------------------------------------
@@ -449,18 +524,26 @@ def group_pairs(F: Fields, rows=None):
 
 
 def decode(F: Fields, M: int, rows=None) -> np.ndarray:
-    """Eq. (4): W_hat^(M) = (1 - m) * (lo_M + s_M u_M) + P, fp64 [rows, inp]."""
+    """Eq. (4): W_hat^(M) = (1 - m) * (lo_M + s_M u_M) + P, fp64 [rows, inp].
+    P is the recorded value at a pre-grid entry and the two-bit
+    reconstruction lo + s q plus the recorded residual at a post-grid entry
+    (Section 3, below Eq. (4))."""
     u = decode_levels(F, M, rows)
     lo_g, s_g = group_pairs(F, rows)
     lo_w = np.repeat(lo_g, F.group, axis=1)
     s_w = np.repeat(s_g, F.group, axis=1)
     main = reconstruct_affine(lo_w, s_w, u, M)
     rows_ = np.arange(F.out) if rows is None else np.asarray(rows)
+    q = F.q if rows is None else F.q[rows_]
+    w2 = lo_w + s_w * q.astype(np.float64)               # two-bit reconstruction, Eq. (10) at M = 2
     m = held_out_mask(F, rows_)
+    post = F.post_flags
     P = np.zeros_like(main)
     for i, r in enumerate(rows_):
         sl = slice(F.row_ptr[r], F.row_ptr[r + 1])
-        P[i, F.col[sl]] = F.val[sl].astype(np.float64)
+        c = F.col[sl]
+        v = F.val[sl].astype(np.float64)
+        P[i, c] = np.where(post[sl], w2[i, c] + v, v)
     return np.where(m, 0.0, main) + P
 
 

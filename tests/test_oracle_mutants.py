@@ -1,6 +1,8 @@
 """Planted mistakes in the oracle (CPU only): each plausible slip -- a dropped
 term, a wrong sign, a wrong exponent, swapped nibbles -- must make at least
 one pin in test_oracle_pins fail."""
+import dataclasses
+
 import numpy as np
 import pytest
 
@@ -48,6 +50,32 @@ def _base_digit_truncating(w, lo, s):
     return np.clip(np.floor((np.asarray(w, dtype=np.float64) - lo) / s), 0, 3).astype(np.int64)
 
 
+_select_post_guard = O.select_post_guard
+_decode = O.decode
+
+
+def _decode_post_as_recorded_value(F, M, rows=None):
+    """Takes a post-grid residual as if it were a recorded value (drops the
+    two-bit reconstruction from P)."""
+    return _decode(dataclasses.replace(F, post=None), M, rows)
+
+
+def _post_guard_wrong_error(W, W2, held):
+    """Scores |w| instead of the two-bit error (the reconstruction dropped)."""
+    return _select_post_guard(W, np.zeros_like(W2), held)
+
+
+def _ratio_guard_second_excluded_wrongly(W, group, T):
+    out, inp = W.shape
+    A = np.abs(W.astype(np.float64)).reshape(out, inp // group, group)
+    j1 = np.argmax(A, axis=2)
+    a1 = np.take_along_axis(A, j1[:, :, None], axis=2)[:, :, 0]
+    a2 = np.sort(A, axis=2)[:, :, -1]            # compares with the largest itself, not the second
+    mask = np.zeros(A.shape, dtype=bool)
+    np.put_along_axis(mask, j1[:, :, None], (a1 > T * a2)[:, :, None], axis=2)
+    return mask.reshape(out, inp)
+
+
 @pytest.mark.parametrize("name,mutant,pins", [
     ("grid_at", _grid_wrong_sign, ["test_eq9_equals_eq10_all_digit_patterns", "test_figure1_every_prefix_is_a_grid_point"]),
     ("grid_at", _grid_wrong_spacing, ["test_every_precision_is_a_uniform_grid", "test_midpoint_split_is_the_mmse_split"]),
@@ -55,6 +83,10 @@ def _base_digit_truncating(w, lo, s):
     ("composite_level", _composite_dropped_plane, ["test_eq9_equals_eq10_all_digit_patterns"]),
     ("pair_table", _pair_table_swapped, ["test_gemv_against_scalar_brute_force"]),
     ("base_digit", _base_digit_truncating, ["test_sign_planes_equal_nearest_level_rounding"]),
+    ("select_ratio_guard", _ratio_guard_second_excluded_wrongly, ["test_ratio_guard_matches_brute_force"]),
+    ("select_post_guard", _post_guard_wrong_error, ["test_post_guard_is_the_row_argmax_of_two_bit_error"]),
+    ("decode", _decode_post_as_recorded_value, ["test_post_entries_reconstruct_w_at_every_precision",
+                                                "test_gemv_with_guards_against_scalar_brute_force"]),
 ])
 def test_planted_mistake_is_caught(monkeypatch, name, mutant, pins):
     monkeypatch.setattr(O, name, mutant)

@@ -320,3 +320,130 @@ def test_codebooks_are_uniform_over_initial_pair_range():
     exact = ls.min() + np.arange(16) * (ls.max() - ls.min()) / 15
     ulp = float(np.spacing(np.float16(np.abs(ls).max())))
     assert np.all(np.abs(F.cb_log2s.astype(np.float64) - exact) <= ulp / 2)
+
+
+# ------------------------------------------------ guards (Section 3.5, Appendix E)
+
+def _brute_ratio_guard(W, group, T):
+    out, inp = W.shape
+    m = np.zeros((out, inp), dtype=bool)
+    for r in range(out):
+        for g0 in range(0, inp, group):
+            a = [abs(float(W[r, g0 + j])) for j in range(group)]
+            j1 = 0
+            for j in range(1, group):
+                if a[j] > a[j1]:
+                    j1 = j
+            second = max([a[j] for j in range(group) if j != j1], default=0.0)
+            if a[j1] > T * second:
+                m[r, g0 + j1] = True
+    return m
+
+
+def test_ratio_guard_matches_brute_force():
+    rng = np.random.default_rng(4)
+    W = (rng.standard_normal((6, 64)) * 0.02).astype(np.float16)
+    W[0, 3] = 0.5                 # dominant: > 4x the rest of its group
+    W[1, 17:19] = 0.4             # two equal largest: nothing held out
+    W[2, 32:48] = 0.0
+    W[2, 40] = 0.01               # the only nonzero of its group
+    W[3, 48:64] = 0.0             # all-zero group: nothing held out
+    for T in (4.0, 2.0, 8.0):
+        m = O.select_ratio_guard(W, 16, T)
+        assert np.array_equal(m, _brute_ratio_guard(W, 16, T)), T
+    m = O.select_ratio_guard(W, 16, 4.0)
+    assert m[0, 3] and not m[1, 16:32].any() and m[2, 40] and not m[3, 48:64].any()
+    assert (m.reshape(6, 4, 16).sum(axis=2) <= 1).all()   # at most one entry per group
+
+
+def test_post_guard_is_the_row_argmax_of_two_bit_error():
+    """Each row's post-grid entry is the non-held position with the largest
+    (w - (lo + s q))^2 (first on ties), recomputed here with scalar loops from
+    the stored digits and pairs; its base digit is the grid's, its planes 0."""
+    W = synth.weights(10, 256, seed=31)
+    F = O.encode(W, group=64, n_planes=2, mode="fast", guard="ratio", ratio_T=4.0)
+    post = F.post_flags
+    cbs = [float(v) for v in F.cb_log2s]
+    cbr = [float(v) for v in F.cb_lo_over_s]
+    for r in range(F.out):
+        sl = slice(F.row_ptr[r], F.row_ptr[r + 1])
+        pre_cols = set(int(c) for c, p in zip(F.col[sl], post[sl]) if not p)
+        post_cols = [int(c) for c, p in zip(F.col[sl], post[sl]) if p]
+        best, best_c = -1.0, None
+        for c in range(F.inp):
+            if c in pre_cols:
+                continue
+            p = int(F.pair_idx[r, c // F.group])
+            s = 2.0 ** cbs[p >> 4]
+            lo = cbr[p & 15] * s
+            w = float(W[r, c])
+            q = min(3, max(0, math.floor((w - lo) / s + 0.5)))   # nearest rounding under the fixed grid
+            e = (w - (lo + s * q)) ** 2
+            if e > best:
+                best, best_c = e, c
+        assert post_cols == [best_c], r
+        assert F.planes[:, r, best_c].sum() == 0
+        p = int(F.pair_idx[r, best_c // F.group])
+        s = 2.0 ** cbs[p >> 4]
+        lo = cbr[p & 15] * s
+        assert int(F.q[r, best_c]) == min(3, max(0, math.floor((float(W[r, best_c]) - lo) / s + 0.5)))
+
+
+def test_post_entries_reconstruct_w_at_every_precision():
+    """At a post-grid entry P = two-bit reconstruction + fp16 residual: the
+    same at every M, and within the residual's fp16 rounding of w; pre-grid
+    entries return the recorded fp16 value exactly."""
+    W = synth.weights(16, 512, seed=33)
+    F = O.encode(W, group=32, n_planes=4, mode="fast", guard="ratio", ratio_T=4.0)
+    post = F.post_flags
+    assert post.sum() == 16 and (~post).sum() > 0
+    r = np.repeat(np.arange(F.out), np.diff(F.row_ptr))
+    w = W[r, F.col].astype(np.float64)
+    got = [O.decode(F, M)[r, F.col] for M in range(2, 7)]
+    for g in got[1:]:
+        assert np.array_equal(g, got[0])
+    res = np.abs(F.val[post].astype(np.float64))
+    assert np.all(np.abs(got[0][post] - w[post]) <= res * 2.0 ** -11 + 1e-12)
+    assert np.array_equal(got[0][~post], w[~post])
+
+
+def test_ratio_guard_without_hold_outs_is_the_main_stream():
+    """T = infinity and no post-grid guard hold nothing out: the stream equals
+    the density-0 encoding field for field."""
+    W = synth.weights(8, 256, seed=35)
+    A = O.encode(W, group=64, n_planes=2, density=0.0, mode="fast")
+    B = O.encode(W, group=64, n_planes=2, mode="fast", guard="ratio", ratio_T=math.inf, post_guard=False)
+    assert B.nnz == 0
+    for k in ("q", "planes", "pair_idx", "cb_log2s", "cb_lo_over_s"):
+        assert np.array_equal(getattr(A, k), getattr(B, k)), k
+
+
+def test_gemv_with_guards_against_scalar_brute_force():
+    W = synth.weights(6, 256, seed=37)
+    F = O.encode(W, group=64, n_planes=2, mode="search", guard="ratio", ratio_T=4.0)
+    x = synth.activations(1, 256, seed=38)[0]
+    cbs = [float(v) for v in F.cb_log2s]
+    cbr = [float(v) for v in F.cb_lo_over_s]
+    for M in (2, 3, 4):
+        y = O.gemv(F, M, x[None])[0]
+        ref = []
+        for r in range(F.out):
+            acc = 0.0
+            ent = {int(F.col[e]): (float(F.val[e]), bool(F.post_flags[e]))
+                   for e in range(F.row_ptr[r], F.row_ptr[r + 1])}
+            for c in range(F.inp):
+                p = int(F.pair_idx[r, c // F.group])
+                s = 2.0 ** cbs[p >> 4]
+                lo = cbr[p & 15] * s
+                if c in ent and not ent[c][1]:
+                    w = ent[c][0]
+                elif c in ent:
+                    w = lo + s * int(F.q[r, c]) + ent[c][0]
+                else:
+                    u = int(F.q[r, c]) << (M - 2)
+                    for k in range(3, M + 1):
+                        u += int(F.planes[k - 3, r, c]) << (M - k)
+                    w = lo - s * (2 ** (M - 2) - 1) / 2 ** (M - 1) + s / 2 ** (M - 2) * u
+                acc += w * float(x[c])
+            ref.append(acc)
+        assert np.allclose(y, ref, rtol=1e-12, atol=1e-14), M
