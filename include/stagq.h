@@ -75,10 +75,15 @@ typedef struct stagq_matrix* stagq_handle;   /* opaque; owned by the library */
  *   planes    [n_planes*out*in]   b_k in {0,1}; plane k (k = 3..2+n_planes) at offset (k-3)*out*in
  *   pair_idx  [out*(in/group)]    8-bit pair: high nibble = log2(s) codebook index, low = lo/s index
  *   row_ptr   [out+1]             side record (CSR): entries of row r are [row_ptr[r], row_ptr[r+1])
- *   col       [nnz]               column of each held-out weight, increasing inside a row
- *   val       [nnz]               recorded fp16 value P (pre-grid guard, Eq. 4)
- * Held-out positions carry zero digits (q = 0, all b_k = 0).
+ *   col       [nnz]               column of each held-out weight, increasing inside a row;
+ *                                 bit 15 (STAGQ_SIDE_POST) marks a post-grid entry
+ *   val       [nnz]               fp16: the recorded value (pre-grid entry, P = val) or the
+ *                                 residual r against the two-bit reconstruction (post-grid
+ *                                 entry, P = lo + s q + r; Section 3 below Eq. 4)
+ * Pre-grid positions carry zero digits (q = 0, all b_k = 0); post-grid
+ * positions keep their base digit q and carry zero planes.
  */
+#define STAGQ_SIDE_POST 0x8000u
 typedef struct {
     int32_t out, in, group, n_planes;
     int64_t nnz;
@@ -125,6 +130,28 @@ typedef struct {
 
 /* Number of side-record entries for a density: round(density*out*in), half up. */
 int64_t stagq_side_record_count(int32_t out, int32_t in, double density);
+
+/*
+ * Side-record capacity of stagq_encode_guarded: one pre-grid entry per group
+ * and one post-grid entry per row at most, out*(in/group) + out.
+ */
+int64_t stagq_guard_capacity(int32_t out, int32_t in, int32_t group);
+
+/*
+ * The encoder with the paper's guards in place of the density record:
+ * pre-grid ratio criterion (Section 3.5: a group's largest-|w| entry is held
+ * out when it exceeds ratio_T times the second largest; T = 4 on
+ * Llama-3.1-8B, Table 6) and, if post_guard != 0, the post-grid guard of a
+ * ratio-criterion matrix (Appendix E: per row, the position with the largest
+ * two-bit error (w - (lo + s q))^2 under the fitted grid, recorded as an
+ * fp16 residual with STAGQ_SIDE_POST in its column). The rest is
+ * stagq_encode's steps 2-7.
+ *   f->nnz   in: capacity of f->col / f->val, at least stagq_guard_capacity();
+ *            out: the entries written.
+ * Errors: as stagq_encode; STAGQ_EINVAL if ratio_T < 1 or the capacity is short.
+ */
+int stagq_encode_guarded(const uint16_t* w, double ratio_T, int32_t post_guard, int32_t pair_mode,
+                         int32_t n_threads, stagq_fields* f);
 
 /*
  * Encoder of Sections 3.1-3.6 / Appendices B, E for a synthetic fp16 matrix

@@ -23,6 +23,7 @@ STAGQ_PAIR_FAST = 1
 STAGQ_Y_F32 = 1
 STAGQ_KERNEL_GENERAL = 2
 STAGQ_KERNEL_SINGLE = 4
+STAGQ_SIDE_POST = 0x8000
 STAGQ_MAX_PLANES = 4
 STAGQ_MAX_BATCH = 4
 
@@ -51,6 +52,8 @@ class _Info(ctypes.Structure):
 _SIGNATURES = {
     "stagq_side_record_count": (_i64, [_i32, _i32, _dbl]),
     "stagq_encode": (ctypes.c_int, [_c_p, _dbl, _i32, _i32, ctypes.POINTER(_Fields)]),
+    "stagq_guard_capacity": (_i64, [_i32, _i32, _i32]),
+    "stagq_encode_guarded": (ctypes.c_int, [_c_p, _dbl, _i32, _i32, _i32, ctypes.POINTER(_Fields)]),
     "stagq_stream_plane_bytes": (_i64, [_i32, _i32, _i32]),
     "stagq_pack": (ctypes.c_int, [ctypes.POINTER(_Fields), _c_p]),
     "stagq_unpack_levels_host": (ctypes.c_int, [ctypes.POINTER(_HostStream), ctypes.c_int, _c_p]),
@@ -175,12 +178,25 @@ def stagq_stream_plane_bytes(out: int, inp: int, n_planes: int) -> int:
     return int(lib().stagq_stream_plane_bytes(out, inp, n_planes))
 
 
+def stagq_guard_capacity(out: int, inp: int, group: int) -> int:
+    return int(lib().stagq_guard_capacity(out, inp, group))
+
+
 def stagq_encode(w: np.ndarray, group: int = 128, n_planes: int = 2, density: float = 0.005,
-                 mode: str = "search", n_threads: int = 0) -> Fields:
-    """Encode an fp16 [out, inp] matrix (library encoder, host)."""
+                 mode: str = "search", n_threads: int = 0, guard: str = "density", ratio_T: float = 4.0,
+                 post_guard: bool = True) -> Fields:
+    """Encode an fp16 [out, inp] matrix (library encoder, host). guard
+    "density": global top-|w| record of `density` (stagq_encode); "ratio": the
+    pre-grid ratio guard with `ratio_T` and, if post_guard, the post-grid guard
+    (stagq_encode_guarded; post-grid columns carry STAGQ_SIDE_POST)."""
     w = np.ascontiguousarray(w, dtype=np.float16)
     out, inp = w.shape
-    nnz = stagq_side_record_count(out, inp, density)
+    if guard == "density":
+        nnz = stagq_side_record_count(out, inp, density)
+    elif guard == "ratio":
+        nnz = stagq_guard_capacity(out, inp, group)
+    else:
+        raise ValueError("guard must be 'density' or 'ratio'")
     F = Fields(out, inp, group, n_planes,
                q=np.empty((out, inp), np.uint8),
                planes=np.empty((n_planes, out, inp), np.uint8),
@@ -190,7 +206,13 @@ def stagq_encode(w: np.ndarray, group: int = 128, n_planes: int = 2, density: fl
                val=np.empty(nnz, np.uint16))
     cf = F._c()
     m = {"search": STAGQ_PAIR_SEARCH, "fast": STAGQ_PAIR_FAST}[mode]
-    _check(lib().stagq_encode(w.ctypes.data, density, m, n_threads, ctypes.byref(cf)), "stagq_encode")
+    if guard == "density":
+        _check(lib().stagq_encode(w.ctypes.data, density, m, n_threads, ctypes.byref(cf)), "stagq_encode")
+    else:
+        _check(lib().stagq_encode_guarded(w.ctypes.data, ratio_T, int(post_guard), m, n_threads, ctypes.byref(cf)),
+               "stagq_encode_guarded")
+        F.col = F.col[:cf.nnz].copy()
+        F.val = F.val[:cf.nnz].copy()
     F.cb_log2s = np.array(cf.codebook_log2s[:], dtype=np.uint16)
     F.cb_lo_over_s = np.array(cf.codebook_lo_over_s[:], dtype=np.uint16)
     return F

@@ -50,9 +50,13 @@ struct DeviceGuard {
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Per-precision (lo_M, s_M c_M) for the 256 pairs, Eq. (10) in fp64, stored fp32.
-void build_tables(const stagq_host_stream* s, std::vector<float2>& t) {
+// and, per precision, lo - lo_M of every pair: at a post-grid entry the main
+// stream decodes lo_M + s q (zero planes), the reconstruction is lo + s q + r,
+// so the correction is r + (lo - lo_M).
+void build_tables(const stagq_host_stream* s, std::vector<float2>& t, std::vector<float>& dlo) {
   const int N = 2 + s->n_planes;
   t.assign((size_t)(N - 1) * 256, make_float2(0.f, 0.f));
+  dlo.assign((size_t)(N - 1) * 256, 0.f);
   for (int M = 2; M <= N; ++M) {
     for (int p = 0; p < 256; ++p) {
       const double sp = std::exp2(half_to_double(s->codebook_log2s[p >> 4]));
@@ -60,6 +64,7 @@ void build_tables(const stagq_host_stream* s, std::vector<float2>& t) {
       const double sM = sp / std::ldexp(1.0, M - 2);
       const double loM = lo - sp * (std::ldexp(1.0, M - 2) - 1.0) / std::ldexp(1.0, M - 1);
       t[(size_t)(M - 2) * 256 + p] = make_float2((float)loM, (float)(sM * composite_factor(M)));
+      dlo[(size_t)(M - 2) * 256 + p] = (float)(lo - loM);
     }
   }
 }
@@ -74,6 +79,10 @@ int check_handle_bits(stagq_handle h, int bits) {
 }  // namespace stagq
 
 using namespace stagq;
+
+namespace {
+constexpr uint16_t kColMask = 0x7FFF;  // side-record column without the post-grid flag
+}
 
 extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* out) {
   if (!out) return fail(STAGQ_EINVAL, "stagq_load: null output handle");
@@ -98,6 +107,9 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   const size_t pair_row = (size_t)(in / s->group), pair_stride = align_up(pair_row, 16);
   const size_t pair_bytes = (size_t)out_ * pair_stride;
   const size_t tab_bytes = (size_t)(np + 1) * 256 * sizeof(float2);
+  const size_t dlo_bytes = (size_t)(np + 1) * 256 * sizeof(float);
+  int has_post = 0;
+  for (int64_t e = 0; e < s->nnz; ++e) has_post |= (s->col[e] & STAGQ_SIDE_POST) != 0;
   // Side record cut per CTA of the GEMV grid (see DeviceMatrix::side).
   const int grid = gemv_grid(s->out, s->in, prop.multiProcessorCount);
   const int KW = k_slices(s->in), RG = row_groups(KW);
@@ -134,6 +146,7 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   const size_t o_side = off; off = align_up(off + side_bytes, 256);
   const size_t o_side1 = off; off = align_up(off + side1_bytes, 256);
   const size_t o_tab = off; off = align_up(off + tab_bytes, 256);
+  const size_t o_dlo = off; off = align_up(off + dlo_bytes, 256);
   const size_t o_status = off; off = align_up(off + 4, 256);
   const size_t total = off;
 
@@ -150,7 +163,8 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   uint8_t* d = static_cast<uint8_t*>(h->d_mem);
 
   std::vector<float2> tabs;
-  build_tables(s, tabs);
+  std::vector<float> dlo;
+  build_tables(s, tabs, dlo);
   std::vector<uint8_t> side(side_bytes, 0);
   {
     for (int b = 0; b < grid; ++b) {
@@ -168,8 +182,9 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
             o[m] = pos;
             int64_t e = s->row_ptr[r];
             const int64_t e1 = s->row_ptr[r + 1];
-            while (e < e1 && s->col[e] < (int64_t)kw * kSliceWeights) ++e;  // columns increase within a row
-            for (; e < e1 && s->col[e] < (int64_t)(kw + 1) * kSliceWeights; ++e)
+            // columns increase within a row; the entry keeps the post-grid flag (bit 15)
+            while (e < e1 && (s->col[e] & kColMask) < (int64_t)kw * kSliceWeights) ++e;
+            for (; e < e1 && (s->col[e] & kColMask) < (int64_t)(kw + 1) * kSliceWeights; ++e)
               ent[pos++] = (uint32_t)s->col[e] | ((uint32_t)s->val[e] << 16);
           }
           o[nm] = pos;
@@ -187,7 +202,8 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
     for (int64_t r = 0; r < n; ++r) {
       offs[r] = pos;
       for (int64_t e = s->row_ptr[ra + r]; e < s->row_ptr[ra + r + 1]; ++e)
-        ent[pos++] = (uint32_t)xq_slot_of_column(s->col[e]) | ((uint32_t)s->val[e] << 16);
+        ent[pos++] = (uint32_t)xq_slot_of_column(s->col[e] & kColMask) | (uint32_t)(s->col[e] & STAGQ_SIDE_POST) |
+                     ((uint32_t)s->val[e] << 16);
     }
     offs[n] = pos;
   }
@@ -201,6 +217,7 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   copies.push_back({o_side, side.data(), side_bytes});
   copies.push_back({o_side1, side1.data(), side1_bytes});
   copies.push_back({o_tab, tabs.data(), tab_bytes});
+  copies.push_back({o_dlo, dlo.data(), dlo_bytes});
   for (const Copy& c : copies) {
     e = cudaMemcpy(d + c.off, c.src, c.n, cudaMemcpyHostToDevice);
     if (e != cudaSuccess) {
@@ -236,6 +253,8 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   m.side1_grid = grid1;
   m.side1_max = (int32_t)max_cta1;
   m.tables = reinterpret_cast<const float2*>(d + o_tab);
+  m.dlo = reinterpret_cast<const float*>(d + o_dlo);
+  m.has_post = has_post;
   m.status = reinterpret_cast<uint32_t*>(d + o_status);
   m.num_sms = prop.multiProcessorCount;
   m.smem_pair_budget = smem_sm / 2 - smem_reserved;

@@ -43,7 +43,8 @@ struct DeviceMatrix {
   // classes (local row mod RG); its entries are ordered by (class, K slice,
   // row, column), and int32 offsets [RG][KW][class_rows + 1] give where each
   // row of a class starts within its (class, K slice) run, plus the run's end.
-  // The entries (column | fp16 value << 16) start at side_ent_off.
+  // The entries (column | fp16 value << 16; bit 15 marks a post-grid entry,
+  // whose value is the residual r) start at side_ent_off.
   const uint8_t* side;
   int32_t side_stride, side_ent_off, side_grid;
   // The same side record cut for the single-vector kernel (gemv1.cu): per CTA
@@ -54,6 +55,8 @@ struct DeviceMatrix {
   const uint8_t* side1;
   int32_t side1_stride, side1_ent_off, side1_grid, side1_max;
   const float2* tables;       // [n_planes+1][256]: (lo_M, s_M * c_M) for M = 2..2+n_planes
+  const float* dlo;           // [n_planes+1][256]: lo - lo_M, the correction of a post-grid entry beside r
+  int32_t has_post;           // the side record holds post-grid entries (bit 15 of the column / slot)
   uint32_t* status;           // nonzero once a kernel gave up waiting for its copies
   int num_sms;
   int smem_limit;             // opt-in shared memory per block

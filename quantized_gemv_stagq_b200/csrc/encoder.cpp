@@ -18,12 +18,20 @@
 //   6. base by nearest rounding (half up), 7. planes = sign of the residual
 //      with sign(0) = +1 and half-steps s / 2^(k-1) (Eq. 7); held-out
 //      positions keep zero digits.
+// stagq_encode_guarded replaces step 1 by the paper's pre-grid ratio guard
+// (Section 3.5: a group's largest-|w| entry when it exceeds T times the
+// second largest) and adds the post-grid guard (Appendix E: per row, the
+// position with the largest two-bit error (w - (lo + s q))^2; its base digit
+// stays, its planes are zero, and it records the fp16 residual; the
+// reconstruction there is lo + s q + residual, Eq. 4). The post-grid entry's
+// column carries STAGQ_SIDE_POST.
 // Every floating-point step is fp64 and sums run in index order, so the
 // fields are reproducible bit for bit.
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <functional>
+#include <string>
 #include <thread>
 #include <vector>
 
@@ -79,24 +87,73 @@ extern "C" int64_t stagq_side_record_count(int32_t out, int32_t in, double densi
   return (int64_t)std::floor(density * (double)out * (double)in + 0.5);
 }
 
+namespace {
+
+// Steps 2-7 (and the post-grid guard) for a given pre-grid hold-out set;
+// writes at most `cap` side-record entries and sets f->nnz.
+int encode_with(const uint16_t* w, const std::vector<uint8_t>& held, bool post_guard, int32_t pair_mode,
+                int32_t n_threads, int64_t cap, stagq_fields* f);
+
+int check_encode_args(const uint16_t* w, stagq_fields* f, int32_t pair_mode, const char* who) {
+  if (!w || !f) return fail(STAGQ_EINVAL, std::string(who) + ": null argument");
+  const int64_t out = f->out, in = f->in, g = f->group;
+  if (out <= 0 || in <= 0 || g <= 0 || in % g) return fail(STAGQ_EINVAL, std::string(who) + ": bad shape or group");
+  if (in > STAGQ_MAX_IN) return fail(STAGQ_EINVAL, std::string(who) + ": in exceeds STAGQ_MAX_IN");
+  if (f->n_planes < 0 || f->n_planes > STAGQ_MAX_PLANES)
+    return fail(STAGQ_EINVAL, std::string(who) + ": n_planes out of range");
+  if (pair_mode != STAGQ_PAIR_SEARCH && pair_mode != STAGQ_PAIR_FAST)
+    return fail(STAGQ_EINVAL, std::string(who) + ": unknown pair mode");
+  if (!f->q || (f->n_planes && !f->planes) || !f->pair_idx || !f->row_ptr)
+    return fail(STAGQ_EINVAL, std::string(who) + ": null field buffer");
+  return STAGQ_OK;
+}
+
+}  // namespace
+
+extern "C" int64_t stagq_guard_capacity(int32_t out, int32_t in, int32_t group) {
+  if (out <= 0 || in <= 0 || group <= 0) return 0;
+  return (int64_t)out * (in / group) + out;
+}
+
+extern "C" int stagq_encode_guarded(const uint16_t* w, double ratio_T, int32_t post_guard, int32_t pair_mode,
+                                    int32_t n_threads, stagq_fields* f) {
+  int st = check_encode_args(w, f, pair_mode, "stagq_encode_guarded");
+  if (st) return st;
+  if (!(ratio_T >= 1.0)) return fail(STAGQ_EINVAL, "stagq_encode_guarded: ratio_T must be >= 1");
+  const int64_t out = f->out, in = f->in, g = f->group, ng = in / g;
+  const int64_t cap = f->nnz;
+  if (cap < stagq_guard_capacity((int32_t)out, (int32_t)in, (int32_t)g))
+    return fail(STAGQ_EINVAL, "stagq_encode_guarded: f->nnz must be at least stagq_guard_capacity");
+  if (cap && (!f->col || !f->val)) return fail(STAGQ_EINVAL, "stagq_encode_guarded: null field buffer");
+  // pre-grid ratio guard: per group the first largest |w| (fp16 magnitude
+  // bits order like |w|), held out when |w1| > T |w2|, w2 the largest of the rest.
+  std::vector<uint8_t> held(out * in, 0);
+  parallel_for(out * ng, n_threads, [&](int64_t a, int64_t b) {
+    for (int64_t G = a; G < b; ++G) {
+      const int64_t base = (G / ng) * in + (G % ng) * g;
+      int64_t j1 = 0;
+      for (int64_t c = 1; c < g; ++c)
+        if ((w[base + c] & 0x7FFF) > (w[base + j1] & 0x7FFF)) j1 = c;
+      double a2 = 0.0;
+      for (int64_t c = 0; c < g; ++c)
+        if (c != j1) a2 = std::max(a2, half_to_double(w[base + c] & 0x7FFF));
+      const double a1 = half_to_double(w[base + j1] & 0x7FFF);
+      if (a1 > ratio_T * a2) held[base + j1] = 1;
+    }
+  });
+  return encode_with(w, held, post_guard != 0, pair_mode, n_threads, cap, f);
+}
+
 extern "C" int stagq_encode(const uint16_t* w, double density, int32_t pair_mode, int32_t n_threads,
                             stagq_fields* f) {
-  if (!w || !f) return fail(STAGQ_EINVAL, "stagq_encode: null argument");
-  const int64_t out = f->out, in = f->in, g = f->group;
-  const int n_planes = f->n_planes;
-  if (out <= 0 || in <= 0 || g <= 0 || in % g) return fail(STAGQ_EINVAL, "stagq_encode: bad shape or group");
-  if (in > STAGQ_MAX_IN) return fail(STAGQ_EINVAL, "stagq_encode: in exceeds STAGQ_MAX_IN");
-  if (n_planes < 0 || n_planes > STAGQ_MAX_PLANES) return fail(STAGQ_EINVAL, "stagq_encode: n_planes out of range");
+  int st = check_encode_args(w, f, pair_mode, "stagq_encode");
+  if (st) return st;
   if (!(density >= 0.0 && density <= 1.0)) return fail(STAGQ_EINVAL, "stagq_encode: density outside [0,1]");
-  if (pair_mode != STAGQ_PAIR_SEARCH && pair_mode != STAGQ_PAIR_FAST)
-    return fail(STAGQ_EINVAL, "stagq_encode: unknown pair mode");
+  const int64_t out = f->out, in = f->in;
   const int64_t nnz = stagq_side_record_count((int32_t)out, (int32_t)in, density);
   if (f->nnz != nnz) return fail(STAGQ_EINVAL, "stagq_encode: f->nnz must equal stagq_side_record_count");
-  if (!f->q || (n_planes && !f->planes) || !f->pair_idx || !f->row_ptr || (nnz && (!f->col || !f->val)))
-    return fail(STAGQ_EINVAL, "stagq_encode: null field buffer");
-
-  const int N = 2 + n_planes;
-  const int64_t total = out * in, ng = in / g, ngroups = out * ng;
+  if (nnz && (!f->col || !f->val)) return fail(STAGQ_EINVAL, "stagq_encode: null field buffer");
+  const int64_t total = out * in;
 
   // 1. side record: top-|w| by the magnitude bits (monotone in |w|), ties to the smaller index.
   std::vector<uint8_t> held(total, 0);
@@ -118,6 +175,17 @@ extern "C" int stagq_encode(const uint16_t* w, double density, int32_t pair_mode
       else if (m == thr && need_tied > 0) { held[i] = 1; --need_tied; }
     }
   }
+  return encode_with(w, held, false, pair_mode, n_threads, nnz, f);
+}
+
+namespace {
+
+int encode_with(const uint16_t* w, const std::vector<uint8_t>& held, bool post_guard, int32_t pair_mode,
+                int32_t n_threads, int64_t cap, stagq_fields* f) {
+  const int64_t out = f->out, in = f->in, g = f->group;
+  const int n_planes = f->n_planes;
+  const int N = 2 + n_planes;
+  const int64_t total = out * in, ng = in / g, ngroups = out * ng;
 
   // 2-3. clipped groups and initial pairs.
   std::vector<double> lo0(ngroups), s0(ngroups);
@@ -243,17 +311,48 @@ extern "C" int stagq_encode(const uint16_t* w, double density, int32_t pair_mode
     }
   });
 
+  // post-grid guard: per row, the first position (not held out) with the
+  // largest (w - (lo + s q))^2; keep q, zero its planes, record the residual.
+  std::vector<int64_t> post_col(out, -1);
+  std::vector<uint16_t> post_val(out, 0);
+  if (post_guard) {
+    parallel_for(out, n_threads, [&](int64_t a, int64_t b) {
+      for (int64_t r = a; r < b; ++r) {
+        double best = -1.0, best_r2 = 0.0;
+        int64_t bc = -1;
+        for (int64_t c = 0; c < in; ++c) {
+          const int64_t idx = r * in + c;
+          if (held[idx]) continue;
+          const int p = f->pair_idx[r * ng + c / g];
+          const double r2 = tab_lo[p] + tab_s[p] * (double)f->q[idx];
+          const double d = half_to_double(w[idx]) - r2;
+          const double e = d * d;
+          if (e > best) { best = e; bc = c; best_r2 = r2; }
+        }
+        if (bc < 0) continue;
+        post_col[r] = bc;
+        post_val[r] = double_to_half(half_to_double(w[r * in + bc]) - best_r2);
+        for (int k = 0; k < n_planes; ++k) f->planes[(int64_t)k * total + r * in + bc] = 0;
+      }
+    });
+  }
+
   // side record, row-major CSR
   int64_t e = 0;
   for (int64_t r = 0; r < out; ++r) {
     f->row_ptr[r] = (int32_t)e;
     for (int64_t c = 0; c < in; ++c) {
-      if (!held[r * in + c]) continue;
-      f->col[e] = (uint16_t)c;
-      f->val[e] = w[r * in + c];
+      const bool pre = held[r * in + c] != 0, post = post_col[r] == c;
+      if (!pre && !post) continue;
+      if (e >= cap) return fail(STAGQ_EINVAL, "encoder: side record exceeds f->nnz");
+      f->col[e] = (uint16_t)(post ? (c | STAGQ_SIDE_POST) : c);
+      f->val[e] = post ? post_val[r] : w[r * in + c];
       ++e;
     }
   }
   f->row_ptr[out] = (int32_t)e;
+  f->nnz = e;
   return STAGQ_OK;
 }
+
+}  // namespace

@@ -83,9 +83,19 @@ struct GemvKernelArgs {
   DeviceMatrix m;
   GemvPlan plan;
   const float2* table;  // (lo_M, s_M c_M) of this precision
+  const float* dlo;     // lo - lo_M of this precision (post-grid entries)
   const __half* x;
   void* y;
   int y_f32;
+};
+
+// What a post-grid entry needs beside its residual: the pair byte of its
+// group (row u's pair bytes start at prow + u * pstep in the slot) and
+// lo - lo_M of that pair.
+struct PostCtx {
+  const uint8_t* prow;
+  uint32_t pstep;
+  const float* dlo;
 };
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // a copy that has not landed in 2 s never will
@@ -248,9 +258,20 @@ __device__ __forceinline__ int lo_index(int col, int gs) {
 // the 32 / NR lanes of group u (lane / (32 / NR)). Adds x~_c (v - lo_M) to
 // v[u]; lo_M of column c's group is read from lo_s[u][c's lane][group], where
 // every lane of the warp left its own lo_M per row and group.
+// The correction factor of entry `en` of row ur: v - lo_M for a pre-grid
+// entry, r + (lo - lo_M) for a post-grid one (bit 15), Eq. (4).
+template <int G>
+__device__ __forceinline__ float entry_delta(uint32_t en, int col, const float* lo_row, int gs, const PostCtx& pc,
+                                             int ur) {
+  const float v = __half2float(__ushort_as_half((unsigned short)(en >> 16)));
+  if (en & 0x8000u) return v + __ldg(pc.dlo + pc.prow[ur * pc.pstep + (col >> gs)]);
+  return v - lo_row[lo_index<G>(col, gs)];
+}
+
 template <int NR, int G>
 __device__ __forceinline__ void side_record(int o_lo, int o_hi, const uint32_t* ents, const int16_t* xq,
-                                            const float* xscale, const float* lo_s, int lane, int gs, float (&v)[NR]) {
+                                            const float* xscale, const float* lo_s, int lane, int gs,
+                                            const PostCtx& pc, float (&v)[NR]) {
   constexpr int LPR = 32 / NR;  // lanes per row
   const int ur = lane / LPR;
   const float* lo_row = lo_s + ur * 32 * G;
@@ -258,9 +279,9 @@ __device__ __forceinline__ void side_record(int o_lo, int o_hi, const uint32_t* 
   for (int j = o_lo + lane % LPR; __any_sync(kFull, j < o_hi); j += LPR) {
     if (j < o_hi) {
       const uint32_t en = ents[j];
-      const int col = (int)(en & 0xFFFFu);
+      const int col = (int)(en & 0x7FFFu);
       const float xv = (float)xq[xq_elem(col)] * xscale[col >> 6];
-      cs = fmaf(xv, __half2float(__ushort_as_half((unsigned short)(en >> 16))) - lo_row[lo_index<G>(col, gs)], cs);
+      cs = fmaf(xv, entry_delta<G>(en, col, lo_row, gs, pc, ur), cs);
     }
   }
 #pragma unroll
@@ -271,7 +292,7 @@ __device__ __forceinline__ void side_record(int o_lo, int o_hi, const uint32_t* 
 template <int NR, int NB, int G>
 __device__ __forceinline__ void side_record_nb(int o_lo, int o_hi, const uint32_t* ents, const int16_t* xq,
                                                const float* xscale, int in, int nchunk, const float* lo_s, int lane,
-                                               int gs, float (&v)[NB][NR]) {
+                                               int gs, const PostCtx& pc, float (&v)[NB][NR]) {
   constexpr int LPR = 32 / NR;  // lanes per row
   const int ur = lane / LPR;
   const float* lo_row = lo_s + ur * 32 * G;
@@ -281,8 +302,8 @@ __device__ __forceinline__ void side_record_nb(int o_lo, int o_hi, const uint32_
   for (int e = o_lo + lane % LPR; __any_sync(kFull, e < o_hi); e += LPR) {
     if (e < o_hi) {
       const uint32_t en = ents[e];
-      const int col = (int)(en & 0xFFFFu);
-      const float d = __half2float(__ushort_as_half((unsigned short)(en >> 16))) - lo_row[lo_index<G>(col, gs)];
+      const int col = (int)(en & 0x7FFFu);
+      const float d = entry_delta<G>(en, col, lo_row, gs, pc, ur);
       const int xe = xq_elem(col);
 #pragma unroll
       for (int j = 0; j < NB; ++j) cs[j] = fmaf((float)xq[j * in + xe] * xscale[j * nchunk + (col >> 6)], d, cs[j]);
@@ -303,8 +324,9 @@ __device__ __forceinline__ void block_rows(const uint32_t (&X)[32], float xs, co
                                            int nchunk, int cc, bool active, const uint8_t* sb, RowOffsets off,
                                            RowOffsets step, uint32_t plane_stride, const float2* tab, int mine,
                                            const int32_t* o, const uint32_t* ents, float* lo_w, int lane, int gs,
-                                           float* pout, int pstep) {
+                                           const float* dlo, float* pout, int pstep) {
   float v[NB][NR], lo[NR][G];
+  const PostCtx pc = {sb + off.g - ((cc * kChunk) >> gs), step.g, dlo};
   if constexpr (NB == 1) {
     rows_dot<M, NR, G>(X, xs, xsg, sb, off, step, plane_stride, tab, v[0], lo);
   } else {
@@ -319,10 +341,10 @@ __device__ __forceinline__ void block_rows(const uint32_t (&X)[32], float xs, co
   const int ur = lane / (32 / NR);
   if constexpr (NB == 1) {
     side_record<NR, G>(o[ur < mine ? ur : mine], o[ur + 1 < mine ? ur + 1 : mine], ents, xq, xscale, lo_w, lane, gs,
-                       v[0]);
+                       pc, v[0]);
   } else {
     side_record_nb<NR, NB, G>(o[ur < mine ? ur : mine], o[ur + 1 < mine ? ur + 1 : mine], ents, xq, xscale, in,
-                              nchunk, lo_w, lane, gs, v);
+                              nchunk, lo_w, lane, gs, pc, v);
   }
 #pragma unroll
   for (int j = 0; j < NB; ++j) {
@@ -519,12 +541,13 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
     const int mine = nr == BR ? UP : (nr > rg ? (nr - rg + RG - 1) / RG : 0);
     if (mine == UP || 2 * mine > UP) {
       block_rows<M, UP, NB, G>(X, xs, xsg, xq, xscale, xsum, xsum16, in, nchunk, cc, active, sb, off, step,
-                               plane_stride, tab, mine, o, ents, lo_w, lane, P.group_shift, pout, pstep);
+                               plane_stride, tab, mine, o, ents, lo_w, lane, P.group_shift, a.dlo, pout, pstep);
     } else {
       for (int u = 0; u < mine; ++u) {
         const RowOffsets ou = {off.b + u * step.b, off.p + u * step.p, off.g + u * step.g};
         block_rows<M, 1, NB, G>(X, xs, xsg, xq, xscale, xsum, xsum16, in, nchunk, cc, active, sb, ou, step,
-                                plane_stride, tab, 1, o + u, ents, lo_w, lane, P.group_shift, pout + u * pstep, pstep);
+                                plane_stride, tab, 1, o + u, ents, lo_w, lane, P.group_shift, a.dlo, pout + u * pstep,
+                                pstep);
         __syncwarp();  // lo_w is rewritten by the next row
       }
     }
@@ -616,6 +639,7 @@ cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const vo
   a.m = m;
   a.plan = plan;
   a.table = m.tables + 256 * (M - 2);
+  a.dlo = m.dlo + 256 * (M - 2);
   a.x = reinterpret_cast<const __half*>(x);
   a.y = y;
   a.y_f32 = y_f32;

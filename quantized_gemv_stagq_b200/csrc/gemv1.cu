@@ -60,6 +60,7 @@ struct Gemv1Args {
   DeviceMatrix m;
   Gemv1Plan plan;
   const float2* table;  // (lo_M, s_M c_M) of this precision
+  const float* dlo;     // lo - lo_M of this precision (post-grid entries)
   const __half* x;
   void* y;
   int y_f32;
@@ -399,10 +400,13 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
         const int j = jb + 32 * k;
         if (j < j1) {
           const uint32_t en = ents[j];
-          const int e = (int)(en & 0xFFFFu);  // x~ slot; e >> 6 is the column's 64-chunk
+          const int e = (int)(en & 0x7FFFu);  // x~ slot; e >> 6 is the column's 64-chunk
           const int grp = G == 1 ? e >> gs : column_of_xq_slot(e) >> gs;  // the column's group
-          const float lo = tab[pairs[(int)rowid[j] * ps + grp]].x;
-          term[j] = (float)xq[e] * xscale[e >> 6] * (__half2float(__ushort_as_half((unsigned short)(en >> 16))) - lo);
+          const int pb = pairs[(int)rowid[j] * ps + grp];
+          const float v = __half2float(__ushort_as_half((unsigned short)(en >> 16)));
+          // pre-grid: v - lo_M; post-grid (bit 15): r + (lo - lo_M), Eq. (4)
+          const float d = (en & 0x8000u) ? v + __ldg(a.dlo + pb) : v - tab[pb].x;
+          term[j] = (float)xq[e] * xscale[e >> 6] * d;
         }
       }
     }
@@ -464,6 +468,7 @@ cudaError_t launch1_mu(const DeviceMatrix& m, const Gemv1Plan& plan, const void*
   a.m = m;
   a.plan = plan;
   a.table = m.tables + 256 * (M - 2);
+  a.dlo = m.dlo + 256 * (M - 2);
   a.x = reinterpret_cast<const __half*>(x);
   a.y = y;
   a.y_f32 = y_f32;

@@ -40,11 +40,13 @@ int validate_stream(const stagq_host_stream* s) {
     if (s->row_ptr[r + 1] - s->row_ptr[r] > s->in) return fail(STAGQ_EFORMAT, "row holds more entries than columns");
   }
   if (s->row_ptr[s->out] != s->nnz) return fail(STAGQ_EFORMAT, "row_ptr[out] != nnz");
+  constexpr uint16_t kCol = 0x7FFF;  // bit 15: post-grid flag (STAGQ_SIDE_POST)
   for (int64_t e = 0; e < s->nnz; ++e)
-    if (s->col[e] >= s->in) return fail(STAGQ_EFORMAT, "side-record column >= in");
+    if ((s->col[e] & kCol) >= s->in) return fail(STAGQ_EFORMAT, "side-record column >= in");
   for (int64_t r = 0; r < s->out; ++r)
     for (int64_t e = (int64_t)s->row_ptr[r] + 1; e < s->row_ptr[r + 1]; ++e)
-      if (s->col[e] <= s->col[e - 1]) return fail(STAGQ_EFORMAT, "side-record columns not increasing in a row");
+      if ((s->col[e] & kCol) <= (s->col[e - 1] & kCol))
+        return fail(STAGQ_EFORMAT, "side-record columns not increasing in a row");
   return STAGQ_OK;
 }
 

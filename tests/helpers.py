@@ -16,8 +16,14 @@ def to_lib_fields(F) -> "Q.Fields":
                     pair_idx=np.ascontiguousarray(F.pair_idx, np.uint8),
                     cb_log2s=F.cb_log2s.view(np.uint16).copy(),
                     cb_lo_over_s=F.cb_lo_over_s.view(np.uint16).copy(),
-                    row_ptr=F.row_ptr.astype(np.int32), col=F.col.astype(np.uint16),
+                    row_ptr=F.row_ptr.astype(np.int32), col=lib_columns(F),
                     val=F.val.view(np.uint16).copy())
+
+
+def lib_columns(F) -> np.ndarray:
+    """The oracle's side-record columns as the library stores them: bit 15
+    (STAGQ_SIDE_POST) marks a post-grid entry."""
+    return (F.col.astype(np.uint16) | (F.post_flags.astype(np.uint16) << 15)).astype(np.uint16)
 
 
 def fields_equal(F, P) -> dict:
@@ -28,7 +34,7 @@ def fields_equal(F, P) -> dict:
         pair_idx=bool(np.array_equal(F.pair_idx, P.pair_idx)),
         q=bool(np.array_equal(F.q, P.q)),
         planes=bool(np.array_equal(F.planes, P.planes)),
-        side_record=bool(np.array_equal(F.row_ptr, P.row_ptr) and np.array_equal(F.col, P.col)
+        side_record=bool(np.array_equal(F.row_ptr, P.row_ptr) and np.array_equal(lib_columns(F), P.col)
                          and np.array_equal(F.val.view(np.uint16), P.val)),
     )
 

@@ -196,15 +196,15 @@ LLAMA = list(synth.LLAMA31_8B_LINEARS.items())
 SAMPLE_ROWS = 48
 
 
-def _sampled_rows_case(out, inp, group, n_planes, density, seed, bits_list, kernels, batch4=True):
+def _sampled_rows_case(out, inp, group, n_planes, density, seed, bits_list, kernels, batch4=True, **guard):
     """Library encoder -> GPU (as the bench does); the oracle encodes the same
     weights itself on sampled rows; fields and y agree on those rows."""
     W = synth.weights(out, inp, seed=seed)
-    P = Q.stagq_encode(W, group, n_planes, density, "fast")
+    P = Q.stagq_encode(W, group, n_planes, density, "fast", **guard)
     m = Q.stagq_load(Q.stagq_pack(P), 0)
     rng = np.random.default_rng(out + inp)
     rows = np.unique(np.concatenate([[0, out - 1], rng.choice(out, SAMPLE_ROWS, replace=False)]))
-    F = O.encode(W, group, n_planes, density, "fast", rows=rows)
+    F = O.encode(W, group, n_planes, density, "fast", rows=rows, **guard)
     Psub = Q.Fields(F.out, inp, group, n_planes, P.q[rows], P.planes[:, rows], P.pair_idx[rows],
                     P.cb_log2s, P.cb_lo_over_s,
                     np.concatenate([[0], np.cumsum(np.diff(P.row_ptr)[rows])]).astype(np.int32),
@@ -256,3 +256,56 @@ def test_full_size_phi4_olmo2_sampled_rows(name, shape):
 def test_full_size_sweep_sampled_rows(group, density):
     """The precision/structure sweep: base + 4 planes read at 2..6 bits."""
     _sampled_rows_case(14336, 4096, group, 4, density, 3000 + group, (2, 3, 4, 5, 6), _kernels(), batch4=False)
+
+
+# ------------------------------------- side-record guards (Section 3.5, Appendix E)
+
+GUARDED = [
+    # out, in, group, n_planes, ratio T, post-grid guard, seed
+    (512, 512, 32, 2, 4.0, True, 21),      # the tiny workload at the paper's g = 32
+    (96, 2048, 64, 4, 4.0, True, 22),      # deep stream, p2..p6
+    (37, 640, 128, 3, 2.0, True, 23),      # ragged K, fewer rows than SMs, lower T
+    (300, 5120, 16, 2, 4.0, True, 24),     # g = 16, K = 2.5 warp tiles
+    (1, 4096, 128, 2, 4.0, True, 25),      # a single row
+    (200, 4096, 128, 1, 8.0, False, 26),   # pre-grid guard only
+]
+
+
+def _guarded_fields(case):
+    out, inp, g, npl, T, post, seed = case
+    W = synth.weights(out, inp, seed)
+    W[0, 7] = np.float16(0.8)              # a dominant entry in row 0's first group
+    return O.encode(W, g, npl, mode="fast", guard="ratio", ratio_T=T, post_guard=post)
+
+
+@pytest.mark.parametrize("case", GUARDED, ids=lambda c: f"{c[0]}x{c[1]}g{c[2]}p{c[3]}T{c[4]}{'post' if c[5] else ''}")
+def test_guarded_gemv_matches_oracle(case):
+    """Pre-grid entries (P = recorded value) and post-grid entries (P = lo + s q
+    + r, zero planes) through both n = 1 kernels and the batched launch."""
+    F = _guarded_fields(case)
+    assert F.nnz > 0 and F.post_flags.sum() == (F.out if case[5] else 0)
+    m = _load(F)
+    u = torch.empty(F.out, F.inp, dtype=torch.uint8, device="cuda")
+    for M in range(2, 3 + F.n_planes):
+        Q.stagq_decode_levels(m, M, u)
+        torch.cuda.synchronize()
+        assert np.array_equal(u.cpu().numpy(), O.decode_levels(F, M)), f"levels p{M}"
+        x = synth.activations(4, F.inp, case[6] + M)
+        ref = O.gemv(F, M, x)
+        for kern in (Q.STAGQ_KERNEL_GENERAL, Q.STAGQ_KERNEL_SINGLE):
+            check_close(_gemv(m, M, x[:1], kernel=kern)[0], ref[0], f"p{M} kernel {kern}")
+        for n in (2, 4):
+            got = _gemv(m, M, x[:n])
+            for j in range(n):
+                check_close(got[j], ref[j], f"p{M} n{n} col{j}")
+    Q.stagq_check(m)
+    m.free()
+
+
+@pytest.mark.parametrize("name,shape,group", [("gate_proj", (14336, 4096), 32), ("down_proj", (4096, 14336), 128)])
+def test_full_size_guarded_sampled_rows(name, shape, group):
+    """Full Llama-3.1-8B shapes with the ratio guard (T = 4) and the post-grid
+    guard, as the paper configures its feed-forward matrices (Table 6)."""
+    out, inp = shape
+    _sampled_rows_case(out, inp, group, 2, 0.0, 4000 + out + group, (2, 3, 4), _kernels(), batch4=True,
+                       guard="ratio", ratio_T=4.0)

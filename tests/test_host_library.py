@@ -45,6 +45,34 @@ def test_encoder_matches_oracle_bit_exactly(out, inp, g, npl, dens, mode):
     assert all(eq.values()), eq
 
 
+@pytest.mark.parametrize("out,inp,g,npl,T,post,mode", [
+    (64, 512, 64, 2, 4.0, True, "fast"),
+    (48, 256, 16, 4, 4.0, True, "search"),
+    (40, 384, 32, 3, 2.0, True, "fast"),
+    (16, 256, 128, 2, 8.0, False, "search"),
+    (8, 128, 64, 1, 4.0, True, "fast"),
+])
+def test_guarded_encoder_matches_oracle_bit_exactly(out, inp, g, npl, T, post, mode):
+    """The paper's guards (pre-grid ratio criterion, post-grid per-row guard):
+    every field, the post-grid flags in the columns and the residuals."""
+    W = synth.weights(out, inp, seed=out * 5 + inp)
+    W[3, 5] = np.float16(0.9)                 # a dominant entry: the ratio guard takes it
+    F = O.encode(W, group=g, n_planes=npl, mode=mode, guard="ratio", ratio_T=T, post_guard=post)
+    P = Q.stagq_encode(W, group=g, n_planes=npl, mode=mode, guard="ratio", ratio_T=T, post_guard=post, n_threads=3)
+    eq = fields_equal(F, P)
+    assert all(eq.values()), eq
+    assert F.post_flags.sum() == (out if post else 0)
+    assert ((P.col & Q.STAGQ_SIDE_POST) != 0).sum() == F.post_flags.sum()
+
+
+def test_guarded_stream_packs_and_rereads():
+    W = synth.weights(24, 640, seed=7)
+    F = O.encode(W, group=32, n_planes=2, mode="fast", guard="ratio", ratio_T=4.0)
+    S = Q.stagq_pack(to_lib_fields(F))
+    for M in (2, 3, 4):
+        assert np.array_equal(Q.stagq_unpack_levels_host(S, M), O.decode_levels(F, M)), M
+
+
 def test_encoder_handles_constant_and_zero_groups():
     W = np.zeros((4, 256), np.float16)
     W[1, :128] = np.float16(0.25)
