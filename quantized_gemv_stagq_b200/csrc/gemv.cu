@@ -260,6 +260,8 @@ __device__ __forceinline__ int lo_index(int col, int gs) {
 // every lane of the warp left its own lo_M per row and group.
 // The correction factor of entry `en` of row ur: v - lo_M for a pre-grid
 // entry, r + (lo - lo_M) for a post-grid one (bit 15), Eq. (4).
+// Kernels of a matrix with post-grid entries (POST) use it; the others keep
+// the plain pre-grid expression (bit 15 is never set there).
 template <int G>
 __device__ __forceinline__ float entry_delta(uint32_t en, int col, const float* lo_row, int gs, const PostCtx& pc,
                                              int ur) {
@@ -268,7 +270,7 @@ __device__ __forceinline__ float entry_delta(uint32_t en, int col, const float* 
   return v - lo_row[lo_index<G>(col, gs)];
 }
 
-template <int NR, int G>
+template <int NR, int G, bool POST>
 __device__ __forceinline__ void side_record(int o_lo, int o_hi, const uint32_t* ents, const int16_t* xq,
                                             const float* xscale, const float* lo_s, int lane, int gs,
                                             const PostCtx& pc, float (&v)[NR]) {
@@ -279,9 +281,10 @@ __device__ __forceinline__ void side_record(int o_lo, int o_hi, const uint32_t* 
   for (int j = o_lo + lane % LPR; __any_sync(kFull, j < o_hi); j += LPR) {
     if (j < o_hi) {
       const uint32_t en = ents[j];
-      const int col = (int)(en & 0x7FFFu);
+      const int col = (int)(en & (POST ? 0x7FFFu : 0xFFFFu));  // bit 15: post-grid flag
       const float xv = (float)xq[xq_elem(col)] * xscale[col >> 6];
-      cs = fmaf(xv, entry_delta<G>(en, col, lo_row, gs, pc, ur), cs);
+      if constexpr (POST) cs = fmaf(xv, entry_delta<G>(en, col, lo_row, gs, pc, ur), cs);
+      else cs = fmaf(xv, __half2float(__ushort_as_half((unsigned short)(en >> 16))) - lo_row[lo_index<G>(col, gs)], cs);
     }
   }
 #pragma unroll
@@ -289,7 +292,7 @@ __device__ __forceinline__ void side_record(int o_lo, int o_hi, const uint32_t* 
 }
 
 // As side_record for NB activation vectors: v[j][u] += x~_j,c (v - lo_M).
-template <int NR, int NB, int G>
+template <int NR, int NB, int G, bool POST>
 __device__ __forceinline__ void side_record_nb(int o_lo, int o_hi, const uint32_t* ents, const int16_t* xq,
                                                const float* xscale, int in, int nchunk, const float* lo_s, int lane,
                                                int gs, const PostCtx& pc, float (&v)[NB][NR]) {
@@ -302,8 +305,10 @@ __device__ __forceinline__ void side_record_nb(int o_lo, int o_hi, const uint32_
   for (int e = o_lo + lane % LPR; __any_sync(kFull, e < o_hi); e += LPR) {
     if (e < o_hi) {
       const uint32_t en = ents[e];
-      const int col = (int)(en & 0x7FFFu);
-      const float d = entry_delta<G>(en, col, lo_row, gs, pc, ur);
+      const int col = (int)(en & (POST ? 0x7FFFu : 0xFFFFu));  // bit 15: post-grid flag
+      float d;
+      if constexpr (POST) d = entry_delta<G>(en, col, lo_row, gs, pc, ur);
+      else d = __half2float(__ushort_as_half((unsigned short)(en >> 16))) - lo_row[lo_index<G>(col, gs)];
       const int xe = xq_elem(col);
 #pragma unroll
       for (int j = 0; j < NB; ++j) cs[j] = fmaf((float)xq[j * in + xe] * xscale[j * nchunk + (col >> 6)], d, cs[j]);
@@ -318,7 +323,7 @@ __device__ __forceinline__ void side_record_nb(int o_lo, int o_hi, const uint32_
 // The UP rows (or, for a short block, `mine` rows one at a time) of one block
 // for this lane's chunk: dot products, side record, and the cross-lane sums
 // into pout[u * pstep + j] (row u, vector j).
-template <int M, int NR, int NB, int G>
+template <int M, int NR, int NB, int G, bool POST>
 __device__ __forceinline__ void block_rows(const uint32_t (&X)[32], float xs, const float (&xsg)[G], const int16_t* xq,
                                            const float* xscale, const float* xsum, const float* xsum16, int in,
                                            int nchunk, int cc, bool active, const uint8_t* sb, RowOffsets off,
@@ -326,7 +331,6 @@ __device__ __forceinline__ void block_rows(const uint32_t (&X)[32], float xs, co
                                            const int32_t* o, const uint32_t* ents, float* lo_w, int lane, int gs,
                                            const float* dlo, float* pout, int pstep) {
   float v[NB][NR], lo[NR][G];
-  const PostCtx pc = {sb + off.g - ((cc * kChunk) >> gs), step.g, dlo};
   if constexpr (NB == 1) {
     rows_dot<M, NR, G>(X, xs, xsg, sb, off, step, plane_stride, tab, v[0], lo);
   } else {
@@ -339,11 +343,13 @@ __device__ __forceinline__ void block_rows(const uint32_t (&X)[32], float xs, co
     for (int g = 0; g < G; ++g) lo_w[(u * 32 + lane) * G + g] = lo[u][g];
   __syncwarp();
   const int ur = lane / (32 / NR);
+  PostCtx pc = {nullptr, 0u, nullptr};
+  if constexpr (POST) pc = {sb + off.g - ((cc * kChunk) >> gs), step.g, dlo};  // read by post-grid entries only
   if constexpr (NB == 1) {
-    side_record<NR, G>(o[ur < mine ? ur : mine], o[ur + 1 < mine ? ur + 1 : mine], ents, xq, xscale, lo_w, lane, gs,
+    side_record<NR, G, POST>(o[ur < mine ? ur : mine], o[ur + 1 < mine ? ur + 1 : mine], ents, xq, xscale, lo_w, lane, gs,
                        pc, v[0]);
   } else {
-    side_record_nb<NR, NB, G>(o[ur < mine ? ur : mine], o[ur + 1 < mine ? ur + 1 : mine], ents, xq, xscale, in,
+    side_record_nb<NR, NB, G, POST>(o[ur < mine ? ur : mine], o[ur + 1 < mine ? ur + 1 : mine], ents, xq, xscale, in,
                               nchunk, lo_w, lane, gs, pc, v);
   }
 #pragma unroll
@@ -353,7 +359,7 @@ __device__ __forceinline__ void block_rows(const uint32_t (&X)[32], float xs, co
   }
 }
 
-template <int M, int UP, int NB, int G>
+template <int M, int UP, int NB, int G, bool POST>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKernelArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const GemvPlan& P = a.plan;
@@ -540,12 +546,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
     // missing rows masked, unless fewer than half of them are there
     const int mine = nr == BR ? UP : (nr > rg ? (nr - rg + RG - 1) / RG : 0);
     if (mine == UP || 2 * mine > UP) {
-      block_rows<M, UP, NB, G>(X, xs, xsg, xq, xscale, xsum, xsum16, in, nchunk, cc, active, sb, off, step,
+      block_rows<M, UP, NB, G, POST>(X, xs, xsg, xq, xscale, xsum, xsum16, in, nchunk, cc, active, sb, off, step,
                                plane_stride, tab, mine, o, ents, lo_w, lane, P.group_shift, a.dlo, pout, pstep);
     } else {
       for (int u = 0; u < mine; ++u) {
         const RowOffsets ou = {off.b + u * step.b, off.p + u * step.p, off.g + u * step.g};
-        block_rows<M, 1, NB, G>(X, xs, xsg, xq, xscale, xsum, xsum16, in, nchunk, cc, active, sb, ou, step,
+        block_rows<M, 1, NB, G, POST>(X, xs, xsg, xq, xscale, xsum, xsum16, in, nchunk, cc, active, sb, ou, step,
                                 plane_stride, tab, 1, o + u, ents, lo_w, lane, P.group_shift, a.dlo, pout + u * pstep,
                                 pstep);
         __syncwarp();  // lo_w is rewritten by the next row
@@ -616,11 +622,11 @@ __global__ void decode_levels_kernel(const DeviceMatrix m, uint8_t* u) {
 cudaError_t ensure_smem(const void* kern, int key, size_t smem) {
   constexpr int kMaxDev = 64;
   static std::mutex mu;
-  static size_t granted[kMaxDev][192] = {};  // key < 180: (M - 2, rows per warp, vectors, groups per chunk)
+  static size_t granted[kMaxDev][384] = {};  // key < 360: (M - 2, rows per warp, vectors, groups, post)
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (dev < 0 || dev >= kMaxDev || key < 0 || key >= 192) return cudaErrorInvalidValue;
+  if (dev < 0 || dev >= kMaxDev || key < 0 || key >= 384) return cudaErrorInvalidValue;
   std::lock_guard<std::mutex> lock(mu);
   if (granted[dev][key] >= smem) return cudaSuccess;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -644,8 +650,9 @@ cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const vo
   a.y = y;
   a.y_f32 = y_f32;
   const SmemLayout L = smem_layout(plan, m.in, M);
-  auto kern = gemv_kernel<M, UP, NB, G>;
-  const int key = (((M - 2) * 3 + (UP == 4 ? 2 : UP - 1)) * 4 + (NB - 1)) * 3 + (G == 4 ? 2 : G - 1);
+  auto kern = m.has_post ? gemv_kernel<M, UP, NB, G, true> : gemv_kernel<M, UP, NB, G, false>;
+  const int key = ((((M - 2) * 3 + (UP == 4 ? 2 : UP - 1)) * 4 + (NB - 1)) * 3 + (G == 4 ? 2 : G - 1)) * 2 +
+                  (m.has_post ? 1 : 0);
   cudaError_t err = ensure_smem(reinterpret_cast<const void*>(kern), key, L.total);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
