@@ -223,7 +223,8 @@ int stagq_gemv_n(stagq_handle h, int bits, const void* x, int n, void* y, void* 
  * As stagq_gemv_n; flags STAGQ_Y_F32 makes y fp32. For n = 1 the library has
  * two kernels with the same arithmetic per vector (results agree to fp32
  * rounding, each is deterministic): by default the single-vector kernel
- * serves matrices of more than 2^24 weights, where it measured faster, and the
+ * serves matrices of more than 2^24 weights or with groups below 64, where it
+ * measured faster, and the
  * general kernel everything else.
  * STAGQ_KERNEL_GENERAL / STAGQ_KERNEL_SINGLE force one of them (for tests and
  * measurements); forcing the single-vector kernel on a shape it cannot plan

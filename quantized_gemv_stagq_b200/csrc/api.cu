@@ -267,7 +267,10 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   // (entry rows, side-record terms, row sums), measured on chains of GEMVs at
   // 2..6 bits. On smaller matrices those phases dominate and the general
   // kernel is faster.
-  const bool large = (int64_t)s->out * s->in > ((int64_t)1 << 24);
+  // Groups below 64 weights give the general kernel one row per warp per
+  // block (registers); the single-vector kernel keeps two, so it serves them
+  // at any size.
+  const bool large = (int64_t)s->out * s->in > ((int64_t)1 << 24) || s->group < 64;
   for (int b = 2; b <= 2 + np; ++b) {
     h->plan1_ok[b] = make_plan1(m, b, &h->plan1[b]);
     h->prefer1[b] = large;

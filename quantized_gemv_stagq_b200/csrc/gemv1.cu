@@ -43,6 +43,7 @@
 
 #include <cstdint>
 #include <mutex>
+#include <type_traits>
 
 #include "device_matrix.hpp"
 #include "kernel_common.cuh"
@@ -394,22 +395,32 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
   if (ok) {
     const int nw = NW + 1, E = offs[rows];
     const int j0 = (int)((int64_t)E * warp / nw), j1 = (int)((int64_t)E * (warp + 1) / nw);
-    for (int jb = j0 + lane; jb < j1; jb += 4 * 32) {
+    // pre-grid entry: v - lo_M; post-grid entry (bit 15): r + (lo - lo_M), Eq. (4)
+    auto terms = [&](auto with_post) {
+      for (int jb = j0 + lane; jb < j1; jb += 4 * 32) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int j = jb + 32 * k;
-        if (j < j1) {
-          const uint32_t en = ents[j];
-          const int e = (int)(en & 0x7FFFu);  // x~ slot; e >> 6 is the column's 64-chunk
-          const int grp = G == 1 ? e >> gs : column_of_xq_slot(e) >> gs;  // the column's group
-          const int pb = pairs[(int)rowid[j] * ps + grp];
-          const float v = __half2float(__ushort_as_half((unsigned short)(en >> 16)));
-          // pre-grid: v - lo_M; post-grid (bit 15): r + (lo - lo_M), Eq. (4)
-          const float d = (en & 0x8000u) ? v + __ldg(a.dlo + pb) : v - tab[pb].x;
-          term[j] = (float)xq[e] * xscale[e >> 6] * d;
+        for (int k = 0; k < 4; ++k) {
+          const int j = jb + 32 * k;
+          if (j < j1) {
+            const uint32_t en = ents[j];
+            const int e = (int)(en & 0x7FFFu);  // x~ slot; e >> 6 is the column's 64-chunk
+            const int grp = G == 1 ? e >> gs : column_of_xq_slot(e) >> gs;  // the column's group
+            const int pb = pairs[(int)rowid[j] * ps + grp];
+            const float v = __half2float(__ushort_as_half((unsigned short)(en >> 16)));
+            float d;
+            if constexpr (decltype(with_post)::value) {
+              if (en & 0x8000u) d = v + __ldg(a.dlo + pb);
+              else d = v - tab[pb].x;
+            } else {
+              d = v - tab[pb].x;
+            }
+            term[j] = (float)xq[e] * xscale[e >> 6] * d;
+          }
         }
       }
-    }
+    };
+    if (a.m.has_post) terms(std::true_type{});
+    else terms(std::false_type{});
   }
   if (!ok && lane == 0) *flag = 1u;
   __syncthreads();
