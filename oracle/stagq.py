@@ -12,7 +12,9 @@ It covers three things:
 * the encoder of Sections 3.1-3.6 (+ Appendices B and E) for synthetic
   weights: side record (the workloads' global top-|w| density, or the
   paper's pre-grid ratio guard plus the post-grid guard), clipping, initial
-  pair, uniform codebooks, per-group pair choice by Eq. (5)-(6),
+  pair, codebooks (uniform, or Appendix E's choice among uniform, Lloyd and
+  anchored Lloyd placement with its fallback), per-group pair choice by
+  Eq. (5)-(6),
   nearest-rounding base, sign planes (Eq. (7));
 * the decoder: composite integer Eq. (8), affine map Eq. (10) (with the
   additive form Eq. (9) kept as a cross-check), complete reconstruction
@@ -41,6 +43,11 @@ INIT_EDGE_FRACTION = 0.06
 FLOOR_LAMBDA = 4.0
 # Section 3.1: two sixteen-entry codebooks per matrix.
 CODEBOOK_SIZE = 16
+# Appendix E, Lloyd's rule: Reading -- at most this many assignment steps.
+LLOYD_MAX_STEPS = 100
+# Appendix E: a matrix whose deepest-precision error exceeds this fraction of
+# its two-bit error under the chosen codebooks falls back to uniform placement.
+FALLBACK_RATIO = 0.1
 # Reading: a group whose clipped range is zero has no initial step; it gets
 # this placeholder, stays out of the codebook fit and takes its pair by the
 # Eq. (5) search in every mode.
@@ -304,6 +311,97 @@ def uniform_codebook(values: np.ndarray) -> np.ndarray:
     return np.array(cb, dtype=np.float64).astype(np.float16)
 
 
+def lloyd_codebook(values: np.ndarray, anchored: bool) -> np.ndarray:
+    """Appendix E, Lloyd's rule (and Lloyd's rule with its ends anchored at
+    the range of the initial pairs): sixteen points, each the mean of the
+    values nearest to it, as fp16.
+
+    Reading: the points start at the uniform placement (fp64); a step assigns
+    every value to its nearest point (ties to the lower index) and moves each
+    point to the mean of its values, summed in index order; a point with no
+    value stays; anchored, points 0 and 15 stay at the range ends. The steps
+    stop when no assignment changes, or after LLOYD_MAX_STEPS. With no values
+    the codebook is all zeros.
+    """
+    if values.size == 0:
+        return np.zeros(CODEBOOK_SIZE, dtype=np.float16)
+    v = np.asarray(values, dtype=np.float64).reshape(-1)
+    vmin, vmax = float(v.min()), float(v.max())
+    c = np.array([vmin + i * (vmax - vmin) / (CODEBOOK_SIZE - 1) for i in range(CODEBOOK_SIZE)])
+    assign = None
+    for _ in range(LLOYD_MAX_STEPS):
+        a = np.argmin(np.abs(v[:, None] - c[None, :]), axis=1)
+        if assign is not None and np.array_equal(a, assign):
+            break
+        assign = a
+        for i in range(CODEBOOK_SIZE):
+            if anchored and i in (0, CODEBOOK_SIZE - 1):
+                continue
+            sel = v[a == i]
+            if sel.size:
+                c[i] = _sum_in_order(sel) / sel.size
+    return c.astype(np.float16)
+
+
+CODEBOOK_RULES = ("uniform", "lloyd", "anchored")
+
+
+def codebook_by_rule(values: np.ndarray, rule: str) -> np.ndarray:
+    if rule == "uniform":
+        return uniform_codebook(values)
+    return lloyd_codebook(values, anchored=(rule == "anchored"))
+
+
+def first_term_min(Vc: np.ndarray, group: int, N: int, lo_tab, s_tab, skip,
+                   chunk: int = 256) -> np.ndarray:
+    """Per group: the smallest first term of Eq. (5) (the distortion averaged
+    over M = 2..N, no floor term) over the 256 pairs; groups in ``skip`` give 0."""
+    out, inp = Vc.shape
+    G = Vc.reshape(out * (inp // group), group)
+    best = np.empty(G.shape[0])
+    for c0 in range(0, G.shape[0], chunk):
+        V = G[c0:c0 + chunk][:, None, :]
+        _, _, recons = encode_digits(V, lo_tab[None, :, None], s_tab[None, :, None], N)
+        first = 0.0
+        for rec in recons:
+            first = first + _sum_in_order((V - rec) ** 2)
+        best[c0:c0 + chunk] = (first / (N - 1)).min(axis=1)
+    return np.where(skip.reshape(-1), 0.0, best)
+
+
+def choose_codebook_rules(Vc, group: int, N: int, lo0, s0, skip, empty):
+    """Appendix E: of the nine combinations of a rule for the log2(s)
+    codebook and a rule for the lo/s codebook, the one whose per-group best
+    first term of Eq. (5), summed over the matrix (group order), is smallest.
+    Reading: ties go to the first combination, s-rule outer, in the order
+    uniform, Lloyd, anchored Lloyd. The codebooks are fitted to the groups
+    not in ``skip``; every group with a retained entry (not ``empty``) counts
+    in the sum. Returns (rule_s, rule_lo)."""
+    keep = ~skip
+    ls, rl = np.log2(s0[keep]), lo0[keep] / s0[keep]
+    best, arg = None, None
+    for rs in CODEBOOK_RULES:
+        for rr in CODEBOOK_RULES:
+            lo_tab, s_tab = pair_table(codebook_by_rule(ls, rs), codebook_by_rule(rl, rr))
+            tot = _sum_in_order(first_term_min(Vc, group, N, lo_tab, s_tab, empty))
+            if best is None or tot < best:
+                best, arg = tot, (rs, rr)
+    return arg
+
+
+def precision_errors(Vc, group: int, N: int, pair_idx, lo_tab, s_tab, skip):
+    """Sum over the matrix (group order, then index order) of the two-bit and
+    the deepest-precision (M = N) errors sum_c (V_c - W_c^(M))^2 of the
+    clipped groups under their pairs; groups in ``skip`` count 0."""
+    out, inp = Vc.shape
+    G = Vc.reshape(out * (inp // group), group)
+    p = pair_idx.reshape(-1).astype(np.int64)
+    _, _, recons = encode_digits(G, lo_tab[p][:, None], s_tab[p][:, None], N)
+    e2 = np.where(skip.reshape(-1), 0.0, _sum_in_order((G - recons[0]) ** 2))
+    eN = np.where(skip.reshape(-1), 0.0, _sum_in_order((G - recons[-1]) ** 2))
+    return _sum_in_order(e2), _sum_in_order(eN)
+
+
 def fit_codebooks(lo0: np.ndarray, s0: np.ndarray, skip: np.ndarray):
     """Section 3.1: one codebook in log2(s) and one in lo/s per matrix, fitted
     to the initial pairs of the groups not marked in ``skip`` (Reading: groups
@@ -399,7 +497,7 @@ def choose_pairs(Vc: np.ndarray, group: int, N: int, lo_tab, s_tab, empty,
 def encode(W: np.ndarray, group: int = 128, n_planes: int = 2,
            density: float = 0.005, mode: str = "search", rows=None,
            row_block: int = 512, guard: str = "density", ratio_T: float = 4.0,
-           post_guard: bool = True) -> Fields:
+           post_guard: bool = True, codebooks: str = "uniform") -> Fields:
     """Figure 3's encoder for synthetic weights (no AWQ scale: with x ~ N(0,1)
     every channel scale is equal):
 
@@ -408,7 +506,13 @@ def encode(W: np.ndarray, group: int = 128, n_planes: int = 2,
        the pre-grid ratio guard of Section 3.5 (``select_ratio_guard``, T =
        ``ratio_T``); P = fp16 value;
     2. clip held-out entries inward for the fit (``clip_held_out``);
-    3. initial pairs (Appendix B), 4. uniform codebooks (Appendix E),
+    3. initial pairs (Appendix B), 4. codebooks: ``codebooks="uniform"``
+       places both uniformly (Appendix E's first rule); ``"appendix_e"``
+       picks one of the nine rule combinations (``choose_codebook_rules``)
+       and falls back to uniform placement when the deepest precision's error
+       exceeds FALLBACK_RATIO of the two-bit error under the chosen codebooks
+       and the final pair choice (Reading: "six-bit" is the stream's deepest
+       precision N; with N = 2 the test always falls back);
     5. pair per group (Eq. (5) search, or the labelled fast rule),
     6. base by nearest rounding, 7. sign planes k = 3..N; held-out positions
        store zero digits (Reading: the planes skip them, Section 3.6, and the
@@ -446,6 +550,18 @@ def encode(W: np.ndarray, group: int = 128, n_planes: int = 2,
     Vc, empty = clip_held_out(W, mask, group)
     lo0, s0, flat = initial_pairs(Vc, group)
     cb_log2s, cb_lo_over_s = fit_codebooks(lo0, s0, empty | flat)
+    if codebooks == "appendix_e":
+        rs, rr = choose_codebook_rules(Vc, group, N, lo0, s0, empty | flat, empty)
+        keep = ~(empty | flat)
+        cand = (codebook_by_rule(np.log2(s0[keep]), rs), codebook_by_rule(lo0[keep] / s0[keep], rr))
+        lo_c, s_c = pair_table(*cand)
+        pidx = choose_pairs(Vc, group, N, lo_c, s_c, empty, mode=mode, lo0=lo0, s0=s0,
+                            cb_log2s=cand[0], cb_lo_over_s=cand[1], flat=flat)
+        e2, eN = precision_errors(Vc, group, N, pidx, lo_c, s_c, empty)
+        if not eN > FALLBACK_RATIO * e2:
+            cb_log2s, cb_lo_over_s = cand
+    elif codebooks != "uniform":
+        raise ValueError("codebooks must be 'uniform' or 'appendix_e'")
     lo_tab, s_tab = pair_table(cb_log2s, cb_lo_over_s)
 
     rows = np.arange(out) if rows is None else np.asarray(rows, dtype=np.int64)

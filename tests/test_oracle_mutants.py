@@ -51,6 +51,27 @@ def _base_digit_truncating(w, lo, s):
 
 
 _select_post_guard = O.select_post_guard
+
+
+def _lloyd_median(values, anchored):
+    """Moves points to the median of their values instead of the mean."""
+    v = np.asarray(values, dtype=np.float64).reshape(-1)
+    c = np.linspace(v.min(), v.max(), 16)
+    for _ in range(100):
+        a = np.argmin(np.abs(v[:, None] - c[None, :]), axis=1)
+        for i in range(16):
+            if anchored and i in (0, 15):
+                continue
+            if np.any(a == i):
+                c[i] = np.median(v[a == i])
+    return c.astype(np.float16)
+
+
+def _lloyd_unanchored(values, anchored):
+    return _lloyd_codebook(values, False)
+
+
+_lloyd_codebook = O.lloyd_codebook
 _decode = O.decode
 
 
@@ -85,6 +106,8 @@ def _ratio_guard_second_excluded_wrongly(W, group, T):
     ("base_digit", _base_digit_truncating, ["test_sign_planes_equal_nearest_level_rounding"]),
     ("select_ratio_guard", _ratio_guard_second_excluded_wrongly, ["test_ratio_guard_matches_brute_force"]),
     ("select_post_guard", _post_guard_wrong_error, ["test_post_guard_is_the_row_argmax_of_two_bit_error"]),
+    ("lloyd_codebook", _lloyd_median, ["test_lloyd_points_are_the_cluster_means"]),
+    ("lloyd_codebook", _lloyd_unanchored, ["test_lloyd_points_are_the_cluster_means"]),
     ("decode", _decode_post_as_recorded_value, ["test_post_entries_reconstruct_w_at_every_precision",
                                                 "test_gemv_with_guards_against_scalar_brute_force"]),
 ])

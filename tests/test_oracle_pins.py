@@ -447,3 +447,109 @@ def test_gemv_with_guards_against_scalar_brute_force():
                 acc += w * float(x[c])
             ref.append(acc)
         assert np.allclose(y, ref, rtol=1e-12, atol=1e-14), M
+
+
+# ------------------------------------------- codebook rules (Appendix E)
+
+def _clusters(rng, centers, counts, spread=1e-3):
+    return np.concatenate([c + spread * rng.standard_normal(n) for c, n in zip(centers, counts)])
+
+
+def test_lloyd_points_are_the_cluster_means():
+    """Sixteen tight clusters near the uniform points: Lloyd's rule moves each
+    point to the mean of its cluster (fp16 of the exact mean); anchored, the
+    two end points stay at the range ends."""
+    rng = np.random.default_rng(1)
+    centers = np.linspace(-3.0, 2.0, 16) + rng.uniform(-0.05, 0.05, 16)
+    counts = rng.integers(3, 40, 16)
+    v = _clusters(rng, centers, counts)
+    groups = np.split(v, np.cumsum(counts)[:-1])
+    means = np.array([math.fsum(gv) / gv.size for gv in groups])
+    c = O.lloyd_codebook(v, anchored=False)
+    assert np.array_equal(c, means.astype(np.float16))
+    a = O.lloyd_codebook(v, anchored=True)
+    assert a[0] == np.float16(v.min()) and a[15] == np.float16(v.max())
+    assert np.array_equal(a[1:15], means[1:15].astype(np.float16))
+
+
+def _distortion(v, c):
+    c = c.astype(np.float64)
+    return float(np.sum(np.min((v[:, None] - c[None, :]) ** 2, axis=1)))
+
+
+def test_lloyd_never_worse_than_uniform():
+    """Lloyd's rule starts at the uniform points and never raises the
+    quantisation distortion of the values (up to the fp16 rounding of the
+    points)."""
+    rng = np.random.default_rng(2)
+    for trial in range(5):
+        v = np.concatenate([rng.standard_normal(300) * 0.3, rng.standard_normal(40) * 2.0 + 3.0])
+        u = O.uniform_codebook(v)
+        for anchored in (False, True):
+            l = O.lloyd_codebook(v, anchored)
+            assert _distortion(v, l) <= _distortion(v, u) * (1 + 1e-3) + 1e-9, (trial, anchored)
+
+
+def _weights_with_spread_scales(out, inp, seed):
+    rng = np.random.default_rng(seed)
+    scale = np.exp(rng.standard_normal((out, 1)) * 1.5) * 0.02
+    scale[:3] *= 30
+    return (rng.standard_normal((out, inp)) * scale).astype(np.float16)
+
+
+def test_codebook_rule_choice_matches_brute_force():
+    """The nine combinations scored with scalar loops: per group the smallest
+    first term of Eq. (5) over the 256 pairs (digits of R8, Eq. (7)), summed
+    over the matrix; the oracle picks the same combination."""
+    W = _weights_with_spread_scales(6, 64, 5)
+    g, N = 16, 3
+    Vc, empty = O.clip_held_out(W, np.zeros_like(W, dtype=bool), g)
+    lo0, s0, flat = O.initial_pairs(Vc, g)
+    keep = ~(empty | flat)
+    ls, rl = np.log2(s0[keep]), lo0[keep] / s0[keep]
+    best, arg = None, None
+    for rs in ("uniform", "lloyd", "anchored"):
+        for rr in ("uniform", "lloyd", "anchored"):
+            cbs = [float(x) for x in O.codebook_by_rule(ls, rs)]
+            cbr = [float(x) for x in O.codebook_by_rule(rl, rr)]
+            total = 0.0
+            for r in range(W.shape[0]):
+                for g0 in range(0, W.shape[1], g):
+                    V = [float(x) for x in Vc[r, g0:g0 + g]]
+                    gb = None
+                    for p in range(256):
+                        s = 2.0 ** cbs[p >> 4]
+                        lo = cbr[p & 15] * s
+                        first = 0.0
+                        errs = [0.0] * (N - 1)
+                        for v in V:
+                            q = min(3, max(0, math.floor((v - lo) / s + 0.5)))
+                            rec = lo + s * q
+                            errs[0] += (v - rec) ** 2
+                            for k in range(3, N + 1):
+                                rec += s / 2 ** (k - 1) if v - rec >= 0 else -s / 2 ** (k - 1)
+                                errs[k - 2] += (v - rec) ** 2
+                        first = sum(errs) / (N - 1)
+                        gb = first if gb is None else min(gb, first)
+                    total += gb
+            if best is None or total < best * (1 - 1e-12):
+                best, arg = total, (rs, rr)
+    assert O.choose_codebook_rules(Vc, g, N, lo0, s0, empty | flat, empty) == arg
+
+
+def test_codebook_rules_keep_lloyd_or_fall_back():
+    """Spread group scales: a Lloyd rule wins and the deep-precision test keeps
+    it (its error is below a tenth of the two-bit error); with no planes the
+    deepest precision is two bits, so the matrix falls back to uniform."""
+    W = _weights_with_spread_scales(24, 256, 0)
+    A = O.encode(W, 32, 2, 0.0, "search", codebooks="appendix_e")
+    U = O.encode(W, 32, 2, 0.0, "search")
+    assert not np.array_equal(A.cb_log2s, U.cb_log2s)
+    Vc, empty = O.clip_held_out(W, np.zeros_like(W, dtype=bool), 32)
+    lo_t, s_t = O.pair_table(A.cb_log2s, A.cb_lo_over_s)
+    e2, e4 = O.precision_errors(Vc, 32, 4, A.pair_idx, lo_t, s_t, empty)
+    assert e4 <= 0.1 * e2
+    assert ((O.decode(A, 2) - W) ** 2).sum() < ((O.decode(U, 2) - W) ** 2).sum()
+    A0 = O.encode(W, 32, 0, 0.0, "fast", codebooks="appendix_e")
+    U0 = O.encode(W, 32, 0, 0.0, "fast")
+    assert np.array_equal(A0.cb_log2s, U0.cb_log2s) and np.array_equal(A0.cb_lo_over_s, U0.cb_lo_over_s)
