@@ -58,6 +58,12 @@ extern "C" {
 /* Pair search mode of the encoder (Section 3.1). */
 #define STAGQ_PAIR_SEARCH 0     /* argmin of Eq. (5) over all 256 codebook pairs */
 #define STAGQ_PAIR_FAST 1       /* nearest codebook entry per coordinate (labelled shortcut) */
+/* OR'ed into the pair mode: codebooks by Appendix E's rules -- of the nine
+ * combinations of uniform, Lloyd and anchored-Lloyd placement for the two
+ * codebooks, the one with the smallest summed first term of Eq. (5); uniform
+ * placement instead if, under it, the deepest precision's error exceeds a
+ * tenth of the two-bit error. Without it both codebooks are uniform. */
+#define STAGQ_CODEBOOK_RULES 0x100
 
 /* Flags of stagq_gemv_ex. */
 #define STAGQ_Y_F32 1u          /* y is fp32 instead of fp16 */

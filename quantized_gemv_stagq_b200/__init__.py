@@ -24,6 +24,7 @@ STAGQ_Y_F32 = 1
 STAGQ_KERNEL_GENERAL = 2
 STAGQ_KERNEL_SINGLE = 4
 STAGQ_SIDE_POST = 0x8000
+STAGQ_CODEBOOK_RULES = 0x100
 STAGQ_MAX_PLANES = 4
 STAGQ_MAX_BATCH = 4
 
@@ -184,11 +185,12 @@ def stagq_guard_capacity(out: int, inp: int, group: int) -> int:
 
 def stagq_encode(w: np.ndarray, group: int = 128, n_planes: int = 2, density: float = 0.005,
                  mode: str = "search", n_threads: int = 0, guard: str = "density", ratio_T: float = 4.0,
-                 post_guard: bool = True) -> Fields:
+                 post_guard: bool = True, codebooks: str = "uniform") -> Fields:
     """Encode an fp16 [out, inp] matrix (library encoder, host). guard
     "density": global top-|w| record of `density` (stagq_encode); "ratio": the
     pre-grid ratio guard with `ratio_T` and, if post_guard, the post-grid guard
-    (stagq_encode_guarded; post-grid columns carry STAGQ_SIDE_POST)."""
+    (stagq_encode_guarded; post-grid columns carry STAGQ_SIDE_POST). codebooks
+    "uniform" or "appendix_e" (STAGQ_CODEBOOK_RULES)."""
     w = np.ascontiguousarray(w, dtype=np.float16)
     out, inp = w.shape
     if guard == "density":
@@ -206,6 +208,10 @@ def stagq_encode(w: np.ndarray, group: int = 128, n_planes: int = 2, density: fl
                val=np.empty(nnz, np.uint16))
     cf = F._c()
     m = {"search": STAGQ_PAIR_SEARCH, "fast": STAGQ_PAIR_FAST}[mode]
+    if codebooks == "appendix_e":
+        m |= STAGQ_CODEBOOK_RULES
+    elif codebooks != "uniform":
+        raise ValueError("codebooks must be 'uniform' or 'appendix_e'")
     if guard == "density":
         _check(lib().stagq_encode(w.ctypes.data, density, m, n_threads, ctypes.byref(cf)), "stagq_encode")
     else:

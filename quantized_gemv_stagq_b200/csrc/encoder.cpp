@@ -11,8 +11,11 @@
 //      from the group's ends; groups with no retained entry or zero range
 //      stay out of the codebook fit (the latter are always searched, the
 //      former take pair 0 and zero digits);
-//   4. uniform fp16 codebooks over the initial pairs' log2(s) and lo/s
-//      (Appendix E);
+//   4. fp16 codebooks over the initial pairs' log2(s) and lo/s (Appendix
+//      E): uniform placement, or (STAGQ_CODEBOOK_RULES) the best of the nine
+//      combinations of uniform, Lloyd and anchored-Lloyd placement by the
+//      first term of Eq. 5, kept unless the deepest precision's error exceeds
+//      a tenth of the two-bit error;
 //   5. per-group pair: argmin of Eq. (5)-(6) with unit channel weights, or
 //      the labelled "fast" rule (nearest codebook entry per coordinate);
 //   6. base by nearest rounding (half up), 7. planes = sign of the residual
@@ -78,6 +81,120 @@ inline int digits(double w, double lo, double s, int N, uint8_t* bits, double* r
   return (int)qf;
 }
 
+// A codebook: fp64 values of its fp16 points, and the fp16 bits.
+struct Book {
+  double cb[16];
+  uint16_t h[16];
+};
+constexpr int kRuleUniform = 0, kRuleLloyd = 1, kRuleAnchored = 2;
+constexpr int kLloydMaxSteps = 100;        // Appendix E, Lloyd's rule: at most this many assignment steps
+constexpr double kFallbackRatio = 0.1;      // Appendix E: deepest-precision error vs two-bit error
+
+// Uniform placement (Appendix E): v_min + i (v_max - v_min) / 15; Lloyd's rule
+// from there (each point the mean of its nearest values, summed in index
+// order, ties to the lower point, empty points stay, at most 100 steps, until
+// no assignment changes); anchored: points 0 and 15 stay at the range ends.
+// No values: all zeros.
+Book codebook_by_rule(const std::vector<double>& v, int rule) {
+  Book b{};
+  if (v.empty()) return b;
+  double vmin = INFINITY, vmax = -INFINITY;
+  for (double x : v) { vmin = std::min(vmin, x); vmax = std::max(vmax, x); }
+  double c[16];
+  for (int i = 0; i < 16; ++i) c[i] = vmin + (double)i * (vmax - vmin) / 15.0;
+  if (rule != kRuleUniform) {
+    std::vector<int> assign(v.size(), -1), a(v.size());
+    for (int step = 0; step < kLloydMaxSteps; ++step) {
+      for (size_t j = 0; j < v.size(); ++j) {
+        int bi = 0;
+        for (int i = 1; i < 16; ++i)
+          if (std::fabs(v[j] - c[i]) < std::fabs(v[j] - c[bi])) bi = i;
+        a[j] = bi;
+      }
+      if (step > 0 && a == assign) break;
+      assign = a;
+      for (int i = 0; i < 16; ++i) {
+        if (rule == kRuleAnchored && (i == 0 || i == 15)) continue;
+        double sm = 0.0;
+        int64_t n = 0;
+        for (size_t j = 0; j < v.size(); ++j)
+          if (a[j] == i) { sm = sm + v[j]; ++n; }
+        if (n) c[i] = sm / (double)n;
+      }
+    }
+  }
+  for (int i = 0; i < 16; ++i) {
+    b.h[i] = double_to_half(c[i]);
+    b.cb[i] = half_to_double(b.h[i]);
+  }
+  return b;
+}
+
+// The 256 (lo, s) of a codebook pair (Section 3.1), fp64 from the fp16 points.
+struct PairTable {
+  double lo[256], s[256], cbs[16], cbr[16];
+};
+PairTable make_pair_table(const Book& bs, const Book& br) {
+  PairTable T;
+  for (int i = 0; i < 16; ++i) { T.cbs[i] = bs.cb[i]; T.cbr[i] = br.cb[i]; }
+  for (int p = 0; p < 256; ++p) {
+    T.s[p] = std::exp2(T.cbs[p >> 4]);
+    T.lo[p] = T.cbr[p & 15] * T.s[p];
+  }
+  return T;
+}
+
+// Eq. (5)-(6) of one group under (lo, s): (first term / (N-1), floor term sum).
+std::pair<double, double> pair_terms(const double* V, int64_t g, int N, double lo, double s, double reach_sum,
+                                     double* rec) {
+  double recon_one[8];
+  for (int64_t c = 0; c < g; ++c) {
+    digits(V[c], lo, s, N, nullptr, recon_one);
+    for (int M = 2; M <= N; ++M) rec[(size_t)(M - 2) * g + c] = recon_one[M - 2];
+  }
+  double first = 0.0;
+  for (int M = 2; M <= N; ++M) {
+    double sm = 0.0;
+    for (int64_t c = 0; c < g; ++c) {
+      const double e = V[c] - rec[(size_t)(M - 2) * g + c];
+      sm = sm + e * e;
+    }
+    first = first + sm;
+  }
+  first = first / (double)(N - 1);
+  const double rho = s * reach_sum;
+  double fl = 0.0;
+  for (int64_t c = 0; c < g; ++c) {
+    double e = std::fabs(V[c] - rec[c]) - rho;
+    e = e > 0.0 ? e : 0.0;
+    fl = fl + e * e;
+  }
+  return {first, fl};
+}
+
+// Pair of one (non-empty) group: the Eq. (5) argmin (ties to the smaller
+// index), or the labelled fast rule for groups with a nonzero range.
+int choose_pair(const double* V, int64_t g, int N, const PairTable& T, int pair_mode, bool flat, double lo0, double s0,
+                double reach_sum, double* rec) {
+  if (pair_mode == STAGQ_PAIR_FAST && !flat) {
+    const double L = std::log2(s0), r = lo0 / s0;
+    int ba = 0, bb = 0;
+    for (int i = 1; i < 16; ++i) {
+      if (std::fabs(T.cbs[i] - L) < std::fabs(T.cbs[ba] - L)) ba = i;
+      if (std::fabs(T.cbr[i] - r) < std::fabs(T.cbr[bb] - r)) bb = i;
+    }
+    return ba * 16 + bb;
+  }
+  double best = INFINITY;
+  int pair = 0;
+  for (int p = 0; p < 256; ++p) {
+    const std::pair<double, double> t = pair_terms(V, g, N, T.lo[p], T.s[p], reach_sum, rec);
+    const double D = t.first + kFloorLambda * t.second;
+    if (D < best) { best = D; pair = p; }
+  }
+  return pair;
+}
+
 }  // namespace
 }  // namespace stagq
 
@@ -101,7 +218,8 @@ int check_encode_args(const uint16_t* w, stagq_fields* f, int32_t pair_mode, con
   if (in > STAGQ_MAX_IN) return fail(STAGQ_EINVAL, std::string(who) + ": in exceeds STAGQ_MAX_IN");
   if (f->n_planes < 0 || f->n_planes > STAGQ_MAX_PLANES)
     return fail(STAGQ_EINVAL, std::string(who) + ": n_planes out of range");
-  if (pair_mode != STAGQ_PAIR_SEARCH && pair_mode != STAGQ_PAIR_FAST)
+  const int32_t pm = pair_mode & ~(int32_t)STAGQ_CODEBOOK_RULES;
+  if (pm != STAGQ_PAIR_SEARCH && pm != STAGQ_PAIR_FAST)
     return fail(STAGQ_EINVAL, std::string(who) + ": unknown pair mode");
   if (!f->q || (f->n_planes && !f->planes) || !f->pair_idx || !f->row_ptr)
     return fail(STAGQ_EINVAL, std::string(who) + ": null field buffer");
@@ -180,8 +298,10 @@ extern "C" int stagq_encode(const uint16_t* w, double density, int32_t pair_mode
 
 namespace {
 
-int encode_with(const uint16_t* w, const std::vector<uint8_t>& held, bool post_guard, int32_t pair_mode,
+int encode_with(const uint16_t* w, const std::vector<uint8_t>& held, bool post_guard, int32_t pair_mode_flags,
                 int32_t n_threads, int64_t cap, stagq_fields* f) {
+  const bool codebook_rules = (pair_mode_flags & STAGQ_CODEBOOK_RULES) != 0;
+  const int32_t pair_mode = pair_mode_flags & ~(int32_t)STAGQ_CODEBOOK_RULES;
   const int64_t out = f->out, in = f->in, g = f->group;
   const int n_planes = f->n_planes;
   const int N = 2 + n_planes;
@@ -213,32 +333,86 @@ int encode_with(const uint16_t* w, const std::vector<uint8_t>& held, bool post_g
     }
   });
 
-  // 4. uniform codebooks over the groups with retained entries and a nonzero range.
-  double lmin = INFINITY, lmax = -INFINITY, rmin = INFINITY, rmax = -INFINITY;
-  bool any_group = false;
-  for (int64_t G = 0; G < ngroups; ++G) {
-    if (empty[G] || flat[G]) continue;
-    const double L = std::log2(s0[G]);
-    const double r = lo0[G] / s0[G];
-    lmin = std::min(lmin, L); lmax = std::max(lmax, L);
-    rmin = std::min(rmin, r); rmax = std::max(rmax, r);
-    any_group = true;
-  }
-  for (int i = 0; i < 16; ++i) {
-    f->codebook_log2s[i] = any_group ? double_to_half(lmin + (double)i * (lmax - lmin) / 15.0) : 0;
-    f->codebook_lo_over_s[i] = any_group ? double_to_half(rmin + (double)i * (rmax - rmin) / 15.0) : 0;
-  }
-  double cbs[16], cbr[16], tab_lo[256], tab_s[256];
-  for (int i = 0; i < 16; ++i) {
-    cbs[i] = half_to_double(f->codebook_log2s[i]);
-    cbr[i] = half_to_double(f->codebook_lo_over_s[i]);
-  }
-  for (int p = 0; p < 256; ++p) {
-    tab_s[p] = std::exp2(cbs[p >> 4]);
-    tab_lo[p] = cbr[p & 15] * tab_s[p];
-  }
+  // clipped group values for the pair fit
+  auto clipped = [&](int64_t G, double* V) {
+    const int64_t base = (G / ng) * in + (G % ng) * g;
+    double mx = -INFINITY, mn = INFINITY;
+    for (int64_t c = 0; c < g; ++c)
+      if (!held[base + c]) { const double v = half_to_double(w[base + c]); mx = std::max(mx, v); mn = std::min(mn, v); }
+    for (int64_t c = 0; c < g; ++c) {
+      const double v = half_to_double(w[base + c]);
+      V[c] = held[base + c] ? (v >= 0.0 ? mx : mn) : v;
+    }
+  };
   double reach_sum = 0.0;
   for (int k = 3; k <= N; ++k) reach_sum += std::ldexp(1.0, -(k - 1));
+
+  // 4. codebooks over the initial pairs of the groups with retained entries
+  // and a nonzero range (group order): uniform placement, or with
+  // STAGQ_CODEBOOK_RULES Appendix E's choice among uniform, Lloyd and
+  // anchored-Lloyd placement for each codebook and its fallback.
+  std::vector<double> vls, vrl;
+  for (int64_t G = 0; G < ngroups; ++G) {
+    if (empty[G] || flat[G]) continue;
+    vls.push_back(std::log2(s0[G]));
+    vrl.push_back(lo0[G] / s0[G]);
+  }
+  Book chosen_s = codebook_by_rule(vls, kRuleUniform), chosen_r = codebook_by_rule(vrl, kRuleUniform);
+  if (codebook_rules) {
+    Book bs[3], br[3];
+    for (int r = 0; r < 3; ++r) { bs[r] = codebook_by_rule(vls, r); br[r] = codebook_by_rule(vrl, r); }
+    std::vector<double> gmin(ngroups);
+    double best = INFINITY;
+    int best_s = 0, best_r = 0;
+    for (int rs = 0; rs < 3; ++rs) {
+      for (int rr = 0; rr < 3; ++rr) {
+        const PairTable T = make_pair_table(bs[rs], br[rr]);
+        parallel_for(ngroups, n_threads, [&](int64_t a, int64_t b) {
+          std::vector<double> V(g), rec((size_t)g * (N - 1));
+          for (int64_t G = a; G < b; ++G) {
+            if (empty[G]) { gmin[G] = 0.0; continue; }
+            clipped(G, V.data());
+            double m = INFINITY;
+            for (int p = 0; p < 256; ++p) m = std::min(m, pair_terms(V.data(), g, N, T.lo[p], T.s[p], reach_sum, rec.data()).first);
+            gmin[G] = m;
+          }
+        });
+        double tot = 0.0;
+        for (int64_t G = 0; G < ngroups; ++G) tot = tot + gmin[G];
+        if (tot < best) { best = tot; best_s = rs; best_r = rr; }
+      }
+    }
+    // fallback: the deepest precision's error against the two-bit error under
+    // the chosen codebooks and the final pair choice
+    const PairTable T = make_pair_table(bs[best_s], br[best_r]);
+    std::vector<double> e2g(ngroups, 0.0), eNg(ngroups, 0.0);
+    parallel_for(ngroups, n_threads, [&](int64_t a, int64_t b) {
+      std::vector<double> V(g), rec((size_t)g * (N - 1));
+      double recon_one[8];
+      for (int64_t G = a; G < b; ++G) {
+        if (empty[G]) continue;
+        clipped(G, V.data());
+        const int pair = choose_pair(V.data(), g, N, T, pair_mode, flat[G], lo0[G], s0[G], reach_sum, rec.data());
+        double e2 = 0.0, eN = 0.0;
+        for (int64_t c = 0; c < g; ++c) {
+          digits(V[c], T.lo[pair], T.s[pair], N, nullptr, recon_one);
+          const double d2 = V[c] - recon_one[0], dN = V[c] - recon_one[N - 2];
+          e2 = e2 + d2 * d2;
+          eN = eN + dN * dN;
+        }
+        e2g[G] = e2;
+        eNg[G] = eN;
+      }
+    });
+    double e2 = 0.0, eN = 0.0;
+    for (int64_t G = 0; G < ngroups; ++G) { e2 = e2 + e2g[G]; eN = eN + eNg[G]; }
+    if (!(eN > kFallbackRatio * e2)) { chosen_s = bs[best_s]; chosen_r = br[best_r]; }
+  }
+  for (int i = 0; i < 16; ++i) {
+    f->codebook_log2s[i] = chosen_s.h[i];
+    f->codebook_lo_over_s[i] = chosen_r.h[i];
+  }
+  const PairTable T = make_pair_table(chosen_s, chosen_r);
 
   // 5-7. pair per group, then the digits.
   parallel_for(ngroups, n_threads, [&](int64_t a, int64_t b) {
@@ -249,54 +423,11 @@ int encode_with(const uint16_t* w, const std::vector<uint8_t>& held, bool post_g
       const int64_t row = G / ng, base = row * in + (G % ng) * g;
       int pair = 0;
       if (!empty[G]) {
-        // clipped group values
-        double mx = -INFINITY, mn = INFINITY;
-        for (int64_t c = 0; c < g; ++c)
-          if (!held[base + c]) { const double v = half_to_double(w[base + c]); mx = std::max(mx, v); mn = std::min(mn, v); }
-        for (int64_t c = 0; c < g; ++c) {
-          const double v = half_to_double(w[base + c]);
-          V[c] = held[base + c] ? (v >= 0.0 ? mx : mn) : v;
-        }
-        if (pair_mode == STAGQ_PAIR_FAST && !flat[G]) {
-          const double L = std::log2(s0[G]), r = lo0[G] / s0[G];
-          int ba = 0, bb = 0;
-          for (int i = 1; i < 16; ++i) {
-            if (std::fabs(cbs[i] - L) < std::fabs(cbs[ba] - L)) ba = i;
-            if (std::fabs(cbr[i] - r) < std::fabs(cbr[bb] - r)) bb = i;
-          }
-          pair = ba * 16 + bb;
-        } else {
-          double best = INFINITY;
-          for (int p = 0; p < 256; ++p) {
-            const double lo = tab_lo[p], s = tab_s[p];
-            for (int64_t c = 0; c < g; ++c) {
-              digits(V[c], lo, s, N, nullptr, recon_one);
-              for (int M = 2; M <= N; ++M) rec[(size_t)(M - 2) * g + c] = recon_one[M - 2];
-            }
-            double first = 0.0;
-            for (int M = 2; M <= N; ++M) {
-              double sm = 0.0;
-              for (int64_t c = 0; c < g; ++c) {
-                const double e = V[c] - rec[(size_t)(M - 2) * g + c];
-                sm = sm + e * e;
-              }
-              first = first + sm;
-            }
-            first = first / (double)(N - 1);
-            const double rho = s * reach_sum;
-            double fl = 0.0;
-            for (int64_t c = 0; c < g; ++c) {
-              double e = std::fabs(V[c] - rec[c]) - rho;
-              e = e > 0.0 ? e : 0.0;
-              fl = fl + e * e;
-            }
-            const double D = first + kFloorLambda * fl;
-            if (D < best) { best = D; pair = p; }
-          }
-        }
+        clipped(G, V.data());
+        pair = choose_pair(V.data(), g, N, T, pair_mode, flat[G], lo0[G], s0[G], reach_sum, rec.data());
       }
       f->pair_idx[G] = (uint8_t)pair;
-      const double lo = tab_lo[pair], s = tab_s[pair];
+      const double lo = T.lo[pair], s = T.s[pair];
       for (int64_t c = 0; c < g; ++c) {
         const int64_t idx = base + c;
         if (held[idx]) {
@@ -324,7 +455,7 @@ int encode_with(const uint16_t* w, const std::vector<uint8_t>& held, bool post_g
           const int64_t idx = r * in + c;
           if (held[idx]) continue;
           const int p = f->pair_idx[r * ng + c / g];
-          const double r2 = tab_lo[p] + tab_s[p] * (double)f->q[idx];
+          const double r2 = T.lo[p] + T.s[p] * (double)f->q[idx];
           const double d = half_to_double(w[idx]) - r2;
           const double e = d * d;
           if (e > best) { best = e; bc = c; best_r2 = r2; }

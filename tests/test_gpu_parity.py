@@ -309,3 +309,23 @@ def test_full_size_guarded_sampled_rows(name, shape, group):
     out, inp = shape
     _sampled_rows_case(out, inp, group, 2, 0.0, 4000 + out + group, (2, 3, 4), _kernels(), batch4=True,
                        guard="ratio", ratio_T=4.0)
+
+
+def test_appendix_e_codebooks_gemv_matches_oracle():
+    """Lloyd-placed codebooks (Appendix E's rules win on groups of widely
+    spread scales) through both n = 1 kernels and n = 4."""
+    from tests.test_oracle_pins import _weights_with_spread_scales
+    W = _weights_with_spread_scales(64, 1024, 9)
+    F = O.encode(W, 32, 2, 0.005, "fast", codebooks="appendix_e")
+    assert not np.array_equal(F.cb_log2s, O.encode(W, 32, 2, 0.005, "fast").cb_log2s)
+    m = _load(F)
+    x = synth.activations(4, 1024, 10)
+    for M in (2, 3, 4):
+        ref = O.gemv(F, M, x)
+        for kern in (Q.STAGQ_KERNEL_GENERAL, Q.STAGQ_KERNEL_SINGLE):
+            check_close(_gemv(m, M, x[:1], kernel=kern)[0], ref[0], f"p{M} kernel {kern}")
+        got = _gemv(m, M, x)
+        for j in range(4):
+            check_close(got[j], ref[j], f"p{M} n4 col{j}")
+    Q.stagq_check(m)
+    m.free()

@@ -65,6 +65,25 @@ def test_guarded_encoder_matches_oracle_bit_exactly(out, inp, g, npl, T, post, m
     assert ((P.col & Q.STAGQ_SIDE_POST) != 0).sum() == F.post_flags.sum()
 
 
+@pytest.mark.parametrize("out,inp,g,npl,mode,dens", [
+    (24, 256, 32, 2, "search", 0.0),
+    (24, 256, 32, 3, "fast", 0.01),
+    (16, 512, 64, 0, "fast", 0.0),       # no planes: the fallback keeps uniform placement
+    (40, 384, 16, 2, "search", 0.02),
+])
+def test_codebook_rules_encoder_matches_oracle_bit_exactly(out, inp, g, npl, mode, dens):
+    """Appendix E's codebook rules (Lloyd / anchored Lloyd / uniform, the
+    nine-combination choice, the fallback): every field bit for bit."""
+    from tests.test_oracle_pins import _weights_with_spread_scales
+    W = _weights_with_spread_scales(out, inp, out + g)
+    F = O.encode(W, g, npl, dens, mode, codebooks="appendix_e")
+    P = Q.stagq_encode(W, g, npl, dens, mode, codebooks="appendix_e", n_threads=3)
+    eq = fields_equal(F, P)
+    assert all(eq.values()), eq
+    U = O.encode(W, g, npl, dens, mode)
+    assert np.array_equal(F.cb_log2s, U.cb_log2s) == (npl == 0)
+
+
 def test_guarded_stream_packs_and_rereads():
     W = synth.weights(24, 640, seed=7)
     F = O.encode(W, group=32, n_planes=2, mode="fast", guard="ratio", ratio_T=4.0)
