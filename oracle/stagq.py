@@ -663,10 +663,17 @@ def decode(F: Fields, M: int, rows=None) -> np.ndarray:
     return np.where(m, 0.0, main) + P
 
 
-def gemv(F: Fields, M: int, x: np.ndarray, rows=None) -> np.ndarray:
+def gemv(F: Fields, M: int, x: np.ndarray, rows=None, in_scale=None) -> np.ndarray:
     """y = W_hat^(M) x in fp64 for x [n, inp] (fp16 values taken exactly);
-    returns [n, len(rows)] (all rows by default)."""
+    returns [n, len(rows)] (all rows by default).
+
+    ``in_scale`` [inp] (fp32 values taken exactly): the run-time inverse
+    activation scale of Section 4 / Appendix E -- the quantizer saw W diag(a),
+    so the decoder multiplies channel c of x by 1/a_c (given here) before the
+    product: y = W_hat (x * in_scale)."""
     x = np.atleast_2d(np.asarray(x)).astype(np.float64)
+    if in_scale is not None:
+        x = x * np.asarray(in_scale, dtype=np.float64)[None, :]
     What = decode(F, M, rows)
     return x @ What.T
 

@@ -553,3 +553,23 @@ def test_codebook_rules_keep_lloyd_or_fall_back():
     A0 = O.encode(W, 32, 0, 0.0, "fast", codebooks="appendix_e")
     U0 = O.encode(W, 32, 0, 0.0, "fast")
     assert np.array_equal(A0.cb_log2s, U0.cb_log2s) and np.array_equal(A0.cb_lo_over_s, U0.cb_lo_over_s)
+
+
+# ------------------------------------- run-time inverse activation scale
+
+def test_input_scale_is_a_column_scaling_of_w_hat():
+    """y = W_hat (x * s) equals (W_hat diag(s)) x, and power-of-two scales
+    equal the GEMV of the scaled x exactly; all-ones is the plain GEMV."""
+    W = synth.weights(12, 256, seed=41)
+    F = O.encode(W, group=64, n_planes=2, density=0.01, mode="fast")
+    x = synth.activations(2, 256, seed=42)
+    rng = np.random.default_rng(43)
+    s = rng.uniform(0.25, 4.0, 256).astype(np.float32)
+    p2 = (2.0 ** rng.integers(-3, 4, 256)).astype(np.float32)
+    for M in (2, 3, 4):
+        D = O.decode(F, M)
+        assert np.allclose(O.gemv(F, M, x, in_scale=s), x.astype(np.float64) @ (D * s.astype(np.float64)[None, :]).T,
+                           rtol=1e-12, atol=1e-13)
+        xs = (x.astype(np.float64) * p2.astype(np.float64)).astype(np.float64)
+        assert np.array_equal(O.gemv(F, M, x, in_scale=p2), xs @ D.T)
+        assert np.array_equal(O.gemv(F, M, x, in_scale=np.ones(256, np.float32)), O.gemv(F, M, x))
