@@ -13,13 +13,17 @@ device time, in GB/s. Per-GEMV microseconds for every shape and precision are
 in ``per_gemv``.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl stagq|reference]
-                  [--workload llama31_8b_linears_b1 | phi4_olmo2_linears_b1 | precision_sweep | llama31_8b_stack]
+                  [--workload llama31_8b_linears_b1 | phi4_olmo2_linears_b1 | precision_sweep |
+                              llama31_8b_stack | llama31_8b_guarded]
 
 The default workload is the Llama-3.1-8B layer above. The others print one
 JSON line each with per-GEMV (or per-token) times:
   phi4_olmo2_linears_b1  Phi-4 and OLMo-2-7B linears at 2/3/4 bits, batch 1,
                          each alone and as one layer's chain (q k v o gate up
                          down, one CUDA graph);
+  llama31_8b_guarded     the Llama-3.1-8B linears at group 32 with the paper's
+                         side-record guards (ratio T = 4 + post-grid), each
+                         alone and as a layer chain;
   precision_sweep        14336x4096 and 4096x14336 with base + 4 planes, read at
                          2..6 bits, group 16, 32, 64 and 128, side record
                          0 / 0.1 / 1 %;
@@ -62,7 +66,8 @@ def _args():
     p.add_argument("--copies", type=int, default=6, help="device copies of the layer rotated over")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--workload", default=WORKLOAD,
-                   choices=[WORKLOAD, "phi4_olmo2_linears_b1", "precision_sweep", "llama31_8b_stack"])
+                   choices=[WORKLOAD, "phi4_olmo2_linears_b1", "precision_sweep", "llama31_8b_stack",
+                            "llama31_8b_guarded"])
     p.add_argument("--stack-distinct", type=int, default=4,
                    help="llama31_8b_stack: distinct encoded layers (the 32 resident layers cycle over them)")
     return p.parse_args()
@@ -291,11 +296,11 @@ def run_extra(args):
     results = {}
     launches = 0
 
-    def per_gemv(shapes, bits_list, group, n_planes, density, batch=1, tag=""):
+    def per_gemv(shapes, bits_list, group, n_planes, density, batch=1, tag="", **enc):
         nonlocal launches
         for name, (out, inp) in shapes:
             S = Q.stagq_pack(Q.stagq_encode(synth.weights(out, inp, seed=out + 3 * inp), group, n_planes,
-                                            density, "fast"))
+                                            density, "fast", **enc))
             m0 = Q.stagq_load(S, 0)
             C = copies_for(Q, m0.device_bytes, l2)
             mats = [m0] + [Q.stagq_load(S, 0) for _ in range(C - 1)]
@@ -312,19 +317,19 @@ def run_extra(args):
                 m.free()
             del S
 
-    def layer_chain(model, linears, bits_list, group, n_planes, density):
+    def layer_chain(model, linears, bits_list, group, n_planes, density, **enc):
         """One layer's linears in order as one CUDA graph (the chain a decode
         step runs), rotating over enough device copies that reads come from
         HBM; µs per layer."""
         nonlocal launches
-        enc = {}
+        streams = {}
         for _, (out, inp) in linears:
-            if (out, inp) not in enc:
-                enc[(out, inp)] = Q.stagq_pack(Q.stagq_encode(synth.weights(out, inp, seed=out + 3 * inp), group,
-                                                              n_planes, density, "fast"))
-        first = [Q.stagq_load(enc[v], 0) for _, v in linears]
+            if (out, inp) not in streams:
+                streams[(out, inp)] = Q.stagq_pack(Q.stagq_encode(synth.weights(out, inp, seed=out + 3 * inp),
+                                                                  group, n_planes, density, "fast", **enc))
+        first = [Q.stagq_load(streams[v], 0) for _, v in linears]
         C = copies_for(Q, sum(m.device_bytes for m in first), l2, minimum=2)
-        mats = [first] + [[Q.stagq_load(enc[v], 0) for _, v in linears] for _ in range(C - 1)]
+        mats = [first] + [[Q.stagq_load(streams[v], 0) for _, v in linears] for _ in range(C - 1)]
         xs = {inp: torch.from_numpy(synth.activations(1, inp, seed=inp)).cuda() for _, (_, inp) in linears}
         ys = [torch.empty(1, out, dtype=torch.float16, device="cuda") for _, (out, _) in linears]
         for b in bits_list:
@@ -374,6 +379,20 @@ def run_extra(args):
                     BITS, GROUP, N_PLANES, DENSITY)
         cfg = {"linears_out_x_in": {k: list(v) for k, v in shapes}, "bits": list(BITS), "group": GROUP,
                "n_planes": N_PLANES, "side_record_density": DENSITY, "batch": 1}
+    elif args.workload == "llama31_8b_guarded":
+        # The paper's guards on every linear (pre-grid ratio criterion T = 4 and
+        # the post-grid per-row guard, Table 6 / Appendix E) at its kernel
+        # evaluation's group size 32 (Section 4.3).
+        shapes = _layer_shapes()
+        guard = dict(guard="ratio", ratio_T=4.0, post_guard=True)
+        per_gemv(shapes, BITS, 32, N_PLANES, 0.0, **guard)
+        L = synth.LLAMA31_8B_LINEARS
+        layer_chain("llama31_8b_g32_guarded", [(k, L[k]) for k in ("q_proj", "k_proj", "v_proj", "o_proj",
+                                                                    "gate_proj", "up_proj", "down_proj")],
+                    BITS, 32, N_PLANES, 0.0, **guard)
+        cfg = {"linears_out_x_in": {k: list(v) for k, v in shapes}, "bits": list(BITS), "group": 32,
+               "n_planes": N_PLANES, "side_record": "pre-grid ratio guard T = 4 + post-grid guard (1 per row)",
+               "batch": 1}
     elif args.workload == "precision_sweep":
         shapes = [("gate", (14336, 4096)), ("down", (4096, 14336))]
         for g in (16, 32, 64, 128):
