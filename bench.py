@@ -266,6 +266,24 @@ def time_gemv(Q, torch, mats, bits, x, y, n, stream, reps=24, repeats=5):
     return statistics.median(out)
 
 
+def job_ms(ms: float, dist=None, device: str = "cuda") -> float:
+    """The job's device time: the max over ranks of each replica's CUDA-event
+    time (ms), taken by an all-reduce on `device` (a GPU tensor for NCCL, the
+    CPU for gloo); the local time without a process group."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, step_bytes: int, steps: int, ms: float) -> float:
+    """Whole-job throughput in GB/s: every replica moves step_bytes per step
+    (weak scaling), over the job's time."""
+    return world * step_bytes * steps / (ms * 1e-3) / 1e9
+
+
 def copies_for(Q, stored_bytes, l2, minimum=3):
     """Device copies so that one pass over them is at least 4x the L2 size."""
     return max(minimum, int(4 * l2 // max(stored_bytes, 1)) + 1)
@@ -553,9 +571,7 @@ def run_stagq(args):
     clk = clocks.stop()
 
     if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = job_ms(ms, dist, "cuda")
         dist.barrier()
 
     # ---- end to end through the C ABI with host buffers
@@ -582,7 +598,7 @@ def run_stagq(args):
         return
 
     peak, peak_kind = _peaks()
-    value = world * step_bytes * args.steps / (ms * 1e-3) / 1e9
+    value = job_value(world, step_bytes, args.steps, ms)
     # dominant kernel: the (shape, precision) with the largest share of a step
     dom_key, dom = max(((f"{name}@{pb}", d) for pb, dd in per.items() for name, d in dd.items()),
                        key=lambda kv: kv[1]["us"])
