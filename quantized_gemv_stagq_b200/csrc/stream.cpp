@@ -1,5 +1,7 @@
 // Plane-major packer, host re-read of packed levels, stream validation and
 // the on-disk stream file (host only).
+#include <sys/types.h>
+
 #include <cstdio>
 #include <cstring>
 #include <string>
@@ -178,6 +180,13 @@ int read_stream_file(const char* path, HostStreamBuffers* buf) {
   }
   const int64_t pb = stagq_stream_plane_bytes(h.out, h.in, h.n_planes);
   const int64_t ngr = (int64_t)h.out * (h.in / h.group);
+  // The file must hold exactly what its header declares: checked before any
+  // allocation, so a corrupt or hostile header cannot ask for terabytes.
+  const int64_t expect = (int64_t)sizeof h + pb + ngr + 4 * ((int64_t)h.out + 1) + 4 * h.nnz;
+  if (fseeko(fp, 0, SEEK_END) != 0 || ftello(fp) != (off_t)expect || fseeko(fp, (off_t)sizeof h, SEEK_SET) != 0) {
+    std::fclose(fp);
+    return fail(STAGQ_EFORMAT, "stream file size does not match its header");
+  }
   try {
     buf->planes.resize(pb);
     buf->pair_idx.resize(ngr);

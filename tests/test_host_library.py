@@ -179,3 +179,43 @@ def test_stream_file_header(tmp_path):
     raw = open(p, "rb").read()
     assert raw[:8] == b"STAGQS1\0"
     assert len(raw) == 8 + 4 * 4 + 8 + 64 + S.planes.size + S.pair_idx.size + 4 * (S.out + 1) + 4 * S.nnz
+
+
+def test_load_file_rejects_bad_files_before_any_allocation(tmp_path):
+    """Host-side failures of the file loader return status codes, before any
+    device work: a missing file, a wrong magic, a truncated file, a header that
+    declares more than the file holds (a hostile header asking for terabytes is
+    refused by size, not by an allocation attempt), a null path."""
+    S = _stream()
+    good = str(tmp_path / "good.stagq")
+    Q.stagq_save(S, good)
+    raw = open(good, "rb").read()
+    cases = {
+        "missing": (str(tmp_path / "nope.stagq"), None, 5),
+        "magic": (str(tmp_path / "magic.stagq"), b"NOTSTAGQ" + raw[8:], 2),
+        "truncated": (str(tmp_path / "trunc.stagq"), raw[:-7], 2),
+        "trailing": (str(tmp_path / "long.stagq"), raw + b"\0" * 16, 2),
+    }
+    import struct
+    huge = bytearray(raw)
+    struct.pack_into("<iiii", huge, 8, 1 << 30, 32768, 128, 4)   # 2^30 x 32768 at 6 bits: ~24 TB of planes
+    cases["huge"] = (str(tmp_path / "huge.stagq"), bytes(huge), 2)
+    for name, (path, data, status) in cases.items():
+        if data is not None:
+            open(path, "wb").write(data)
+        with pytest.raises(Q.StagqError) as e:
+            Q.stagq_load_file(path, 0)
+        assert e.value.status == status, (name, e.value.status)
+    assert Q.lib().stagq_load_file(None, 0, None) == 1
+    # the intact file passes every host check; what remains is the device
+    try:
+        import torch
+        has_gpu = torch.cuda.is_available()
+    except Exception:
+        has_gpu = False
+    if has_gpu:
+        Q.stagq_load_file(good, 0).free()
+    else:
+        with pytest.raises(Q.StagqError) as e:
+            Q.stagq_load_file(good, 0)
+        assert e.value.status in (4, 6), e.value.status   # STAGQ_ECUDA / STAGQ_ENODEV: the device step
