@@ -1,5 +1,6 @@
 """Host side of libstagq.so (CPU only): exported symbols, encoder and packer
 against the oracle, the byte-scaling property of the layout, error paths."""
+import ctypes
 import os
 import re
 
@@ -219,3 +220,36 @@ def test_load_file_rejects_bad_files_before_any_allocation(tmp_path):
         with pytest.raises(Q.StagqError) as e:
             Q.stagq_load_file(good, 0)
         assert e.value.status in (4, 6), e.value.status   # STAGQ_ECUDA / STAGQ_ENODEV: the device step
+
+
+def test_encoder_output_does_not_depend_on_thread_count():
+    """Every floating-point step runs in a fixed order inside one group or
+    row, so 1 and 7 encoder threads give the same fields, in every mode."""
+    from tests.test_oracle_pins import _weights_with_spread_scales
+    W = _weights_with_spread_scales(40, 512, 77)
+    for kw in (dict(density=0.01, mode="search"),
+               dict(density=0.0, mode="fast", guard="ratio", ratio_T=4.0),
+               dict(density=0.0, mode="search", codebooks="appendix_e")):
+        a = Q.stagq_encode(W, group=32, n_planes=3, n_threads=1, **kw)
+        b = Q.stagq_encode(W, group=32, n_planes=3, n_threads=7, **kw)
+        for k in ("q", "planes", "pair_idx", "cb_log2s", "cb_lo_over_s", "row_ptr", "col", "val"):
+            assert np.array_equal(getattr(a, k), getattr(b, k)), (kw, k)
+
+
+def test_guarded_encoder_error_paths():
+    W = synth.weights(8, 256, seed=3)
+    with pytest.raises(Q.StagqError) as e:            # T below 1
+        Q.stagq_encode(W, group=64, n_planes=2, mode="fast", guard="ratio", ratio_T=0.5)
+    assert e.value.status == 1
+    with pytest.raises(Q.StagqError) as e:            # unknown pair-mode bits
+        F = Q.Fields(8, 256, 64, 2, q=np.empty((8, 256), np.uint8), planes=np.empty((2, 8, 256), np.uint8),
+                     pair_idx=np.empty((8, 4), np.uint8), cb_log2s=np.zeros(16, np.uint16),
+                     cb_lo_over_s=np.zeros(16, np.uint16), row_ptr=np.empty(9, np.int32),
+                     col=np.empty(Q.stagq_guard_capacity(8, 256, 64) - 1, np.uint16),
+                     val=np.empty(Q.stagq_guard_capacity(8, 256, 64) - 1, np.uint16))
+        cf = F._c()
+        st = Q.lib().stagq_encode_guarded(np.ascontiguousarray(W).ctypes.data, 4.0, 1, Q.STAGQ_PAIR_FAST, 1, ctypes.byref(cf))
+        if st:
+            raise Q.StagqError(st, "capacity")
+    assert e.value.status == 1                        # capacity one short of stagq_guard_capacity
+    assert Q.stagq_guard_capacity(8, 256, 64) == 8 * 4 + 8
