@@ -162,16 +162,18 @@ int stagq_encode_guarded(const uint16_t* w, double ratio_T, int32_t post_guard, 
 /*
  * Encoder of Sections 3.1-3.6 / Appendices B, E for a synthetic fp16 matrix
  * (host, multithreaded): global top-|w| side record with `density`, held-out
- * entries clipped inward for the fit, initial pair (Appendix B), uniform fp16
- * codebooks (Appendix E), pair per group by `pair_mode`, nearest-rounding
- * base, sign planes (Eq. 7), zero digits at held-out positions.
+ * entries clipped inward for the fit, initial pair (Appendix B), fp16
+ * codebooks (Appendix E: uniform placement, or Appendix E's rules with
+ * STAGQ_CODEBOOK_RULES OR'ed into `pair_mode`), pair per group by `pair_mode`
+ * (STAGQ_PAIR_SEARCH / STAGQ_PAIR_FAST), nearest-rounding base, sign planes
+ * (Eq. 7), zero digits at held-out positions.
  *   w        host [out*in] fp16 bits, row-major
  *   f        caller sets out, in, group, n_planes and points every array at a
  *            buffer of the documented size, with nnz = stagq_side_record_count(...);
  *            the encoder fills codebooks and arrays.
  *   n_threads  0 = all hardware threads.
  * Errors: STAGQ_EINVAL (null, group does not divide in, n_planes > STAGQ_MAX_PLANES,
- *         nnz mismatch, in > STAGQ_MAX_IN), STAGQ_ENOMEM.
+ *         nnz mismatch, in > STAGQ_MAX_IN, unknown pair-mode bits), STAGQ_ENOMEM.
  */
 int stagq_encode(const uint16_t* w, double density, int32_t pair_mode, int32_t n_threads,
                  stagq_fields* f);
