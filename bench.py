@@ -14,13 +14,16 @@ in ``per_gemv``.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl stagq|reference]
                   [--workload llama31_8b_linears_b1 | phi4_olmo2_linears_b1 | precision_sweep |
-                              llama31_8b_stack | llama31_8b_guarded]
+                              llama31_8b_stack | llama31_8b_guarded | cublas_context]
 
 The default workload is the Llama-3.1-8B layer above. The others print one
 JSON line each with per-GEMV (or per-token) times:
   phi4_olmo2_linears_b1  Phi-4 and OLMo-2-7B linears at 2/3/4 bits, batch 1,
                          each alone and as one layer's chain (q k v o gate up
                          down, one CUDA graph);
+  cublas_context         dense fp16 torch.mv (cuBLAS) on the Llama-3.1-8B shapes
+                         beside the StagQ GEMVs: the speedups of the paper's
+                         Table 5, as context;
   llama31_8b_guarded     the Llama-3.1-8B linears at group 32 with the paper's
                          side-record guards (ratio T = 4 + post-grid), each
                          alone and as a layer chain;
@@ -67,7 +70,7 @@ def _args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--workload", default=WORKLOAD,
                    choices=[WORKLOAD, "phi4_olmo2_linears_b1", "precision_sweep", "llama31_8b_stack",
-                            "llama31_8b_guarded"])
+                            "llama31_8b_guarded", "cublas_context"])
     p.add_argument("--stack-distinct", type=int, default=4,
                    help="llama31_8b_stack: distinct encoded layers (the 32 resident layers cycle over them)")
     return p.parse_args()
@@ -397,6 +400,53 @@ def run_extra(args):
                     BITS, GROUP, N_PLANES, DENSITY)
         cfg = {"linears_out_x_in": {k: list(v) for k, v in shapes}, "bits": list(BITS), "group": GROUP,
                "n_planes": N_PLANES, "side_record_density": DENSITY, "batch": 1}
+    elif args.workload == "cublas_context":
+        # Context only (the paper's Table 5 reports speedups over cuBLAS): the
+        # dense fp16 GEMV of torch (cuBLAS) on the Llama-3.1-8B shapes, timed
+        # like the StagQ GEMVs (a CUDA graph of launches rotating over device
+        # copies larger than L2), and the StagQ times of the same shapes.
+        shapes = _layer_shapes()
+        per_gemv(shapes, BITS, GROUP, N_PLANES, DENSITY)
+        for name, (out, inp) in shapes:
+            nbytes = 2 * out * inp
+            C = copies_for(Q, nbytes, l2, minimum=2)
+            Ws = [torch.randn(out, inp, device="cuda", dtype=torch.float16) * 0.02 for _ in range(C)]
+            xv = torch.from_numpy(synth.activations(1, inp, seed=inp)[0]).cuda()
+            yv = torch.empty(out, dtype=torch.float16, device="cuda")
+            with torch.cuda.stream(stream):
+                torch.mv(Ws[0], xv, out=yv)
+            torch.cuda.synchronize()
+            reps = 24
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for r in range(reps):
+                    torch.mv(Ws[(r + 1) % C], xv, out=yv)
+            g.replay()
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(3):
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    a0.record(stream)
+                    for _ in range(5):
+                        g.replay()
+                    a1.record(stream)
+                torch.cuda.synchronize()
+                ts.append(a0.elapsed_time(a1) * 1e3 / (5 * reps))
+            del g
+            us = statistics.median(ts)
+            nb = nbytes + 2 * inp + 2 * out
+            r = {"us": round(us, 3), "bytes": nb, "gbs": round(nb / us / 1e3, 1), "frac": round(nb / us / 1e3 / peak, 4)}
+            for b in BITS:
+                st = results.get(f"{name} {out}x{inp} p{b}")
+                if st:
+                    r[f"speedup_p{b}"] = round(us / st["us"], 3)
+            results[f"cublas_fp16 {name} {out}x{inp}"] = r
+            del Ws
+            torch.cuda.empty_cache()
+        cfg = {"linears_out_x_in": {k: list(v) for k, v in shapes}, "bits": list(BITS), "group": GROUP,
+               "n_planes": N_PLANES, "side_record_density": DENSITY, "batch": 1,
+               "note": "context: dense fp16 torch.mv (cuBLAS) on random weights; speedup = t_cuBLAS / t_StagQ"}
     elif args.workload == "llama31_8b_guarded":
         # The paper's guards on every linear (pre-grid ratio criterion T = 4 and
         # the post-grid per-row guard, Table 6 / Appendix E) at its kernel
