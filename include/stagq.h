@@ -261,9 +261,11 @@ int stagq_gemv_host(stagq_handle h, int bits, const void* x_host, int n, void* y
  * no counterpart; this is a property of this library's host interface.
  *   - The array exists on every GPU that loads the library and is held until
  *     the process exits.
- *   - The first call on a device looks up the array's device address with
- *     that device current (cudaGetSymbolAddress); make that first call before
- *     any stream capture.
+ *   - Every call looks up the array's device address with the handle's
+ *     device current (cudaGetSymbolAddress; nothing is cached, so a device
+ *     reset in between is harmless). The first call on a device may also
+ *     load the library's device code there; make that first call before any
+ *     stream capture.
  *   - All calls share the one array, which keeps the last call's contents
  *     (nothing of it is read before being written). Calls that overlap on the
  *     GPU race: issue them one at a time. The call returns after the copy of y

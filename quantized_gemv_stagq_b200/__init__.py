@@ -297,17 +297,60 @@ def stagq_load_file(path: str, device: int = 0) -> Matrix:
     return Matrix(h.value)
 
 
+def _check_device_tensor(t, name: str, dtype_name: str, numel: int, device: int) -> None:
+    """The C ABI takes raw pointers and sizes from the handle: a tensor of the
+    wrong type, layout or size would be read or written out of bounds on the
+    device, so it is refused here (and one on the wrong GPU by
+    _check_on_device)."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    want = getattr(torch, dtype_name)
+    if t.dtype != want:
+        raise TypeError(f"{name} must be {dtype_name}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements; the call needs {numel}")
+
+
+def _check_on_device(t, name: str, device: int) -> None:
+    import torch
+    if not t.is_cuda or (t.device.index if t.device.index is not None else torch.cuda.current_device()) != device:
+        raise ValueError(f"{name} must be on cuda:{device} (the matrix's GPU), got {t.device}")
+
+
+def _check_host_array(a, name: str, numel: int) -> None:
+    if not isinstance(a, np.ndarray) or a.dtype != np.float16:
+        raise TypeError(f"{name} must be a float16 numpy array")
+    if not a.flags["C_CONTIGUOUS"]:
+        raise ValueError(f"{name} must be C-contiguous")
+    if a.size < numel:
+        raise ValueError(f"{name} holds {a.size} elements; the call needs {numel}")
+
+
+def _check_gemv_args(m: Matrix, x, y, n: int, f32: bool) -> None:
+    # (n itself is checked by the library: STAGQ_EINVAL outside 1..STAGQ_MAX_BATCH)
+    _check_device_tensor(x, "x", "float16", n * m.inp, m.device)
+    _check_device_tensor(y, "y", "float32" if f32 else "float16", n * m.out, m.device)
+    _check_on_device(x, "x", m.device)
+    _check_on_device(y, "y", m.device)
+
+
 def stagq_gemv_ex(m: Matrix, bits: int, x, y, n: int = 1, flags: int = 0, stream=None) -> None:
     """x, y: CUDA tensors (x fp16 [n, inp]; y fp16 or fp32 [n, out])."""
+    _check_gemv_args(m, x, y, n, bool(flags & STAGQ_Y_F32))
     _check(lib().stagq_gemv_ex(m.handle, bits, x.data_ptr(), n, y.data_ptr(), flags,
                                _stream_ptr(stream)), "stagq_gemv_ex")
 
 
 def stagq_gemv(m: Matrix, bits: int, x, y, stream=None) -> None:
+    _check_gemv_args(m, x, y, 1, False)
     _check(lib().stagq_gemv(m.handle, bits, x.data_ptr(), y.data_ptr(), _stream_ptr(stream)), "stagq_gemv")
 
 
 def stagq_gemv_n(m: Matrix, bits: int, x, n: int, y, stream=None) -> None:
+    _check_gemv_args(m, x, y, n, False)
     _check(lib().stagq_gemv_n(m.handle, bits, x.data_ptr(), n, y.data_ptr(), _stream_ptr(stream)),
            "stagq_gemv_n")
 
@@ -315,6 +358,8 @@ def stagq_gemv_n(m: Matrix, bits: int, x, n: int, y, stream=None) -> None:
 def stagq_gemv_host(m: Matrix, bits: int, x_host: np.ndarray, y_host: np.ndarray, n: int = 1,
                     stream=None) -> None:
     """Host buffers (pinned or pageable numpy arrays): copies in and out, synchronous."""
+    _check_host_array(x_host, "x_host", n * m.inp)
+    _check_host_array(y_host, "y_host", n * m.out)
     _check(lib().stagq_gemv_host(m.handle, bits, x_host.ctypes.data, n, y_host.ctypes.data,
                                  _stream_ptr(stream)), "stagq_gemv_host")
 
@@ -324,11 +369,15 @@ def stagq_gemv_host_noalloc(m: Matrix, bits: int, x_host: np.ndarray, y_host: np
     """As stagq_gemv_host, staging through the library's static device array
     instead of a device buffer allocated on first use (no device allocation).
     Calls must not overlap on the GPU; see include/stagq.h."""
+    _check_host_array(x_host, "x_host", n * m.inp)
+    _check_host_array(y_host, "y_host", n * m.out)
     _check(lib().stagq_gemv_host_noalloc(m.handle, bits, x_host.ctypes.data, n, y_host.ctypes.data,
                                          _stream_ptr(stream)), "stagq_gemv_host_noalloc")
 
 
 def stagq_decode_levels(m: Matrix, bits: int, u_dev, stream=None) -> None:
+    _check_device_tensor(u_dev, "u_dev", "uint8", m.out * m.inp, m.device)
+    _check_on_device(u_dev, "u_dev", m.device)
     _check(lib().stagq_decode_levels(m.handle, bits, u_dev.data_ptr(), _stream_ptr(stream)),
            "stagq_decode_levels")
 

@@ -439,23 +439,17 @@ constexpr size_t kNoAllocStageBytes = (size_t)STAGQ_NOALLOC_STAGE_BYTES;        
 
 static __device__ __align__(256) uint8_t g_noalloc_stage[kNoAllocStageBytes];
 
-// Device address of g_noalloc_stage on each device. In host code the array's
-// name is only a host-side stand-in, so the address is taken once per device
-// with that device current.
-constexpr int kNoAllocMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
-
-int noalloc_stage(int device, uint8_t** out) {
-  if (device < 0 || device >= kNoAllocMaxDevices) return fail(STAGQ_EINVAL, "device index out of range");
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[device]) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_stage);
-    if (e != cudaSuccess || !p) return cuda_fail(e == cudaSuccess ? cudaErrorInvalidSymbol : e, "cudaGetSymbolAddress");
-    g_noalloc_ptr[device] = p;
-  }
-  *out = static_cast<uint8_t*>(g_noalloc_ptr[device]);
+// Device address of g_noalloc_stage on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is looked up with
+// the handle's device current -- on every call, not cached: a device reset
+// (cudaDeviceReset) rebuilds the context and the array may then sit at a new
+// address. The lookup allocates nothing and costs far less than the call's
+// synchronous copies.
+int noalloc_stage(uint8_t** out) {
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_stage);
+  if (e != cudaSuccess || !p) return cuda_fail(e == cudaSuccess ? cudaErrorInvalidSymbol : e, "cudaGetSymbolAddress");
+  *out = static_cast<uint8_t*>(p);
   return STAGQ_OK;
 }
 
@@ -474,7 +468,7 @@ extern "C" int stagq_gemv_host_noalloc(stagq_handle h, int bits, const void* x_h
   DeviceGuard guard(h->device);
   if (!guard.ok) return fail(STAGQ_ECUDA, "cudaSetDevice failed");
   uint8_t* stage = nullptr;
-  st = noalloc_stage(h->device, &stage);
+  st = noalloc_stage(&stage);
   if (st) return st;
   uint8_t* dx = stage;
   uint8_t* dy = stage + kNoAllocXBytes;

@@ -528,12 +528,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
   const RowOffsets step = {(uint32_t)(RG * rb), (uint32_t)(RG * rp), (uint32_t)(RG * ps)};
   const uint32_t plane_stride = BR * rp;
 
-  bool ok = mbar_wait(side_bar, 0, kWaitLimitNs);
+  // The lanes of a warp leave together: the block code below uses full-warp
+  // shuffles and __syncwarp.
+  bool ok = __all_sync(kFull, mbar_wait(side_bar, 0, kWaitLimitNs));
   const uint8_t* ring_g = smem + L.ring;
   int slot = 0;
   uint32_t phase = 0, round = 0;
   for (int b = 0; ok && b < nblk; ++b) {
-    if (!mbar_wait(full0 + 8 * slot, phase, kWaitLimitNs)) {
+    if (!__all_sync(kFull, mbar_wait(full0 + 8 * slot, phase, kWaitLimitNs))) {
       ok = false;
       break;
     }

@@ -273,7 +273,9 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
       }
     }
   }
-  bool ok = __all_sync(kFull, mbar_wait(side_bar, 0, kWaitLimit1Ns));
+  // Every warp takes the same branch: the term pass reads the entries' local
+  // rows, which all warps write.
+  bool ok = __syncthreads_and(mbar_wait(side_bar, 0, kWaitLimit1Ns)) != 0;
   const int32_t* offs = reinterpret_cast<const int32_t*>(side);
   const uint32_t* ents = reinterpret_cast<const uint32_t*>(side + P.side_ent_off);
   // local row of each held-out entry (a thread per row)

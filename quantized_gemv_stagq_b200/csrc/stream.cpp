@@ -49,6 +49,28 @@ int validate_stream(const stagq_host_stream* s) {
     for (int64_t e = (int64_t)s->row_ptr[r] + 1; e < s->row_ptr[r + 1]; ++e)
       if ((s->col[e] & kCol) <= (s->col[e - 1] & kCol))
         return fail(STAGQ_EFORMAT, "side-record columns not increasing in a row");
+  // Digits under the side record (Section 3.6: the planes skip held-out
+  // positions). The GEMV corrects a held-out position by x_c (v - lo_M) or
+  // x_c (r + lo - lo_M), which is exact only if the main stream decodes lo_M
+  // there (a pre-grid entry: q = 0 and zero planes) or lo_M + s q (a
+  // post-grid entry: zero planes). Checked at the stream's full depth N.
+  const int N = 2 + s->n_planes;
+  const int64_t out = s->out, in = s->in;
+  for (int64_t r = 0; r < out; ++r) {
+    for (int64_t e = s->row_ptr[r]; e < s->row_ptr[r + 1]; ++e) {
+      const int64_t c = s->col[e] & kCol, chunk = c / kChunk;
+      uint32_t base[4];
+      uint32_t pw[STAGQ_MAX_PLANES][2] = {};
+      std::memcpy(base, s->planes + base_chunk_offset(r, in, chunk), 16);
+      for (int k = 3; k <= N; ++k)
+        std::memcpy(pw[k - 3], s->planes + plane_region_offset(out, in, k) + plane_chunk_offset(r, in, chunk), 8);
+      const int u = chunk_level(base, pw, N, (int)(c % kChunk));
+      const bool post = (s->col[e] & STAGQ_SIDE_POST) != 0;
+      if (post ? (u & ((1 << (N - 2)) - 1)) != 0 : u != 0)
+        return fail(STAGQ_EFORMAT, post ? "nonzero plane digit under a post-grid side-record entry"
+                                        : "nonzero digit under a pre-grid side-record entry");
+    }
+  }
   return STAGQ_OK;
 }
 

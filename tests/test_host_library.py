@@ -253,3 +253,68 @@ def test_guarded_encoder_error_paths():
             raise Q.StagqError(st, "capacity")
     assert e.value.status == 1                        # capacity one short of stagq_guard_capacity
     assert Q.stagq_guard_capacity(8, 256, 64) == 8 * 4 + 8
+
+
+def test_stream_with_digits_under_the_side_record_is_refused(tmp_path):
+    """The GEMV's side-record correction needs the zero-digit convention
+    (Section 3.6): a pre-grid position stores q = 0 and zero planes, a
+    post-grid position zero planes (its base digit stays). A stream that
+    breaks it is refused with STAGQ_EFORMAT by stagq_save and stagq_load."""
+    W = synth.weights(16, 256, seed=5)
+    F = O.encode(W, 64, 2, 0.02, "fast")
+    r = int(np.argmax(np.diff(F.row_ptr) > 0))
+    c = int(F.col[F.row_ptr[r]])
+    path = str(tmp_path / "x.stagq")
+    Q.stagq_save(Q.stagq_pack(to_lib_fields(F)), path)            # the convention holds: accepted
+    for what in ("q", "plane3", "plane4"):
+        L = to_lib_fields(F)
+        if what == "q":
+            L.q[r, c] = 2
+        else:
+            L.planes[int(what[-1]) - 3, r, c] = 1
+        S = Q.stagq_pack(L)
+        for call in (lambda: Q.stagq_save(S, path), lambda: Q.stagq_load(S, 0)):
+            with pytest.raises(Q.StagqError) as e:
+                call()
+            assert e.value.status == 2, what
+    # post-grid entries keep their base digit but no plane digit
+    G = O.encode(synth.weights(8, 256, seed=6), 64, 2, mode="fast", guard="ratio", ratio_T=4.0, post_guard=True)
+    e = int(np.flatnonzero(G.post_flags)[0])
+    r = int(np.searchsorted(G.row_ptr, e, side="right") - 1)
+    c = int(G.col[e])
+    L = to_lib_fields(G)
+    L.q[r, c] = 3
+    Q.stagq_save(Q.stagq_pack(L), path)                           # a base digit is allowed
+    L.planes[0, r, c] = 1
+    with pytest.raises(Q.StagqError) as e:
+        Q.stagq_save(Q.stagq_pack(L), path)
+    assert e.value.status == 2
+
+
+def test_binding_refuses_tensors_that_do_not_fit_the_call():
+    """The binding checks every x / y / u against the handle's shape before a
+    pointer reaches the C ABI (a short y would be written out of bounds on the
+    device). No GPU is needed: each bad argument fails before the device check."""
+    import torch
+    m = Q.Matrix.__new__(Q.Matrix)              # a handle's shape without a device
+    m.handle, m.out, m.inp, m.device = None, 64, 512, 0
+    x = torch.zeros(1, 512, dtype=torch.float16)
+    y_short = torch.zeros(1, 63, dtype=torch.float16)
+    with pytest.raises(ValueError, match="y holds 63"):
+        Q.stagq_gemv(m, 2, x, y_short)
+    with pytest.raises(ValueError, match="x holds 512 elements; the call needs 1024"):
+        Q.stagq_gemv_n(m, 2, x, 2, torch.zeros(2, 64, dtype=torch.float16))
+    with pytest.raises(TypeError, match="x must be float16"):
+        Q.stagq_gemv(m, 2, x.float(), torch.zeros(1, 64, dtype=torch.float16))
+    with pytest.raises(TypeError, match="y must be float32"):    # STAGQ_Y_F32 asks for an fp32 y
+        Q.stagq_gemv_ex(m, 2, x, torch.zeros(1, 64, dtype=torch.float16), flags=Q.STAGQ_Y_F32)
+    with pytest.raises(ValueError, match="contiguous"):
+        Q.stagq_gemv(m, 2, torch.zeros(512, 2, dtype=torch.float16).t()[:1], torch.zeros(1, 64, dtype=torch.float16))
+    with pytest.raises(ValueError, match="cuda:0"):              # right type and size, wrong device
+        Q.stagq_gemv(m, 2, x, torch.zeros(1, 64, dtype=torch.float16))
+    with pytest.raises(ValueError, match="u_dev holds"):
+        Q.stagq_decode_levels(m, 2, torch.zeros(64, 511, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="y_host holds"):
+        Q.stagq_gemv_host(m, 2, np.zeros((1, 512), np.float16), np.zeros((1, 32), np.float16))
+    with pytest.raises(TypeError, match="x_host"):
+        Q.stagq_gemv_host_noalloc(m, 2, np.zeros((1, 512), np.float32), np.zeros((1, 64), np.float16))

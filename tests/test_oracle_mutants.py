@@ -97,7 +97,27 @@ def _ratio_guard_second_excluded_wrongly(W, group, T):
     return mask.reshape(out, inp)
 
 
+_choose_pairs = O.choose_pairs
+
+
+def _fast_pairs_nibbles_swapped(Vc, group, N, lo_tab, s_tab, empty, mode="search", **kw):
+    """The fast rule with the log2(s) index in the low nibble."""
+    idx = _choose_pairs(Vc, group, N, lo_tab, s_tab, empty, mode=mode, **kw).astype(np.int64)
+    if mode == "fast":
+        idx = (idx & 15) * 16 + (idx >> 4)
+    return idx.astype(np.uint8)
+
+
+def _fast_pairs_lo_not_divided(Vc, group, N, lo_tab, s_tab, empty, mode="search", lo0=None, s0=None, **kw):
+    """The fast rule matching lo0 itself instead of lo0 / s0 against the lo/s codebook."""
+    if mode == "fast":
+        return _choose_pairs(Vc, group, N, lo_tab, s_tab, empty, mode=mode, lo0=lo0 * s0, s0=s0, **kw)
+    return _choose_pairs(Vc, group, N, lo_tab, s_tab, empty, mode=mode, lo0=lo0, s0=s0, **kw)
+
+
 @pytest.mark.parametrize("name,mutant,pins", [
+    ("choose_pairs", _fast_pairs_nibbles_swapped, ["test_fast_pair_rule_matches_scalar_nearest_entries"]),
+    ("choose_pairs", _fast_pairs_lo_not_divided, ["test_fast_pair_rule_matches_scalar_nearest_entries"]),
     ("grid_at", _grid_wrong_sign, ["test_eq9_equals_eq10_all_digit_patterns", "test_figure1_every_prefix_is_a_grid_point"]),
     ("grid_at", _grid_wrong_spacing, ["test_every_precision_is_a_uniform_grid", "test_midpoint_split_is_the_mmse_split"]),
     ("half_step", _half_step_wrong, ["test_figure1_worked_example", "test_sign_planes_equal_nearest_level_rounding"]),

@@ -573,3 +573,74 @@ def test_input_scale_is_a_column_scaling_of_w_hat():
         xs = (x.astype(np.float64) * p2.astype(np.float64)).astype(np.float64)
         assert np.array_equal(O.gemv(F, M, x, in_scale=p2), xs @ D.T)
         assert np.array_equal(O.gemv(F, M, x, in_scale=np.ones(256, np.float32)), O.gemv(F, M, x))
+
+
+# ------------------------------------- the labelled fast pair rule (Section 3.1)
+
+def _nearest_entry(cb, v):
+    """Index of the codebook entry nearest to v, ties to the smaller index
+    (a scalar scan)."""
+    best = 0
+    for i in range(1, len(cb)):
+        if abs(float(cb[i]) - v) < abs(float(cb[best]) - v):
+            best = i
+    return best
+
+
+def _scalar_fast_pairs(W, held, group, cb_log2s, cb_lo_over_s, N):
+    """The fast rule restated with scalar loops per group: clip held-out
+    entries to the group's retained max (w >= 0) or min (w < 0), take
+    Appendix B's initial pair (lo0 = min + 0.06 R, s0 = (max - 0.06 R - lo0)
+    / 3), then the nearest log2(s) entry (high nibble) and the nearest lo/s
+    entry (low nibble). A group with nothing retained takes pair 0; a group of
+    zero range is searched (Eq. (5) brute force)."""
+    out, inp = W.shape
+    idx = np.zeros((out, inp // group), dtype=np.int64)
+    for r in range(out):
+        for g in range(inp // group):
+            cols = range(g * group, (g + 1) * group)
+            kept = [float(W[r, c]) for c in cols if not held[r, c]]
+            if not kept:
+                idx[r, g] = 0
+                continue
+            hi, lo = max(kept), min(kept)
+            vals = [float(W[r, c]) if not held[r, c] else (hi if float(W[r, c]) >= 0.0 else lo) for c in cols]
+            mn, mx = min(vals), max(vals)
+            if mx == mn:
+                idx[r, g] = _brute_force_pair(vals, cb_log2s, cb_lo_over_s, N)
+                continue
+            R = mx - mn
+            lo0 = mn + 0.06 * R
+            s0 = (mx - 0.06 * R - lo0) / 3.0
+            a = _nearest_entry(cb_log2s, math.log2(s0))
+            b = _nearest_entry(cb_lo_over_s, lo0 / s0)
+            idx[r, g] = 16 * a + b
+    return idx
+
+
+def _fast_rule_weights():
+    W = synth.weights(8, 128, seed=57)
+    W[0, 0:16] = np.float16(0.01)                           # a zero-range group: searched
+    W[1, 16:32] = (np.arange(16) * 0.01 + 1.0).astype(np.float16)  # all held out: pair 0
+    return W
+
+
+def test_fast_pair_rule_matches_scalar_nearest_entries():
+    """The fast rule (used by the large workloads) against its statement in
+    scalar loops, on groups with held-out entries, a zero-range group and a
+    fully held-out group."""
+    W = _fast_rule_weights()
+    density = 24 / W.size
+    for n_planes in (2, 4):
+        F = O.encode(W, group=16, n_planes=n_planes, density=density, mode="fast")
+        held = np.zeros(W.shape, dtype=bool)
+        for r in range(F.out):
+            for e in range(F.row_ptr[r], F.row_ptr[r + 1]):
+                held[r, F.col[e]] = True
+        assert held[1, 16:32].all() and held.sum() == 24
+        want = _scalar_fast_pairs(W, held, 16, F.cb_log2s, F.cb_lo_over_s, 2 + n_planes)
+        assert want[1, 1] == 0
+        assert np.array_equal(F.pair_idx.astype(np.int64), want)
+        # the rule is not the search: on these groups at least one pair differs
+        S = O.encode(W, group=16, n_planes=n_planes, density=density, mode="search")
+        assert not np.array_equal(S.pair_idx, F.pair_idx)

@@ -43,6 +43,26 @@ def test_noalloc_host_gemv_matches_host_gemv_on_consecutive_calls():
     m.free()
 
 
+def test_noalloc_host_gemv_on_a_large_matrix():
+    """A matrix of more than 2^24 weights, where n = 1 runs the single-vector
+    kernel: its reads of x from the static array match the allocating call."""
+    out, inp = 14336, 4096
+    P = Q.stagq_encode(synth.weights(out, inp, seed=81), 128, 2, 0.005, "fast")
+    m = Q.stagq_load(Q.stagq_pack(P), 0)
+    rng = np.random.default_rng(82)
+    for call, bits in enumerate((4, 2)):
+        x = rng.standard_normal((1, inp)).astype(np.float16)
+        y_ref = np.empty((1, out), np.float16)
+        y = np.full((1, out), np.float16(np.nan))
+        Q.stagq_gemv_host(m, bits, x, y_ref)
+        Q.stagq_gemv_host_noalloc(m, bits, x, y)
+        assert np.all(np.isfinite(y)), f"call {call}: y not fully written"
+        check_close(y.astype(np.float64), y_ref.astype(np.float64), f"large call {call} p{bits}")
+        assert np.array_equal(y.view(np.uint16), y_ref.view(np.uint16)), f"large call {call}: not bit-identical"
+    Q.stagq_check(m)
+    m.free()
+
+
 def test_noalloc_host_gemv_rejects_outputs_beyond_the_static_area():
     out, inp = 8192, 128
     P = Q.stagq_encode(synth.weights(out, inp, seed=79), 64, 1, 0.0, "fast")
