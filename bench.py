@@ -1,16 +1,18 @@
 """StagQ batch-one GEMV benchmark on B200.
 
-Workload (one step): the seven linears of one Llama-3.1-8B layer (q/k/v/o,
-gate/up, down; out x in as in the model), synthetic weights, group 128, base +
-2 refinement planes, 0.5 % side record, x fp16 N(0,1), batch 1, each GEMV run
-at 2, 3 and 4 bits -- 21 GEMVs per step. Every step is one CUDA-graph replay;
-steps rotate over several device copies of the layer so every read comes from
-HBM (copies x bytes >> L2).
+Workload (one step): one Llama-3.1-8B layer's linears (q/k/v/o, gate/up, down;
+out x in as in the model), synthetic weights, group 128, base + 2 refinement
+planes, 0.5 % side record, x fp16 N(0,1), batch 1, at 2, then 3, then 4 bits.
+Per precision the layer runs as a decode runs it: q/k/v in one launch (one
+stacked handle: they share x), o, gate/up in one launch, down -- 4 launches,
+12 per step, 21 GEMVs. Each precision pass reads its own device copy of the
+layer, and a copy is read again only after at least 4x the L2 size of other
+reads, so every byte comes from HBM. Every step is one CUDA-graph replay.
 
 Prints one JSON line. ``value`` is the whole job's algorithmic HBM traffic
 (planes read at the chosen precision + pairs + side record + x + y) divided by
-device time, in GB/s. Per-GEMV microseconds for every shape and precision are
-in ``per_gemv``.
+device time, in GB/s. Per-launch microseconds for every launch and precision
+are in ``per_launch``.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl stagq|reference]
                   [--workload llama31_8b_linears_b1 | phi4_olmo2_linears_b1 | precision_sweep |
@@ -66,7 +68,7 @@ def _args():
     p.add_argument("--steps", type=int, default=50)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="stagq", choices=["stagq", "reference"])
-    p.add_argument("--copies", type=int, default=6, help="device copies of the layer rotated over")
+    p.add_argument("--copies", type=int, default=6, help="least device copies of the layer rotated over")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--workload", default=WORKLOAD,
                    choices=[WORKLOAD, "phi4_olmo2_linears_b1", "precision_sweep", "llama31_8b_stack",
@@ -160,11 +162,12 @@ class ClockSampler:
                 "samples": len(sm), "power_w_max": max(power) if power else None}
 
 
-def _kernel_of(key):
-    """Name of the kernel that serves the GEMV `name@pM` at n = 1."""
+def _launch_kernel(key):
+    """Name of the kernel that serves the step launch `name@pM` at n = 1."""
     from quantized_gemv_stagq_b200 import synth
-    out, inp = synth.LLAMA31_8B_LINEARS[key.split("@")[0]]
-    return "gemv1_kernel" if out * inp > LARGE_WEIGHTS else "gemv_kernel"
+    members = dict(LAYER_LAUNCHES)[key.split("@")[0]]
+    weights = sum(synth.LLAMA31_8B_LINEARS[n][0] * synth.LLAMA31_8B_LINEARS[n][1] for n in members)
+    return "gemv1_kernel" if weights > LARGE_WEIGHTS else "gemv_kernel"
 
 
 def _layer_shapes():
@@ -244,7 +247,7 @@ def run_reference(args):
 def time_gemv(Q, torch, mats, bits, x, y, n, stream, reps=24, repeats=5):
     """Device time of one GEMV (µs): a CUDA graph of `reps` launches rotating
     over the device copies in `mats` (so reads come from HBM), replayed
-    `repeats` times between CUDA events; median over 3 such measurements."""
+    `repeats` times between CUDA events; median over 10 such measurements."""
     C = len(mats)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
@@ -255,18 +258,9 @@ def time_gemv(Q, torch, mats, bits, x, y, n, stream, reps=24, repeats=5):
             Q.stagq_gemv_n(mats[(r + 1) % C], bits, x, n, y, stream=stream)
     g.replay()
     torch.cuda.synchronize()
-    out = []
-    for _ in range(3):
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            a0.record(stream)
-            for _ in range(repeats):
-                g.replay()
-            a1.record(stream)
-        torch.cuda.synchronize()
-        out.append(a0.elapsed_time(a1) * 1e3 / (repeats * reps))
+    us = _median_event_us(torch, stream, lambda: [g.replay() for _ in range(repeats)], 10) / (repeats * reps)
     del g
-    return statistics.median(out)
+    return us
 
 
 def job_ms(ms: float, dist=None, device: str = "cuda") -> float:
@@ -339,24 +333,29 @@ def run_extra(args):
             del S
 
     def layer_chain(model, linears, bits_list, group, n_planes, density, **enc):
-        """One layer's linears in order as one CUDA graph (the chain a decode
-        step runs), rotating over enough device copies that reads come from
-        HBM; µs per layer."""
+        """One layer's linears as a decode runs them -- q/k/v stacked in one
+        launch, o, gate/up stacked, down -- as one CUDA graph, rotating over
+        enough device copies that reads come from HBM; µs per layer."""
         nonlocal launches
         streams = {}
         for _, (out, inp) in linears:
             if (out, inp) not in streams:
                 streams[(out, inp)] = Q.stagq_pack(Q.stagq_encode(synth.weights(out, inp, seed=out + 3 * inp),
                                                                   group, n_planes, density, "fast", **enc))
-        first = [Q.stagq_load(streams[v], 0) for _, v in linears]
+        shape = dict(linears)
+        groups = [("q", "k", "v"), ("o",), ("gate", "up"), ("down",)]
+
+        def load():
+            return [Q.stagq_load_stack([streams[shape[n]] for n in grp], 0) for grp in groups]
+        first = load()
         C = copies_for(Q, sum(m.device_bytes for m in first), l2, minimum=2)
-        mats = [first] + [[Q.stagq_load(streams[v], 0) for _, v in linears] for _ in range(C - 1)]
-        xs = {inp: torch.from_numpy(synth.activations(1, inp, seed=inp)).cuda() for _, (_, inp) in linears}
-        ys = [torch.empty(1, out, dtype=torch.float16, device="cuda") for _, (out, _) in linears]
+        mats = [first] + [load() for _ in range(C - 1)]
+        xs = [torch.from_numpy(synth.activations(1, m.inp, seed=m.inp)).cuda() for m in first]
+        ys = [torch.empty(1, m.out, dtype=torch.float16, device="cuda") for m in first]
         for b in bits_list:
             def body(c):
-                for j, (_, (out, inp)) in enumerate(linears):
-                    Q.stagq_gemv(mats[c][j], b, xs[inp], ys[j], stream=stream)
+                for j, m in enumerate(mats[c]):
+                    Q.stagq_gemv(m, b, xs[j], ys[j], stream=stream)
             with torch.cuda.stream(stream):
                 body(0)
             torch.cuda.synchronize()
@@ -367,21 +366,12 @@ def run_extra(args):
                     body(r % C)
             g.replay()
             torch.cuda.synchronize()
-            ts = []
-            for _ in range(3):
-                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                with torch.cuda.stream(stream):
-                    a0.record(stream)
-                    for _ in range(4):
-                        g.replay()
-                    a1.record(stream)
-                torch.cuda.synchronize()
-                ts.append(a0.elapsed_time(a1) * 1e3 / (4 * reps))
-            launches += len(linears) * (1 + 13 * reps)
-            us = statistics.median(ts)
+            us = _median_event_us(torch, stream, lambda: [g.replay() for _ in range(4)], 10) / (4 * reps)
+            launches += len(groups) * (1 + 41 * reps)
             nb = sum(Q.stagq_bytes(m, b, 1) for m in first)
             results[f"{model} layer p{b}"] = {"us": round(us, 3), "bytes": nb, "gbs": round(nb / us / 1e3, 1),
-                                              "frac": round(nb / us / 1e3 / peak, 4), "gemvs": len(linears)}
+                                              "frac": round(nb / us / 1e3 / peak, 4), "gemvs": len(linears),
+                                              "launches": len(groups)}
             del g
         for L in mats:
             for m in L:
@@ -471,13 +461,17 @@ def run_extra(args):
     else:  # llama31_8b_stack
         layers, K = 32, max(1, args.stack_distinct)
         shapes = _layer_shapes()
+        names = [n for n, _ in shapes]
         enc = []
         for li in range(K):
-            enc.append([Q.stagq_pack(Q.stagq_encode(synth.weights(o, i, seed=1000 * li + j), GROUP, N_PLANES,
-                                                    DENSITY, "fast")) for j, (_, (o, i)) in enumerate(shapes)])
-        stack = [[Q.stagq_load(enc[li % K][j], 0) for j in range(len(shapes))] for li in range(layers)]
+            enc.append({n: Q.stagq_pack(Q.stagq_encode(synth.weights(o, i, seed=1000 * li + j), GROUP, N_PLANES,
+                                                       DENSITY, "fast")) for j, (n, (o, i)) in enumerate(shapes)})
+        # per layer the launches a decode runs: q/k/v stacked, o, gate/up stacked, down
+        stack = [[Q.stagq_load_stack([enc[li % K][n] for n in members], 0) for _, members in LAYER_LAUNCHES]
+                 for li in range(layers)]
         del enc
         weights = layers * sum(o * i for _, (o, i) in shapes)
+        shapes = [(name, (stack[0][j].out, stack[0][j].inp)) for j, (name, _) in enumerate(LAYER_LAUNCHES)]
         for batch in (1, 4):
             xs = [torch.from_numpy(synth.activations(batch, i, seed=i + batch)).cuda() for _, (o, i) in shapes]
             ys = [torch.empty(batch, o, dtype=torch.float16, device="cuda") for _, (o, i) in shapes]
@@ -510,13 +504,14 @@ def run_extra(args):
                 results[f"p{b} batch{batch}"] = {"us_per_token_step": round(us, 1),
                                                  "us_per_token": round(us / batch, 1), "bytes": nb,
                                                  "gbs": round(nb / us / 1e3, 1), "frac": round(nb / us / 1e3 / peak, 4),
-                                                 "gemvs": layers * len(shapes)}
+                                                 "gemvs": layers * len(names), "launches": layers * len(shapes)}
                 del g
         stored = sum(m.device_bytes for L in stack for m in L)
         for L in stack:
             for m in L:
                 m.free()
-        cfg = {"layers": layers, "linears_out_x_in": {k: list(v) for k, v in shapes}, "weights": weights,
+        cfg = {"layers": layers, "linears_out_x_in": {k: list(v) for k, v in _layer_shapes()},
+               "launches_per_layer": {name: list(members) for name, members in LAYER_LAUNCHES}, "weights": weights,
                "distinct_encoded_layers": K, "stored_bytes": stored, "bits": list(BITS), "batches": [1, 4],
                "group": GROUP, "n_planes": N_PLANES, "side_record_density": DENSITY,
                "note": f"the 32 resident layers cycle over {K} distinct encodings (timing does not depend on "
@@ -525,6 +520,27 @@ def run_extra(args):
     vals = [r["gbs"] for r in results.values()]
     value = round(statistics.median(vals), 1) if vals else None
     _extra_line(args, args.workload, results, cfg, clk, peak, peak_kind, value, "GB/s", launches)
+
+
+# The layer step: per precision, the launches of one Llama-3.1-8B layer as a
+# decode runs them -- q/k/v stacked in one handle (they share x), o, gate/up
+# stacked (they share x), down -- each on its own input.
+LAYER_LAUNCHES = [("qkv", ("q_proj", "k_proj", "v_proj")), ("o", ("o_proj",)),
+                  ("gate_up", ("gate_proj", "up_proj")), ("down", ("down_proj",))]
+
+
+def _median_event_us(torch, stream, fn, repeats):
+    """Median of `repeats` CUDA-event timings (µs) of fn() on `stream`."""
+    out = []
+    for _ in range(repeats):
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a0.record(stream)
+            fn()
+            a1.record(stream)
+        torch.cuda.synchronize()
+        out.append(a0.elapsed_time(a1) * 1e3)
+    return statistics.median(out)
 
 
 def run_stagq(args):
@@ -542,44 +558,52 @@ def run_stagq(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     torch.cuda.set_device(local)
     dev = local
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
 
-    # ---- encode one layer (library encoder, fast pair rule), load C copies
+    # ---- encode the layer once (library encoder, fast pair rule) and pack
     shapes = _layer_shapes()
-    streams = []
+    packed = {}
     for li, (name, (out, inp)) in enumerate(shapes):
         W = synth.weights(out, inp, seed=100 + li)
-        P = Q.stagq_encode(W, GROUP, N_PLANES, DENSITY, "fast")
-        streams.append((name, out, inp, Q.stagq_pack(P), P.nnz))
-        del W, P
-    C = max(2, args.copies)
-    mats = [[Q.stagq_load(s, dev) for (_, _, _, s, _) in streams] for _ in range(C)]
-    xs = [torch.from_numpy(synth.activations(1, inp, seed=200 + i)).cuda() for i, (_, _, inp, _, _) in enumerate(streams)]
-    ys = [torch.empty(1, out, dtype=torch.float16, device="cuda") for (_, out, _, _, _) in streams]
-    step_bytes = sum(Q.stagq_bytes(mats[0][i], b, 1) for b in BITS for i in range(len(streams)))
-    stored = sum(m.device_bytes for m in mats[0])
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        packed[name] = Q.stagq_pack(Q.stagq_encode(W, GROUP, N_PLANES, DENSITY, "fast"))
+        del W
+
+    def load_layer():
+        return [Q.stagq_load_stack([packed[n] for n in members], dev) for _, members in LAYER_LAUNCHES]
+
+    first = load_layer()
+    stored = sum(m.device_bytes for m in first)
+    step_bytes = sum(Q.stagq_bytes(first[i], b, 1) for b in BITS for i in range(len(first)))
+    # Cold protocol: a step runs p2, p3, p4 each on its own copy of the layer,
+    # and a copy comes back only after at least 4x the L2 size of other reads
+    # (C / 3 - 1 whole steps in between).
+    C = len(BITS) * max(-(-args.copies // len(BITS)), -(-4 * l2 // step_bytes) + 1)
+    layers = [first] + [load_layer() for _ in range(C - 1)]
+    xs = [torch.from_numpy(synth.activations(1, m.inp, seed=200 + i)).cuda() for i, m in enumerate(first)]
+    ys = [torch.empty(1, m.out, dtype=torch.float16, device="cuda") for m in first]
 
     stream = torch.cuda.Stream()
 
-    def step_launches(c):
-        for b in BITS:
-            for i in range(len(streams)):
-                Q.stagq_gemv(mats[c][i], b, xs[i], ys[i], stream=stream)
+    def step_launches(s):
+        for k, b in enumerate(BITS):
+            L = layers[(len(BITS) * s + k) % C]
+            for i, m in enumerate(L):
+                Q.stagq_gemv(m, b, xs[i], ys[i], stream=stream)
 
-    # ---- one CUDA graph per copy
-    graphs = []
+    # ---- one CUDA graph per distinct step (copies cycle every G steps)
+    G = C // len(BITS)
     with torch.cuda.stream(stream):
         step_launches(0)  # warm the launch path outside capture
     torch.cuda.synchronize()
-    for c in range(C):
+    graphs = []
+    for s in range(G):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            step_launches(c)
+            step_launches(s)
         graphs.append(g)
     torch.cuda.synchronize()
-
     for w in range(max(args.warmup, 3)):
-        graphs[w % C].replay()
+        graphs[w % G].replay()
     torch.cuda.synchronize()
 
     clocks = ClockSampler(torch.cuda.current_device() if world == 1 else local)
@@ -592,32 +616,35 @@ def run_stagq(args):
     with torch.cuda.stream(stream):
         e0.record(stream)
         for s in range(args.steps):
-            graphs[s % C].replay()
+            graphs[s % G].replay()
         e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
 
-    # ---- per-GEMV timing (same kernels, one shape/precision at a time)
+    # ---- per launch: each launch of the step alone, a CUDA graph of launches
+    # rotating over enough device copies of it that a pass over them is at
+    # least 4x the L2 size (every read from HBM), median of 10 timings
     per = {}
-    reps = 4 * C
     with torch.cuda.stream(stream):
-        for b in BITS:
-            for i, (name, out, inp, _, nnz) in enumerate(streams):
+        for i, (name, members) in enumerate(LAYER_LAUNCHES):
+            pool = [layers[c][i] for c in range(C)]
+            while len(pool) < copies_for(Q, first[i].device_bytes, l2):
+                pool.append(Q.stagq_load_stack([packed[n] for n in members], dev))
+            reps = 2 * len(pool)
+            for b in BITS:
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g, stream=stream):
                     for r in range(reps):
-                        Q.stagq_gemv(mats[(r + 1) % C][i], b, xs[i], ys[i], stream=stream)
+                        Q.stagq_gemv(pool[r % len(pool)], b, xs[i], ys[i], stream=stream)
                 g.replay()
-                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a0.record(stream)
-                for _ in range(5):
-                    g.replay()
-                a1.record(stream)
                 torch.cuda.synchronize()
-                us = a0.elapsed_time(a1) * 1e3 / (5 * reps)
-                nb = Q.stagq_bytes(mats[0][i], b, 1)
-                per.setdefault(f"p{b}", {})[name] = {"us": round(us, 3), "bytes": nb, "gbs": round(nb / us / 1e3, 1)}
+                us = _median_event_us(torch, stream, g.replay, 10) / reps
+                nb = Q.stagq_bytes(first[i], b, 1)
+                per.setdefault(f"p{b}", {})[name] = {"us": round(us, 3), "bytes": nb, "gbs": round(nb / us / 1e3, 1),
+                                                      "out_x_in": [first[i].out, first[i].inp], "copies": len(pool)}
                 del g
+            for m in pool[C:]:
+                m.free()
     clk = clocks.stop()
 
     if dist:
@@ -627,17 +654,18 @@ def run_stagq(args):
     # ---- end to end through the C ABI with host buffers
     e2e_steps = max(2, min(args.steps, 10))
     xh = [x.cpu().pin_memory().numpy() for x in xs]
-    yh = [torch.empty((1, out), dtype=torch.float16).pin_memory().numpy() for (_, out, _, _, _) in streams]
-    for i in range(len(streams)):
-        Q.stagq_gemv_host(mats[0][i], 2, xh[i], yh[i], stream=stream)
-    h2d = sum(2 * inp for b in BITS for (_, _, inp, _, _) in streams)
-    d2h = sum(2 * out for b in BITS for (_, out, _, _, _) in streams)
+    yh = [torch.empty((1, m.out), dtype=torch.float16).pin_memory().numpy() for m in first]
+    for i, m in enumerate(first):
+        Q.stagq_gemv_host(m, 2, xh[i], yh[i], stream=stream)
+    h2d = sum(2 * m.inp for b in BITS for m in first)
+    d2h = sum(2 * m.out for b in BITS for m in first)
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     for s in range(e2e_steps):
-        for b in BITS:
-            for i in range(len(streams)):
-                Q.stagq_gemv_host(mats[s % C][i], b, xh[i], yh[i], stream=stream)
+        for k, b in enumerate(BITS):
+            L = layers[(len(BITS) * s + k) % C]
+            for i, m in enumerate(L):
+                Q.stagq_gemv_host(m, b, xh[i], yh[i], stream=stream)
     e2e_s = time.perf_counter() - t0
     e2e_gbs = step_bytes * e2e_steps / e2e_s / 1e9
 
@@ -649,7 +677,7 @@ def run_stagq(args):
 
     peak, peak_kind = _peaks()
     value = job_value(world, step_bytes, args.steps, ms)
-    # dominant kernel: the (shape, precision) with the largest share of a step
+    # dominant kernel: the launch with the largest share of a step
     dom_key, dom = max(((f"{name}@{pb}", d) for pb, dd in per.items() for name, d in dd.items()),
                        key=lambda kv: kv[1]["us"])
     traffic, _ = _ncu_traffic()
@@ -664,19 +692,21 @@ def run_stagq(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "int32 dot (u8 codes x i16 x) + fp32", "data": "synthetic",
         "config": {"workload": WORKLOAD, "linears_out_x_in": {n: [o, i] for n, (o, i) in shapes}, "bits": list(BITS),
                    "group": GROUP, "n_planes": N_PLANES, "side_record_density": DENSITY, "batch": 1,
-                   "pair_rule": "fast", "gemvs_per_step": len(BITS) * len(shapes),
-                   "l2": f"inputs larger than L2: {C} rotating device copies x {stored / 1e6:.0f} MB stored, "
-                         f"{step_bytes / 1e6:.0f} MB read per step vs L2 {l2 / 1e6:.0f} MB",
+                   "pair_rule": "fast",
+                   "launches_per_step": {name: list(members) for name, members in LAYER_LAUNCHES},
+                   "gemvs_per_step": len(BITS) * len(shapes), "kernel_launches_per_step": len(BITS) * len(first),
+                   "l2": f"inputs larger than L2: each precision pass of a step reads its own layer copy; {C} copies x "
+                         f"{stored / 1e6:.0f} MB stored, {step_bytes / 1e6:.0f} MB read per step vs L2 {l2 / 1e6:.0f} MB",
                    "parallelism": "replicas" if world > 1 else "single"},
         "frac_of_hbm": round(value / world / peak, 4),
-        "per_gemv": per, "us_per_precision_layer": step_us,
-        "roofline": {"bound": "hbm", "kernel": f"{_kernel_of(dom_key)} {dom_key}", "achieved": dom["gbs"], "peak": peak,
+        "per_launch": per, "us_per_precision_layer": step_us,
+        "roofline": {"bound": "hbm", "kernel": f"{_launch_kernel(dom_key)} {dom_key}", "achieved": dom["gbs"], "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dom["gbs"] / peak, 4),
                      "traffic": traffic, "algorithmic_bytes": dom["bytes"]},
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "stagq_gemv_host (host x/y, copies + sync per call)"},
-        "gpu_launches": len(BITS) * len(shapes) * args.steps,
+        "gpu_launches": len(BITS) * len(first) * args.steps,
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)

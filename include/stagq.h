@@ -46,6 +46,7 @@ extern "C" {
 /* Limits of this implementation. */
 #define STAGQ_MAX_PLANES 4      /* stream depth N = 2 + n_planes <= 6 (the paper evaluates N = 6) */
 #define STAGQ_MAX_BATCH 4       /* columns of x per call in stagq_gemv_n */
+#define STAGQ_MAX_STACK 4       /* member matrices of one stacked handle (stagq_load_stack) */
 #define STAGQ_MAX_IN 32768      /* K; side-record columns are stored as uint16 */
 #define STAGQ_IN_MULTIPLE 128   /* K must be a multiple of this (16-byte plane rows) */
 /* The group size of a loadable stream is a power of two, at least this, dividing
@@ -213,6 +214,23 @@ int stagq_load_file(const char* path, int device, stagq_handle* out);
 int stagq_load(const stagq_host_stream* s, int device, stagq_handle* out);
 
 /*
+ * One handle for up to STAGQ_MAX_STACK matrices that are applied to the same
+ * x (a transformer layer's q/k/v projections, or gate/up): member j's rows
+ * follow member j-1's, so the handle is one (sum of outs) x in matrix and
+ * every GEMV entry point serves all members in one launch, with y the
+ * members' outputs one after the other. Each member keeps its own
+ * codebooks (the paper fits them per matrix, Section 3.1), pair bytes and
+ * side record; the members must share in, group and n_planes. The result of
+ * member j's rows equals what a handle of member j alone computes (same
+ * arithmetic per row). stagq_bytes counts x once.
+ *   members   host array of `count` streams (1 <= count <= STAGQ_MAX_STACK);
+ *             the caller keeps ownership of everything they point to.
+ * Errors: STAGQ_EINVAL (count, null, members that differ in in / group /
+ * n_planes), the errors of stagq_load.
+ */
+int stagq_load_stack(const stagq_host_stream* const* members, int count, int device, stagq_handle* out);
+
+/*
  * y = W_hat^(bits) x for one vector (n = 1), asynchronously on `cuda_stream`
  * (a cudaStream_t; NULL = the legacy default stream).
  *   bits   2 .. 2 + n_planes
@@ -240,6 +258,18 @@ int stagq_gemv_n(stagq_handle h, int bits, const void* x, int n, void* y, void* 
  */
 int stagq_gemv_ex(stagq_handle h, int bits, const void* x, int n, void* y, uint32_t flags,
                   void* cuda_stream);
+
+/*
+ * As stagq_gemv_ex with the run-time inverse activation scale (Appendix E:
+ * the quantiser saw W diag(a), so the decoder multiplies channel c of x by
+ * 1/a_c): y_j = W_hat^(bits) (x_j .* in_scale) for each of the n vectors.
+ *   in_scale  device [in] fp32 (the values 1/a_c), 16-byte aligned.
+ * The product x_c in_scale_c is rounded to fp32, then converted like x
+ * (separate kernel instances: calls without a scale keep their code).
+ * Errors: as stagq_gemv_ex; STAGQ_EINVAL for a null or misaligned in_scale.
+ */
+int stagq_gemv_scaled(stagq_handle h, int bits, const void* x, int n, const float* in_scale, void* y,
+                      uint32_t flags, void* cuda_stream);
 
 /*
  * End-to-end call with HOST buffers: copies x (host [n*in] fp16) to the
@@ -300,6 +330,48 @@ int64_t stagq_bytes(stagq_handle h, int bits, int n);
 int stagq_check(stagq_handle h);
 
 int stagq_info(stagq_handle h, stagq_info_t* info);
+
+/* ------------------------------------------------------------ test hooks */
+
+/*
+ * Test hook for the bounded waits: while stall_ns != 0, every GEMV launched
+ * on the handle (its arguments are taken at launch, so a captured CUDA graph
+ * keeps the value of its capture) first waits at most stall_ns on a barrier
+ * that nothing completes. The wait runs out, the kernel takes its give-up
+ * path -- it lets its own copies in flight land, sets the handle's status
+ * word and returns without writing y -- and the next stagq_check returns
+ * STAGQ_ETIMEOUT. No GPU fault is involved. 0 turns the hook off.
+ */
+int stagq_debug_stall(stagq_handle h, uint32_t stall_ns);
+
+/*
+ * Where the handle's side record lives on the device: the loader re-lays the
+ * CSR record (Eq. 4) per CTA for each kernel's grid.
+ *   General kernel (grid CTAs, stride bytes each): CTA b owns rows
+ *   [b out / grid, (b + 1) out / grid); its rows fall in row_groups classes
+ *   (local row mod row_groups); int32 offsets [row_groups][k_slices]
+ *   [class_rows + 1] give where row m of a class starts within the run of
+ *   its (class, K slice) -- a K slice is 2048 columns -- and the run's end;
+ *   entries (uint32: column with the post-grid flag in bit 15 | fp16 value
+ *   << 16) start at ent_off.
+ *   Single-vector kernel (grid1 CTAs, stride1 bytes each, same row split):
+ *   int32 offsets [rows + 1] per local row, entries at ent_off1 in (row,
+ *   column) order, same word.
+ */
+typedef struct {
+    int32_t grid, stride, ent_off, row_groups, k_slices, class_rows;
+    int32_t grid1, stride1, ent_off1;
+} stagq_side_layout_t;
+
+/*
+ * Test hook: fills *layout and copies the two device cuts of the side record
+ * to host memory (grid * stride and grid1 * stride1 bytes; a null buffer is
+ * skipped), so that a test can check them entry by entry against the CSR.
+ * Errors: STAGQ_EINVAL (null handle or layout, a buffer below its size),
+ * STAGQ_ECUDA.
+ */
+int stagq_debug_side_record(stagq_handle h, stagq_side_layout_t* layout, void* cut_host, int64_t cut_bytes,
+                            void* cut1_host, int64_t cut1_bytes);
 
 /* Release the handle's device memory. Null-safe. */
 void stagq_free(stagq_handle h);

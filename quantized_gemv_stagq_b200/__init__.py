@@ -27,6 +27,7 @@ STAGQ_SIDE_POST = 0x8000
 STAGQ_CODEBOOK_RULES = 0x100
 STAGQ_MAX_PLANES = 4
 STAGQ_MAX_BATCH = 4
+STAGQ_MAX_STACK = 4
 
 _c_p = ctypes.c_void_p
 _i32, _i64, _u32, _dbl = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_double
@@ -45,6 +46,11 @@ class _HostStream(ctypes.Structure):
                 ("planes", _c_p), ("pair_idx", _c_p), ("row_ptr", _c_p), ("col", _c_p), ("val", _c_p)]
 
 
+class _SideLayout(ctypes.Structure):
+    _fields_ = [("grid", _i32), ("stride", _i32), ("ent_off", _i32), ("row_groups", _i32), ("k_slices", _i32),
+                ("class_rows", _i32), ("grid1", _i32), ("stride1", _i32), ("ent_off1", _i32)]
+
+
 class _Info(ctypes.Structure):
     _fields_ = [("out", _i32), ("in_", _i32), ("group", _i32), ("n_planes", _i32), ("nnz", _i64),
                 ("device", _i32), ("device_bytes", _i64)]
@@ -61,15 +67,20 @@ _SIGNATURES = {
     "stagq_save": (ctypes.c_int, [ctypes.POINTER(_HostStream), ctypes.c_char_p]),
     "stagq_load_file": (ctypes.c_int, [ctypes.c_char_p, ctypes.c_int, ctypes.POINTER(_c_p)]),
     "stagq_load": (ctypes.c_int, [ctypes.POINTER(_HostStream), ctypes.c_int, ctypes.POINTER(_c_p)]),
+    "stagq_load_stack": (ctypes.c_int, [ctypes.POINTER(ctypes.POINTER(_HostStream)), ctypes.c_int, ctypes.c_int,
+                                        ctypes.POINTER(_c_p)]),
     "stagq_gemv": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, _c_p, _c_p]),
     "stagq_gemv_n": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _c_p]),
     "stagq_gemv_ex": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _u32, _c_p]),
+    "stagq_gemv_scaled": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _c_p, _u32, _c_p]),
     "stagq_gemv_host": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _c_p]),
     "stagq_gemv_host_noalloc": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _c_p]),
     "stagq_decode_levels": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, _c_p]),
     "stagq_bytes": (_i64, [_c_p, ctypes.c_int, ctypes.c_int]),
     "stagq_info": (ctypes.c_int, [_c_p, ctypes.POINTER(_Info)]),
     "stagq_check": (ctypes.c_int, [_c_p]),
+    "stagq_debug_stall": (ctypes.c_int, [_c_p, _u32]),
+    "stagq_debug_side_record": (ctypes.c_int, [_c_p, ctypes.POINTER(_SideLayout), _c_p, _i64, _c_p, _i64]),
     "stagq_free": (None, [_c_p]),
     "stagq_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "stagq_last_error": (ctypes.c_char_p, []),
@@ -291,6 +302,17 @@ def stagq_load(S: HostStream, device: int = 0) -> Matrix:
     return Matrix(h.value)
 
 
+def stagq_load_stack(streams, device: int = 0) -> Matrix:
+    """One handle for several matrices applied to the same x (q/k/v, gate/up):
+    their rows stacked in order, each with its own codebooks. y of a GEMV is
+    the members' outputs one after the other."""
+    cs = [S._c() for S in streams]
+    arr = (ctypes.POINTER(_HostStream) * len(cs))(*[ctypes.pointer(c) for c in cs])
+    h = ctypes.c_void_p()
+    _check(lib().stagq_load_stack(arr, len(cs), device, ctypes.byref(h)), "stagq_load_stack")
+    return Matrix(h.value)
+
+
 def stagq_load_file(path: str, device: int = 0) -> Matrix:
     h = ctypes.c_void_p()
     _check(lib().stagq_load_file(path.encode(), device, ctypes.byref(h)), "stagq_load_file")
@@ -344,6 +366,16 @@ def stagq_gemv_ex(m: Matrix, bits: int, x, y, n: int = 1, flags: int = 0, stream
                                _stream_ptr(stream)), "stagq_gemv_ex")
 
 
+def stagq_gemv_scaled(m: Matrix, bits: int, x, in_scale, y, n: int = 1, flags: int = 0, stream=None) -> None:
+    """y = W_hat (x * in_scale): in_scale a CUDA fp32 tensor [inp] (the
+    inverse activation scale 1/a), x fp16 [n, inp], y fp16 or fp32 [n, out]."""
+    _check_gemv_args(m, x, y, n, bool(flags & STAGQ_Y_F32))
+    _check_device_tensor(in_scale, "in_scale", "float32", m.inp, m.device)
+    _check_on_device(in_scale, "in_scale", m.device)
+    _check(lib().stagq_gemv_scaled(m.handle, bits, x.data_ptr(), n, in_scale.data_ptr(), y.data_ptr(), flags,
+                                   _stream_ptr(stream)), "stagq_gemv_scaled")
+
+
 def stagq_gemv(m: Matrix, bits: int, x, y, stream=None) -> None:
     _check_gemv_args(m, x, y, 1, False)
     _check(lib().stagq_gemv(m.handle, bits, x.data_ptr(), y.data_ptr(), _stream_ptr(stream)), "stagq_gemv")
@@ -389,6 +421,23 @@ def stagq_bytes(m: Matrix, bits: int, n: int = 1) -> int:
 def stagq_check(m: Matrix) -> None:
     """Synchronise the handle's device and raise on any pending CUDA error."""
     _check(lib().stagq_check(m.handle), "stagq_check")
+
+
+def stagq_debug_stall(m: Matrix, stall_ns: int) -> None:
+    """Test hook: launches on m take one bounded wait of stall_ns that runs out (0: off)."""
+    _check(lib().stagq_debug_stall(m.handle, int(stall_ns)), "stagq_debug_stall")
+
+
+def stagq_debug_side_record(m: Matrix):
+    """Test hook: the layout of the two device cuts of the side record and
+    their bytes, copied to host memory: (layout dict, cut, cut1)."""
+    lay = _SideLayout()
+    _check(lib().stagq_debug_side_record(m.handle, ctypes.byref(lay), None, 0, None, 0), "stagq_debug_side_record")
+    cut = np.empty(lay.grid * lay.stride, np.uint8)
+    cut1 = np.empty(lay.grid1 * lay.stride1, np.uint8)
+    _check(lib().stagq_debug_side_record(m.handle, ctypes.byref(lay), cut.ctypes.data, cut.size, cut1.ctypes.data,
+                                         cut1.size), "stagq_debug_side_record")
+    return {k: getattr(lay, k) for k, _ in _SideLayout._fields_}, cut, cut1
 
 
 def stagq_free(m: Matrix) -> None:

@@ -12,6 +12,7 @@
 
 #include "device_matrix.hpp"
 #include "host_common.hpp"
+#include "layout.cuh"
 #include "stream.hpp"
 
 struct stagq_matrix {
@@ -49,22 +50,28 @@ struct DeviceGuard {
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Per-precision (lo_M, s_M c_M) for the 256 pairs, Eq. (10) in fp64, stored fp32.
-// and, per precision, lo - lo_M of every pair: at a post-grid entry the main
+// Per-precision (lo_M, s_M c_M) for the 256 pairs of each stacked member
+// (its own two codebooks, Section 3.1), Eq. (10) in fp64, stored fp32; and per
+// precision and member lo - lo_M of every pair: at a post-grid entry the main
 // stream decodes lo_M + s q (zero planes), the reconstruction is lo + s q + r,
-// so the correction is r + (lo - lo_M).
-void build_tables(const stagq_host_stream* s, std::vector<float2>& t, std::vector<float>& dlo) {
-  const int N = 2 + s->n_planes;
-  t.assign((size_t)(N - 1) * 256, make_float2(0.f, 0.f));
-  dlo.assign((size_t)(N - 1) * 256, 0.f);
+// so the correction is r + (lo - lo_M). Layout [M - 2][member][pair].
+void build_tables(const stagq_host_stream* const* members, int nmem, std::vector<float2>& t,
+                  std::vector<float>& dlo) {
+  const int N = 2 + members[0]->n_planes;
+  t.assign((size_t)(N - 1) * nmem * 256, make_float2(0.f, 0.f));
+  dlo.assign((size_t)(N - 1) * nmem * 256, 0.f);
   for (int M = 2; M <= N; ++M) {
-    for (int p = 0; p < 256; ++p) {
-      const double sp = std::exp2(half_to_double(s->codebook_log2s[p >> 4]));
-      const double lo = half_to_double(s->codebook_lo_over_s[p & 15]) * sp;
-      const double sM = sp / std::ldexp(1.0, M - 2);
-      const double loM = lo - sp * (std::ldexp(1.0, M - 2) - 1.0) / std::ldexp(1.0, M - 1);
-      t[(size_t)(M - 2) * 256 + p] = make_float2((float)loM, (float)(sM * composite_factor(M)));
-      dlo[(size_t)(M - 2) * 256 + p] = (float)(lo - loM);
+    for (int j = 0; j < nmem; ++j) {
+      const stagq_host_stream* s = members[j];
+      for (int p = 0; p < 256; ++p) {
+        const double sp = std::exp2(half_to_double(s->codebook_log2s[p >> 4]));
+        const double lo = half_to_double(s->codebook_lo_over_s[p & 15]) * sp;
+        const double sM = sp / std::ldexp(1.0, M - 2);
+        const double loM = lo - sp * (std::ldexp(1.0, M - 2) - 1.0) / std::ldexp(1.0, M - 1);
+        const size_t i = ((size_t)(M - 2) * nmem + j) * 256 + p;
+        t[i] = make_float2((float)loM, (float)(sM * composite_factor(M)));
+        dlo[i] = (float)(lo - loM);
+      }
     }
   }
 }
@@ -84,11 +91,13 @@ namespace {
 constexpr uint16_t kColMask = 0x7FFF;  // side-record column without the post-grid flag
 }
 
-extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* out) {
-  if (!out) return fail(STAGQ_EINVAL, "stagq_load: null output handle");
-  *out = nullptr;
-  int st = validate_stream(s);
-  if (st) return st;
+namespace {
+
+// Copies a (possibly stacked) stream to the device. `s` is the whole stream
+// (members' rows stacked in order); members[j] are the member streams, whose
+// codebooks give each member its own pair tables (nmem = 1: s itself).
+int load_impl(const stagq_host_stream* s, const stagq_host_stream* const* members, int nmem, int device,
+              stagq_handle* out) {
   int ndev = 0;
   cudaError_t e = cudaGetDeviceCount(&ndev);
   if (e != cudaSuccess || ndev == 0) return fail(STAGQ_ENODEV, "no CUDA device");
@@ -106,8 +115,8 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   const size_t base_bytes = (size_t)(out_ * in / 4), plane_bytes = (size_t)(out_ * in / 8);
   const size_t pair_row = (size_t)(in / s->group), pair_stride = align_up(pair_row, 16);
   const size_t pair_bytes = (size_t)out_ * pair_stride;
-  const size_t tab_bytes = (size_t)(np + 1) * 256 * sizeof(float2);
-  const size_t dlo_bytes = (size_t)(np + 1) * 256 * sizeof(float);
+  const size_t tab_bytes = (size_t)(np + 1) * nmem * 256 * sizeof(float2);
+  const size_t dlo_bytes = (size_t)(np + 1) * nmem * 256 * sizeof(float);
   int has_post = 0;
   for (int64_t e = 0; e < s->nnz; ++e) has_post |= (s->col[e] & STAGQ_SIDE_POST) != 0;
   // Side record cut per CTA of the GEMV grid (see DeviceMatrix::side).
@@ -164,7 +173,7 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
 
   std::vector<float2> tabs;
   std::vector<float> dlo;
-  build_tables(s, tabs, dlo);
+  build_tables(members, nmem, tabs, dlo);
   std::vector<uint8_t> side(side_bytes, 0);
   {
     for (int b = 0; b < grid; ++b) {
@@ -202,7 +211,7 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
     for (int64_t r = 0; r < n; ++r) {
       offs[r] = pos;
       for (int64_t e = s->row_ptr[ra + r]; e < s->row_ptr[ra + r + 1]; ++e)
-        ent[pos++] = (uint32_t)xq_slot_of_column(s->col[e] & kColMask) | (uint32_t)(s->col[e] & STAGQ_SIDE_POST) |
+        ent[pos++] = (uint32_t)(s->col[e] & kColMask) | (uint32_t)(s->col[e] & STAGQ_SIDE_POST) |
                      ((uint32_t)s->val[e] << 16);
     }
     offs[n] = pos;
@@ -255,6 +264,11 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   m.tables = reinterpret_cast<const float2*>(d + o_tab);
   m.dlo = reinterpret_cast<const float*>(d + o_dlo);
   m.has_post = has_post;
+  m.nmem = nmem;
+  for (int j = 0, r = 0; j < kMaxStack; ++j) {  // first row of each member; absent members never start
+    m.mem_row[j] = j < nmem ? r : INT32_MAX;
+    if (j < nmem) r += members[j]->out;
+  }
   m.status = reinterpret_cast<uint32_t*>(d + o_status);
   m.num_sms = prop.multiProcessorCount;
   m.smem_pair_budget = smem_sm / 2 - smem_reserved;
@@ -284,6 +298,76 @@ extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* 
   return STAGQ_OK;
 }
 
+}  // namespace
+
+extern "C" int stagq_load(const stagq_host_stream* s, int device, stagq_handle* out) {
+  if (!out) return fail(STAGQ_EINVAL, "stagq_load: null output handle");
+  *out = nullptr;
+  int st = validate_stream(s);
+  if (st) return st;
+  const stagq_host_stream* members[1] = {s};
+  return load_impl(s, members, 1, device, out);
+}
+
+extern "C" int stagq_load_stack(const stagq_host_stream* const* members, int count, int device, stagq_handle* out) {
+  if (!out) return fail(STAGQ_EINVAL, "stagq_load_stack: null output handle");
+  *out = nullptr;
+  if (!members || count < 1 || count > STAGQ_MAX_STACK) return fail(STAGQ_EINVAL, "count outside 1..STAGQ_MAX_STACK");
+  int64_t out_total = 0, nnz = 0;
+  for (int j = 0; j < count; ++j) {
+    int st = validate_stream(members[j]);
+    if (st) return st;
+    const stagq_host_stream* m = members[j];
+    if (m->in != members[0]->in || m->group != members[0]->group || m->n_planes != members[0]->n_planes)
+      return fail(STAGQ_EINVAL, "stacked members must share in, group and n_planes");
+    out_total += m->out;
+    nnz += m->nnz;
+  }
+  const int64_t in = members[0]->in;
+  const int np = members[0]->n_planes;
+  int st = check_shape(out_total, in, members[0]->group, np);
+  if (st) return st;
+  // The stacked stream: every plane region holds the members' rows in order
+  // (each plane is row-major), then the pair bytes and the side record
+  // (row pointers shifted by the entries of the members before).
+  HostStreamBuffers buf;
+  try {
+    buf.planes.resize((size_t)stagq_stream_plane_bytes((int32_t)out_total, (int32_t)in, np));
+    buf.pair_idx.resize((size_t)(out_total * (in / members[0]->group)));
+    buf.row_ptr.resize((size_t)out_total + 1);
+    buf.col.resize((size_t)nnz);
+    buf.val.resize((size_t)nnz);
+  } catch (...) {
+    return fail(STAGQ_ENOMEM, "host allocation for the stacked stream failed");
+  }
+  int64_t r0 = 0, e0 = 0;
+  const int64_t ngr = in / members[0]->group;
+  buf.row_ptr[0] = 0;
+  for (int j = 0; j < count; ++j) {
+    const stagq_host_stream* m = members[j];
+    const int64_t rows = m->out;
+    std::memcpy(&buf.planes[(size_t)(r0 * in / 4)], m->planes, (size_t)(rows * in / 4));
+    for (int k = 3; k < 3 + np; ++k)
+      std::memcpy(&buf.planes[(size_t)(plane_region_offset(out_total, in, k) + r0 * in / 8)],
+                  m->planes + plane_region_offset(rows, in, k), (size_t)(rows * in / 8));
+    std::memcpy(&buf.pair_idx[(size_t)(r0 * ngr)], m->pair_idx, (size_t)(rows * ngr));
+    for (int64_t r = 0; r < rows; ++r) buf.row_ptr[(size_t)(r0 + r + 1)] = (int32_t)(e0 + m->row_ptr[r + 1]);
+    if (m->nnz) {
+      std::memcpy(&buf.col[(size_t)e0], m->col, (size_t)m->nnz * 2);
+      std::memcpy(&buf.val[(size_t)e0], m->val, (size_t)m->nnz * 2);
+    }
+    r0 += rows;
+    e0 += m->nnz;
+  }
+  stagq_host_stream& v = buf.view;
+  v.out = (int32_t)out_total; v.in = (int32_t)in; v.group = members[0]->group; v.n_planes = np; v.nnz = nnz;
+  std::memcpy(v.codebook_log2s, members[0]->codebook_log2s, 32);      // per member: see build_tables
+  std::memcpy(v.codebook_lo_over_s, members[0]->codebook_lo_over_s, 32);
+  v.planes = buf.planes.data(); v.pair_idx = buf.pair_idx.data(); v.row_ptr = buf.row_ptr.data();
+  v.col = buf.col.data(); v.val = buf.val.data();
+  return load_impl(&v, members, count, device, out);
+}
+
 extern "C" int stagq_load_file(const char* path, int device, stagq_handle* out) {
   HostStreamBuffers buf;
   int st = read_stream_file(path, &buf);
@@ -291,13 +375,17 @@ extern "C" int stagq_load_file(const char* path, int device, stagq_handle* out) 
   return stagq_load(&buf.view, device, out);
 }
 
-extern "C" int stagq_gemv_ex(stagq_handle h, int bits, const void* x, int n, void* y, uint32_t flags,
-                             void* cuda_stream) {
+namespace {
+
+// y = W_hat^(bits) (x .* in_scale) for n vectors; in_scale null = no scale.
+int gemv_impl(stagq_handle h, int bits, const void* x, int n, const float* in_scale, void* y, uint32_t flags,
+              void* cuda_stream) {
   int st = check_handle_bits(h, bits);
   if (st) return st;
   if (!x || !y) return fail(STAGQ_EINVAL, "null x or y");
   if (n < 1 || n > STAGQ_MAX_BATCH) return fail(STAGQ_EINVAL, "n outside 1..STAGQ_MAX_BATCH");
   if (reinterpret_cast<uintptr_t>(x) % 16) return fail(STAGQ_EINVAL, "x must be 16-byte aligned");
+  if (in_scale && reinterpret_cast<uintptr_t>(in_scale) % 16) return fail(STAGQ_EINVAL, "in_scale must be 16-byte aligned");
   if (flags & ~(STAGQ_Y_F32 | STAGQ_KERNEL_GENERAL | STAGQ_KERNEL_SINGLE)) return fail(STAGQ_EINVAL, "unknown flags");
   const bool force_general = flags & STAGQ_KERNEL_GENERAL, force_single = flags & STAGQ_KERNEL_SINGLE;
   if (force_general && force_single) return fail(STAGQ_EINVAL, "both kernels forced");
@@ -309,12 +397,12 @@ extern "C" int stagq_gemv_ex(stagq_handle h, int bits, const void* x, int n, voi
   const int yf32 = (flags & STAGQ_Y_F32) ? 1 : 0;
   const size_t ysz = yf32 ? 4 : 2;
   if (force_single || (n == 1 && !force_general && h->plan1_ok[bits] && h->prefer1[bits])) {
-    cudaError_t e = launch_gemv1(h->dm, h->plan1[bits], bits, x, y, yf32, stream);
+    cudaError_t e = launch_gemv1(h->dm, h->plan1[bits], bits, x, in_scale, y, yf32, stream);
     if (e != cudaSuccess) return cuda_fail(e, "GEMV launch");
     return STAGQ_OK;
   }
   if (h->plan_ok[bits][n]) {  // one launch: the weights are read once for all n vectors
-    cudaError_t e = launch_gemv(h->dm, h->plan[bits][n], bits, x, y, yf32, stream);
+    cudaError_t e = launch_gemv(h->dm, h->plan[bits][n], bits, x, in_scale, y, yf32, stream);
     if (e != cudaSuccess) return cuda_fail(e, "GEMV launch");
     return STAGQ_OK;
   }
@@ -322,10 +410,23 @@ extern "C" int stagq_gemv_ex(stagq_handle h, int bits, const void* x, int n, voi
   for (int j = 0; j < n; ++j) {  // shapes whose n-vector plan does not fit: one launch per vector
     const void* xj = static_cast<const uint8_t*>(x) + (size_t)j * h->dm.in * 2;
     void* yj = static_cast<uint8_t*>(y) + (size_t)j * h->dm.out * ysz;
-    cudaError_t e = launch_gemv(h->dm, h->plan[bits][1], bits, xj, yj, yf32, stream);
+    cudaError_t e = launch_gemv(h->dm, h->plan[bits][1], bits, xj, in_scale, yj, yf32, stream);
     if (e != cudaSuccess) return cuda_fail(e, "GEMV launch");
   }
   return STAGQ_OK;
+}
+
+}  // namespace
+
+extern "C" int stagq_gemv_ex(stagq_handle h, int bits, const void* x, int n, void* y, uint32_t flags,
+                             void* cuda_stream) {
+  return gemv_impl(h, bits, x, n, nullptr, y, flags, cuda_stream);
+}
+
+extern "C" int stagq_gemv_scaled(stagq_handle h, int bits, const void* x, int n, const float* in_scale, void* y,
+                                 uint32_t flags, void* cuda_stream) {
+  if (!in_scale) return fail(STAGQ_EINVAL, "null in_scale");
+  return gemv_impl(h, bits, x, n, in_scale, y, flags, cuda_stream);
 }
 
 extern "C" int stagq_gemv(stagq_handle h, int bits, const void* x, void* y, void* cuda_stream) {
@@ -402,6 +503,39 @@ extern "C" int stagq_check(stagq_handle h) {
     if (e != cudaSuccess) return cuda_fail(e, "status reset");
     return fail(STAGQ_ETIMEOUT, "a GEMV kernel gave up waiting for its copies (status " + std::to_string(word) + ")");
   }
+  return STAGQ_OK;
+}
+
+extern "C" int stagq_debug_stall(stagq_handle h, uint32_t stall_ns) {
+  if (!h) return fail(STAGQ_EINVAL, "null handle");
+  h->dm.debug_stall_ns = stall_ns;
+  return STAGQ_OK;
+}
+
+extern "C" int stagq_debug_side_record(stagq_handle h, stagq_side_layout_t* layout, void* cut_host, int64_t cut_bytes,
+                                       void* cut1_host, int64_t cut1_bytes) {
+  if (!h || !layout) return fail(STAGQ_EINVAL, "null argument");
+  const DeviceMatrix& m = h->dm;
+  const int KW = k_slices(m.in), RG = row_groups(KW);
+  const int rows_cap = (m.out + m.side_grid - 1) / m.side_grid;
+  layout->grid = m.side_grid;
+  layout->stride = m.side_stride;
+  layout->ent_off = m.side_ent_off;
+  layout->row_groups = RG;
+  layout->k_slices = KW;
+  layout->class_rows = (rows_cap + RG - 1) / RG;
+  layout->grid1 = m.side1_grid;
+  layout->stride1 = m.side1_stride;
+  layout->ent_off1 = m.side1_ent_off;
+  const int64_t need = (int64_t)m.side_grid * m.side_stride, need1 = (int64_t)m.side1_grid * m.side1_stride;
+  if ((cut_host && cut_bytes < need) || (cut1_host && cut1_bytes < need1))
+    return fail(STAGQ_EINVAL, "host buffer smaller than the cut");
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return fail(STAGQ_ECUDA, "cudaSetDevice failed");
+  cudaError_t e = cudaSuccess;
+  if (cut_host) e = cudaMemcpy(cut_host, m.side, (size_t)need, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && cut1_host) e = cudaMemcpy(cut1_host, m.side1, (size_t)need1, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "copy of the side record");
   return STAGQ_OK;
 }
 

@@ -11,6 +11,7 @@ constexpr int kMaxSlots = 8;            // shared-memory ring slots
 constexpr int kMaxRowsPerCta = 2048;    // rows of one CTA
 constexpr int kSliceWeights = 2048;     // K weights per K slice (one warp: 32 lanes x 64)
 constexpr int64_t kTwoCtaWeightsPerSm = 256 * 1024;  // from this many weights per SM on, two GEMV CTAs per SM
+constexpr int kMaxStack = 4;            // member matrices of a stacked handle (STAGQ_MAX_STACK)
 
 // Row groups of a CTA with KW K slices: up to 8 warps in all, at least one group.
 inline int row_groups(int KW) { return KW <= 4 ? 8 / KW : 1; }
@@ -31,6 +32,13 @@ __host__ __device__ inline int column_of_xq_slot(int slot) {
   return c * 64 + ((piece_slot - c) & 7) * 8 + (slot & 7);
 }
 
+struct DeviceMatrix;
+// Offset of the pair table of the member that holds global row `row` (a
+// multiple of 256 entries).
+__host__ __device__ inline int member_table_offset(const int32_t (&mem_row)[kMaxStack], int row) {
+  return 256 * ((row >= mem_row[1]) + (row >= mem_row[2]) + (row >= mem_row[3]));
+}
+
 struct DeviceMatrix {
   int32_t out, in, group, n_planes;
   int64_t nnz;
@@ -47,17 +55,23 @@ struct DeviceMatrix {
   // whose value is the residual r) start at side_ent_off.
   const uint8_t* side;
   int32_t side_stride, side_ent_off, side_grid;
-  // The same side record cut for the single-vector kernel (gemv1.cu): per CTA
-  // of its grid (side1_grid CTAs, one per SM), side1_stride bytes: int32
+  // The same side record cut for the single-vector kernel (gemv1.cu): per
+  // CTA of its grid (side1_grid CTAs, one per SM), side1_stride bytes: int32
   // offsets [rows + 1] (where each local row's entries start, then the end),
-  // and from side1_ent_off the entries (xq_slot_of_column(column) | fp16 value
-  // << 16) in (row, column) order; side1_max entries at most per CTA.
+  // and from side1_ent_off the entries (column | post-grid flag << 15 | fp16
+  // value << 16) in (row, column) order; side1_max entries at most per CTA.
   const uint8_t* side1;
   int32_t side1_stride, side1_ent_off, side1_grid, side1_max;
-  const float2* tables;       // [n_planes+1][256]: (lo_M, s_M * c_M) for M = 2..2+n_planes
-  const float* dlo;           // [n_planes+1][256]: lo - lo_M, the correction of a post-grid entry beside r
+  const float2* tables;       // [n_planes+1][nmem][256]: (lo_M, s_M * c_M) for M = 2..2+n_planes
+  const float* dlo;           // [n_planes+1][nmem][256]: lo - lo_M, the correction of a post-grid entry beside r
+  // A stacked handle holds nmem member matrices (their rows in order, each
+  // with its own codebooks); mem_row[j] is member j's first row (INT32_MAX for
+  // j >= nmem), so a row's member is the number of mem_row[1..] <= row.
+  int32_t nmem;
+  int32_t mem_row[kMaxStack];
   int32_t has_post;           // the side record holds post-grid entries (bit 15 of the column / slot)
   uint32_t* status;           // nonzero once a kernel gave up waiting for its copies
+  uint32_t debug_stall_ns;    // test hook: launches include one bounded wait of this length that runs out
   int num_sms;
   int smem_limit;             // opt-in shared memory per block
   int smem_pair_budget;       // shared memory per block that still lets two blocks share an SM
@@ -76,6 +90,7 @@ struct GemvPlan {
   int group_shift;       // log2(group)
   int pair_stride;
   int pdl;               // launch with programmatic dependent launch
+  int nmem;              // stacked members (pair tables)
   int nb;                // activation vectors per launch (1..4; the weights are read once)
 };
 
@@ -91,14 +106,16 @@ struct Gemv1Plan {
   int group_shift;       // log2(group)
   int pair_stride;
   int pdl;               // launch with programmatic dependent launch
+  int nmem;              // stacked members (pair tables)
 };
 
 // Plan for the single-vector kernel at `bits`; false if it cannot be planned
 // (the general kernel then serves n = 1 too).
 bool make_plan1(const DeviceMatrix& m, int bits, Gemv1Plan* plan);
 int gemv1_grid(int out, int num_sms);
-cudaError_t launch_gemv1(const DeviceMatrix& m, const Gemv1Plan& plan, int bits, const void* x, void* y, int y_f32,
-                         cudaStream_t stream);
+// in_scale: null, or device fp32 [in] multiplying x channel by channel first.
+cudaError_t launch_gemv1(const DeviceMatrix& m, const Gemv1Plan& plan, int bits, const void* x, const float* in_scale,
+                         void* y, int y_f32, cudaStream_t stream);
 
 // Plan for a GEMV at `bits` with `nb` activation vectors; false if the shape
 // cannot be planned.
@@ -109,8 +126,8 @@ uint32_t gemv_smem_bytes(const GemvPlan& plan, int in, int bits);
 
 // y = W_hat^(bits) x for plan.nb vectors (x [nb][in], y [nb][out]). y is fp16
 // (y_f32 = 0) or fp32.
-cudaError_t launch_gemv(const DeviceMatrix& m, const GemvPlan& plan, int bits, const void* x, void* y,
-                        int y_f32, cudaStream_t stream);
+cudaError_t launch_gemv(const DeviceMatrix& m, const GemvPlan& plan, int bits, const void* x, const float* in_scale,
+                        void* y, int y_f32, cudaStream_t stream);
 
 // u_M per weight into u (device [out*in]).
 cudaError_t launch_decode_levels(const DeviceMatrix& m, int bits, uint8_t* u, cudaStream_t stream);

@@ -85,6 +85,7 @@ struct GemvKernelArgs {
   const float2* table;  // (lo_M, s_M c_M) of this precision
   const float* dlo;     // lo - lo_M of this precision (post-grid entries)
   const __half* x;
+  const float* in_scale;  // SC: per-channel multiplier of x (the inverse activation scale)
   void* y;
   int y_f32;
 };
@@ -115,11 +116,11 @@ __host__ __device__ inline SmemLayout smem_layout(const GemvPlan& p, int in, int
   SmemLayout L;
   const uint32_t nchunk = in / kChunk, BR = p.br;
   uint32_t o = 0;
-  L.bar = o; o += 8 * (kMaxSlots + 1);  // full[slot] + side/table barrier
+  L.bar = o; o += 8 * (kMaxSlots + 2);  // full[slot] + side/table barrier + a test barrier nothing completes
   L.cnt = o; o += 4 * kMaxSlots;         // warps done with the slot's blocks so far
   L.last = o; o += 4 * kMaxSlots;        // last block issued into the slot
   o = align_up_u32(o, 16);
-  L.tab = o; o += 256 * 8;
+  L.tab = o; o += 256 * 8 * (uint32_t)p.nmem;  // the pair table of each stacked member
   L.xq = o; o += 2u * in * p.nb;        // x~ of each of the nb vectors
   L.xscale = o; o += 4u * nchunk * p.nb;
   L.xsum = o; o += 4u * nchunk * p.nb;
@@ -173,8 +174,8 @@ __device__ __forceinline__ float group_affine(const float2* tab, uint32_t pairs,
 
 template <int M, int NR, int G>
 __device__ __forceinline__ void rows_dot(const uint32_t (&X)[32], float xs, const float (&xsg)[G], const uint8_t* sb,
-                                         RowOffsets off, RowOffsets step, uint32_t plane_stride, const float2* tab,
-                                         float (&v)[NR], float (&lo)[NR][G]) {
+                                         RowOffsets off, RowOffsets step, uint32_t plane_stride,
+                                         const float2* const (&tb)[NR], float (&v)[NR], float (&lo)[NR][G]) {
 #pragma unroll
   for (int u = 0; u < NR; ++u) {
     const uint4 b4 = *reinterpret_cast<const uint4*>(sb + off.b + u * step.b);
@@ -185,7 +186,7 @@ __device__ __forceinline__ void rows_dot(const uint32_t (&X)[32], float xs, cons
       Pw[k] = *reinterpret_cast<const uint2*>(sb + off.p + u * step.p + k * plane_stride);
     int tot[G];
     chunk_dot_g<M, G>(X, B, Pw, tot);
-    v[u] = group_affine<G>(tab, load_pairs<G>(sb + off.g + u * step.g), tot, xs, xsg, lo[u]);
+    v[u] = group_affine<G>(tb[u], load_pairs<G>(sb + off.g + u * step.g), tot, xs, xsg, lo[u]);
   }
 }
 
@@ -198,7 +199,7 @@ template <int M, int NR, int NB, int G>
 __device__ __forceinline__ void rows_dot_nb(const int16_t* xq, const float* xscale, const float* xsum,
                                             const float* xsum16, int in, int nchunk, int cc, bool active,
                                             const uint8_t* sb, RowOffsets off, RowOffsets step, uint32_t plane_stride,
-                                            const float2* tab, float (&v)[NB][NR], float (&lo)[NR][G]) {
+                                            const float2* const (&tb)[NR], float (&v)[NB][NR], float (&lo)[NR][G]) {
   uint32_t B[NR][4];
   uint2 Pw[NR][M > 2 ? M - 2 : 1];
   uint32_t pr[NR];
@@ -240,7 +241,7 @@ __device__ __forceinline__ void rows_dot_nb(const int16_t* xq, const float* xsca
     for (int u = 0; u < NR; ++u) {
       int tot[G];
       chunk_dot_g<M, G>(X, B[u], Pw[u], tot);
-      v[j][u] = group_affine<G>(tab, pr[u], tot, xs, xsg, lo[u]);
+      v[j][u] = group_affine<G>(tb[u], pr[u], tot, xs, xsg, lo[u]);
     }
   }
 }
@@ -329,12 +330,17 @@ __device__ __forceinline__ void block_rows(const uint32_t (&X)[32], float xs, co
                                            int nchunk, int cc, bool active, const uint8_t* sb, RowOffsets off,
                                            RowOffsets step, uint32_t plane_stride, const float2* tab, int mine,
                                            const int32_t* o, const uint32_t* ents, float* lo_w, int lane, int gs,
-                                           const float* dlo, float* pout, int pstep) {
+                                           const float* dlo, float* pout, int pstep,
+                                           const int32_t (&mem_row)[kMaxStack], int grow0, int rstep) {
+  // global row of the warp's row u: grow0 + rstep u; each row reads its member's pair table
+  const float2* tb[NR];
+#pragma unroll
+  for (int u = 0; u < NR; ++u) tb[u] = tab + member_table_offset(mem_row, grow0 + rstep * u);
   float v[NB][NR], lo[NR][G];
   if constexpr (NB == 1) {
-    rows_dot<M, NR, G>(X, xs, xsg, sb, off, step, plane_stride, tab, v[0], lo);
+    rows_dot<M, NR, G>(X, xs, xsg, sb, off, step, plane_stride, tb, v[0], lo);
   } else {
-    rows_dot_nb<M, NR, NB, G>(xq, xscale, xsum, xsum16, in, nchunk, cc, active, sb, off, step, plane_stride, tab, v,
+    rows_dot_nb<M, NR, NB, G>(xq, xscale, xsum, xsum16, in, nchunk, cc, active, sb, off, step, plane_stride, tb, v,
                               lo);
   }
 #pragma unroll
@@ -344,7 +350,8 @@ __device__ __forceinline__ void block_rows(const uint32_t (&X)[32], float xs, co
   __syncwarp();
   const int ur = lane / (32 / NR);
   PostCtx pc = {nullptr, 0u, nullptr};
-  if constexpr (POST) pc = {sb + off.g - ((cc * kChunk) >> gs), step.g, dlo};  // read by post-grid entries only
+  if constexpr (POST)  // read by post-grid entries only; lane group ur holds row ur
+    pc = {sb + off.g - ((cc * kChunk) >> gs), step.g, dlo + member_table_offset(mem_row, grow0 + rstep * ur)};
   if constexpr (NB == 1) {
     side_record<NR, G, POST>(o[ur < mine ? ur : mine], o[ur + 1 < mine ? ur + 1 : mine], ents, xq, xscale, lo_w, lane, gs,
                        pc, v[0]);
@@ -359,7 +366,7 @@ __device__ __forceinline__ void block_rows(const uint32_t (&X)[32], float xs, co
   }
 }
 
-template <int M, int UP, int NB, int G, bool POST>
+template <int M, int UP, int NB, int G, bool POST, bool SC>
 __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKernelArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const GemvPlan& P = a.plan;
@@ -420,9 +427,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
       last[s] = -1;
     }
     mbar_init(side_bar, 1);
+    mbar_init(side_bar + 8, 1);
     fence_barrier_init();
-    mbar_arrive_expect_tx(side_bar, 256 * 8 + (P.stage_side ? (uint32_t)a.m.side_stride : 0u));
-    bulk_load(sbase + L.tab, a.table, 256 * 8, side_bar);
+    mbar_arrive_expect_tx(side_bar, 256 * 8 * (uint32_t)P.nmem + (P.stage_side ? (uint32_t)a.m.side_stride : 0u));
+    bulk_load(sbase + L.tab, a.table, 256 * 8 * (uint32_t)P.nmem, side_bar);
     if (P.stage_side) bulk_load(sbase + L.side, side_g, (uint32_t)a.m.side_stride, side_bar);
     issue_block(0, 0);
   }
@@ -435,13 +443,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
   // exactly; rounding to nearest even goes through the 1.5 * 2^23 shifter (the
   // low 16 bits of the sum are the two's-complement integer).
   {
-    constexpr float kShift = 12582912.0f;
     constexpr int kBatch = 4;
     const int tpv = 4 * nchunk;  // tasks per vector
     const int ntask = tpv * NB;
     const uint4* x4 = reinterpret_cast<const uint4*>(a.x);
+    const float4* s4 = reinterpret_cast<const float4*>(a.in_scale);
     for (int t0 = 0; t0 < ntask; t0 += kBatch * nthreads) {
       uint4 raw[kBatch][2];
+      float4 sv[kBatch][4];
 #pragma unroll
       for (int q = 0; q < kBatch; ++q) {
         const int t = t0 + q * nthreads + tid;
@@ -449,6 +458,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
         if (t < ntask) {  // x is [NB][in]: task t of the flat list reads 16 values from 16 t on
           raw[q][0] = __ldg(x4 + 2 * t);
           raw[q][1] = __ldg(x4 + 2 * t + 1);
+        }
+        if constexpr (SC) {  // the scale of the task's channels (16 (t mod tpv) on)
+          const int ts = t < ntask ? t % tpv : 0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) sv[q][k] = __ldg(s4 + 4 * ts + k);
         }
       }
       if (t0 == 0 && tid == 0)
@@ -458,34 +472,17 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
         const int tw = t0 + q * nthreads + warp * 32;  // first task of this warp
         if (tw >= ntask) break;                         // warp-uniform
         const int t = tw + lane;
-        const uint32_t* w = reinterpret_cast<const uint32_t*>(raw[q]);
-        __half2 m2 = __habs2(*reinterpret_cast<const __half2*>(&w[0]));
-#pragma unroll
-        for (int k = 1; k < 8; ++k) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __half2*>(&w[k])));
-        float mx = fmaxf(__low2float(m2), __high2float(m2));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-        const int e = mx > 0.f ? 14 - ((int)((__float_as_uint(mx) >> 23) & 0xFF) - 127) : 0;
-        const float sc = __int_as_float((127 + e) << 23);
         uint32_t Q[8];
-        int sumq = 0;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
-          Q[k] = __byte_perm(__float_as_uint(fmaf(f.x, sc, kShift)), __float_as_uint(fmaf(f.y, sc, kShift)), 0x5410);
-          sumq = dp2a_lo(Q[k], 0x0101u, sumq);
-        }
-        const int sum16 = sumq;
-        sumq += __shfl_xor_sync(kFull, sumq, 1);
-        sumq += __shfl_xor_sync(kFull, sumq, 2);
+        float xs_c;
+        int sum16, sumq;
+        convert_x_task<SC>(raw[q], sv[q], Q, xs_c, sum16, sumq);
         if (t < ntask) {
           const int j = t / tpv, tt = t - j * tpv;  // vector, task within it
           uint4* dst = reinterpret_cast<uint4*>(xq + j * in);
           dst[xq_piece(tt >> 2, 2 * (tt & 3))] = make_uint4(Q[0], Q[1], Q[2], Q[3]);
           dst[xq_piece(tt >> 2, 2 * (tt & 3) + 1)] = make_uint4(Q[4], Q[5], Q[6], Q[7]);
-          if constexpr (G > 1) xsum16[t] = __int_as_float((127 - e) << 23) * (float)sum16;  // t = 4 (j nchunk + c) + q
+          if constexpr (G > 1) xsum16[t] = xs_c * (float)sum16;  // t = 4 (j nchunk + c) + q
           if ((tt & 3) == 0) {
-            const float xs_c = __int_as_float((127 - e) << 23);
             xscale[j * nchunk + (tt >> 2)] = xs_c;
             xsum[j * nchunk + (tt >> 2)] = xs_c * (float)sumq;
           }
@@ -531,6 +528,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
   // The lanes of a warp leave together: the block code below uses full-warp
   // shuffles and __syncwarp.
   bool ok = __all_sync(kFull, mbar_wait(side_bar, 0, kWaitLimitNs));
+  // Test hook (stagq_debug_stall): every warp takes one bounded wait that runs
+  // out, so that the give-up path below runs on a healthy launch.
+  if (a.m.debug_stall_ns && !__all_sync(kFull, mbar_wait(side_bar + 8, 0, a.m.debug_stall_ns))) ok = false;
   const uint8_t* ring_g = smem + L.ring;
   int slot = 0;
   uint32_t phase = 0, round = 0;
@@ -549,13 +549,14 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(const GemvKerne
     const int mine = nr == BR ? UP : (nr > rg ? (nr - rg + RG - 1) / RG : 0);
     if (mine == UP || 2 * mine > UP) {
       block_rows<M, UP, NB, G, POST>(X, xs, xsg, xq, xscale, xsum, xsum16, in, nchunk, cc, active, sb, off, step,
-                               plane_stride, tab, mine, o, ents, lo_w, lane, P.group_shift, a.dlo, pout, pstep);
+                               plane_stride, tab, mine, o, ents, lo_w, lane, P.group_shift, a.dlo, pout, pstep,
+                               a.m.mem_row, r0 + b * BR + rg, RG);
     } else {
       for (int u = 0; u < mine; ++u) {
         const RowOffsets ou = {off.b + u * step.b, off.p + u * step.p, off.g + u * step.g};
         block_rows<M, 1, NB, G, POST>(X, xs, xsg, xq, xscale, xsum, xsum16, in, nchunk, cc, active, sb, ou, step,
                                 plane_stride, tab, 1, o + u, ents, lo_w, lane, P.group_shift, a.dlo, pout + u * pstep,
-                                pstep);
+                                pstep, a.m.mem_row, r0 + b * BR + rg + RG * u, RG);
         __syncwarp();  // lo_w is rewritten by the next row
       }
     }
@@ -624,11 +625,11 @@ __global__ void decode_levels_kernel(const DeviceMatrix m, uint8_t* u) {
 cudaError_t ensure_smem(const void* kern, int key, size_t smem) {
   constexpr int kMaxDev = 64;
   static std::mutex mu;
-  static size_t granted[kMaxDev][384] = {};  // key < 360: (M - 2, rows per warp, vectors, groups, post)
+  static size_t granted[kMaxDev][768] = {};  // key < 720: (M - 2, rows per warp, vectors, groups, post, scaled)
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (dev < 0 || dev >= kMaxDev || key < 0 || key >= 384) return cudaErrorInvalidValue;
+  if (dev < 0 || dev >= kMaxDev || key < 0 || key >= 768) return cudaErrorInvalidValue;
   std::lock_guard<std::mutex> lock(mu);
   if (granted[dev][key] >= smem) return cudaSuccess;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -640,21 +641,22 @@ cudaError_t ensure_smem(const void* kern, int key, size_t smem) {
   return err;
 }
 
-template <int M, int UP, int NB, int G>
-cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const void* x, void* y, int y_f32,
-                           cudaStream_t stream) {
+template <int M, int UP, int NB, int G, bool SC>
+cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const void* x, const float* in_scale, void* y,
+                           int y_f32, cudaStream_t stream) {
   GemvKernelArgs a;
   a.m = m;
   a.plan = plan;
-  a.table = m.tables + 256 * (M - 2);
-  a.dlo = m.dlo + 256 * (M - 2);
+  a.table = m.tables + 256 * m.nmem * (M - 2);
+  a.dlo = m.dlo + 256 * m.nmem * (M - 2);
   a.x = reinterpret_cast<const __half*>(x);
+  a.in_scale = in_scale;
   a.y = y;
   a.y_f32 = y_f32;
   const SmemLayout L = smem_layout(plan, m.in, M);
-  auto kern = m.has_post ? gemv_kernel<M, UP, NB, G, true> : gemv_kernel<M, UP, NB, G, false>;
-  const int key = ((((M - 2) * 3 + (UP == 4 ? 2 : UP - 1)) * 4 + (NB - 1)) * 3 + (G == 4 ? 2 : G - 1)) * 2 +
-                  (m.has_post ? 1 : 0);
+  auto kern = m.has_post ? gemv_kernel<M, UP, NB, G, true, SC> : gemv_kernel<M, UP, NB, G, false, SC>;
+  const int key = (((((M - 2) * 3 + (UP == 4 ? 2 : UP - 1)) * 4 + (NB - 1)) * 3 + (G == 4 ? 2 : G - 1)) * 2 +
+                   (m.has_post ? 1 : 0)) * 2 + (SC ? 1 : 0);
   cudaError_t err = ensure_smem(reinterpret_cast<const void*>(kern), key, L.total);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -670,9 +672,9 @@ cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const vo
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <int M>
-cudaError_t launch_gemv_m(const DeviceMatrix& m, const GemvPlan& plan, const void* x, void* y, int y_f32,
-                          cudaStream_t stream) {
+template <int M, bool SC>
+cudaError_t launch_gemv_m(const DeviceMatrix& m, const GemvPlan& plan, const void* x, const float* in_scale, void* y,
+                          int y_f32, cudaStream_t stream) {
   // Instances the planner can select (see make_plan): more vectors or deeper
   // reads take fewer rows per warp, so that the registers do not spill;
   // groups below 64 weights take one row per warp.
@@ -680,44 +682,51 @@ cudaError_t launch_gemv_m(const DeviceMatrix& m, const GemvPlan& plan, const voi
   if (G > 1) {
     if (plan.up != 1) return cudaErrorInvalidValue;
     switch (G * 8 + plan.nb) {
-      case 16 + 1: return launch_gemv_mu<M, 1, 1, 2>(m, plan, x, y, y_f32, stream);
-      case 16 + 2: return launch_gemv_mu<M, 1, 2, 2>(m, plan, x, y, y_f32, stream);
-      case 16 + 3: return launch_gemv_mu<M, 1, 3, 2>(m, plan, x, y, y_f32, stream);
-      case 16 + 4: return launch_gemv_mu<M, 1, 4, 2>(m, plan, x, y, y_f32, stream);
-      case 32 + 1: return launch_gemv_mu<M, 1, 1, 4>(m, plan, x, y, y_f32, stream);
-      case 32 + 2: return launch_gemv_mu<M, 1, 2, 4>(m, plan, x, y, y_f32, stream);
-      case 32 + 3: return launch_gemv_mu<M, 1, 3, 4>(m, plan, x, y, y_f32, stream);
-      case 32 + 4: return launch_gemv_mu<M, 1, 4, 4>(m, plan, x, y, y_f32, stream);
+      case 16 + 1: return launch_gemv_mu<M, 1, 1, 2, SC>(m, plan, x, in_scale, y, y_f32, stream);
+      case 16 + 2: return launch_gemv_mu<M, 1, 2, 2, SC>(m, plan, x, in_scale, y, y_f32, stream);
+      case 16 + 3: return launch_gemv_mu<M, 1, 3, 2, SC>(m, plan, x, in_scale, y, y_f32, stream);
+      case 16 + 4: return launch_gemv_mu<M, 1, 4, 2, SC>(m, plan, x, in_scale, y, y_f32, stream);
+      case 32 + 1: return launch_gemv_mu<M, 1, 1, 4, SC>(m, plan, x, in_scale, y, y_f32, stream);
+      case 32 + 2: return launch_gemv_mu<M, 1, 2, 4, SC>(m, plan, x, in_scale, y, y_f32, stream);
+      case 32 + 3: return launch_gemv_mu<M, 1, 3, 4, SC>(m, plan, x, in_scale, y, y_f32, stream);
+      case 32 + 4: return launch_gemv_mu<M, 1, 4, 4, SC>(m, plan, x, in_scale, y, y_f32, stream);
       default: return cudaErrorInvalidValue;
     }
   }
   if (plan.nb == 1) {
-    if (plan.up == 1) return launch_gemv_mu<M, 1, 1, 1>(m, plan, x, y, y_f32, stream);
-    if (plan.up == 2) return launch_gemv_mu<M, 2, 1, 1>(m, plan, x, y, y_f32, stream);
-    if (plan.up == 4) return launch_gemv_mu<M, 4, 1, 1>(m, plan, x, y, y_f32, stream);
+    if (plan.up == 1) return launch_gemv_mu<M, 1, 1, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
+    if (plan.up == 2) return launch_gemv_mu<M, 2, 1, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
+    if (plan.up == 4) return launch_gemv_mu<M, 4, 1, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
     return cudaErrorInvalidValue;
   }
   if constexpr (M >= 5) {
     if (plan.up != 1) return cudaErrorInvalidValue;
     switch (plan.nb) {
-      case 2: return launch_gemv_mu<M, 1, 2, 1>(m, plan, x, y, y_f32, stream);
-      case 3: return launch_gemv_mu<M, 1, 3, 1>(m, plan, x, y, y_f32, stream);
-      case 4: return launch_gemv_mu<M, 1, 4, 1>(m, plan, x, y, y_f32, stream);
+      case 2: return launch_gemv_mu<M, 1, 2, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
+      case 3: return launch_gemv_mu<M, 1, 3, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
+      case 4: return launch_gemv_mu<M, 1, 4, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
       default: return cudaErrorInvalidValue;
     }
   } else {
     const int k = (plan.up == 4 ? 2 : plan.up - 1) * 4 + plan.nb;
     switch (k) {
-      case 2: return launch_gemv_mu<M, 1, 2, 1>(m, plan, x, y, y_f32, stream);
-      case 3: return launch_gemv_mu<M, 1, 3, 1>(m, plan, x, y, y_f32, stream);
-      case 4: return launch_gemv_mu<M, 1, 4, 1>(m, plan, x, y, y_f32, stream);
-      case 6: return launch_gemv_mu<M, 2, 2, 1>(m, plan, x, y, y_f32, stream);
-      case 7: return launch_gemv_mu<M, 2, 3, 1>(m, plan, x, y, y_f32, stream);
-      case 8: return launch_gemv_mu<M, 2, 4, 1>(m, plan, x, y, y_f32, stream);
-      case 10: return launch_gemv_mu<M, 4, 2, 1>(m, plan, x, y, y_f32, stream);
+      case 2: return launch_gemv_mu<M, 1, 2, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
+      case 3: return launch_gemv_mu<M, 1, 3, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
+      case 4: return launch_gemv_mu<M, 1, 4, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
+      case 6: return launch_gemv_mu<M, 2, 2, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
+      case 7: return launch_gemv_mu<M, 2, 3, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
+      case 8: return launch_gemv_mu<M, 2, 4, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
+      case 10: return launch_gemv_mu<M, 4, 2, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
       default: return cudaErrorInvalidValue;
     }
   }
+}
+
+template <int M>
+cudaError_t launch_gemv_m(const DeviceMatrix& m, const GemvPlan& plan, const void* x, const float* in_scale, void* y,
+                          int y_f32, cudaStream_t stream) {
+  return in_scale ? launch_gemv_m<M, true>(m, plan, x, in_scale, y, y_f32, stream)
+                  : launch_gemv_m<M, false>(m, plan, x, nullptr, y, y_f32, stream);
 }
 
 template <int M>
@@ -762,6 +771,7 @@ bool make_plan(const DeviceMatrix& m, int bits, int nb, GemvPlan* p) {
   q.group_shift = 0;
   while ((1 << q.group_shift) < m.group) ++q.group_shift;
   q.pdl = 1;
+  q.nmem = m.nmem;
   // Rows per warp per block: up to 4, but no more than the CTA's rows call for.
   const int per_rg = (q.rows_cap + q.RG - 1) / q.RG;
   int up_max = per_rg >= 4 ? 4 : per_rg >= 2 ? 2 : 1;
@@ -805,14 +815,14 @@ bool make_plan(const DeviceMatrix& m, int bits, int nb, GemvPlan* p) {
   return false;
 }
 
-cudaError_t launch_gemv(const DeviceMatrix& m, const GemvPlan& plan, int bits, const void* x, void* y, int y_f32,
-                        cudaStream_t stream) {
+cudaError_t launch_gemv(const DeviceMatrix& m, const GemvPlan& plan, int bits, const void* x, const float* in_scale,
+                        void* y, int y_f32, cudaStream_t stream) {
   switch (bits) {
-    case 2: return launch_gemv_m<2>(m, plan, x, y, y_f32, stream);
-    case 3: return launch_gemv_m<3>(m, plan, x, y, y_f32, stream);
-    case 4: return launch_gemv_m<4>(m, plan, x, y, y_f32, stream);
-    case 5: return launch_gemv_m<5>(m, plan, x, y, y_f32, stream);
-    case 6: return launch_gemv_m<6>(m, plan, x, y, y_f32, stream);
+    case 2: return launch_gemv_m<2>(m, plan, x, in_scale, y, y_f32, stream);
+    case 3: return launch_gemv_m<3>(m, plan, x, in_scale, y, y_f32, stream);
+    case 4: return launch_gemv_m<4>(m, plan, x, in_scale, y, y_f32, stream);
+    case 5: return launch_gemv_m<5>(m, plan, x, in_scale, y, y_f32, stream);
+    case 6: return launch_gemv_m<6>(m, plan, x, in_scale, y, y_f32, stream);
     default: return cudaErrorInvalidValue;
   }
 }

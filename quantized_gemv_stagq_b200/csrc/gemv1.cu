@@ -63,6 +63,7 @@ struct Gemv1Args {
   const float2* table;  // (lo_M, s_M c_M) of this precision
   const float* dlo;     // lo - lo_M of this precision (post-grid entries)
   const __half* x;
+  const float* in_scale;  // SC: per-channel multiplier of x (the inverse activation scale)
   void* y;
   int y_f32;
 };
@@ -76,7 +77,7 @@ constexpr uint64_t kDrainLimit1Ns = 100000000ull;  // after a failure: wait for 
 __host__ __device__ inline int part_stride1(int KW) { return KW * kParts1 + 4; }
 
 struct Smem1 {
-  uint32_t full, empty, side_bar, flag, tab, xq, xscale, xsum, xsum16, pairs, side, part, rowid, term, ring;
+  uint32_t full, empty, side_bar, flag, stall, tab, xq, xscale, xsum, xsum16, pairs, side, part, rowid, term, ring;
   uint32_t slot;         // bytes of one ring slot
   uint32_t plane_piece;  // offset of the first read plane inside a slot (base rows at 0)
   uint32_t total;
@@ -92,7 +93,8 @@ __host__ __device__ inline Smem1 smem1(const Gemv1Plan& p, int in, int M) {
   L.empty = o; o += 8 * kMaxSlots;   // every consumer warp is done with the slot
   L.side_bar = o; o += 8;            // pair table, pair bytes and side record landed
   L.flag = o; o += 8;                // a wait gave up (any thread)
-  L.tab = o; o += 256 * 8;
+  L.stall = o; o += 8;               // test hook: a barrier nothing completes
+  L.tab = o; o += 256 * 8 * (uint32_t)p.nmem;  // the pair table of each stacked member
   L.xq = o; o += 2 * in;
   L.xscale = o; o += 4 * nchunk;
   L.xsum = o; o += 4 * nchunk;
@@ -144,7 +146,7 @@ __device__ __forceinline__ bool keeps_partial1(int lane) {
   return UP == 4 ? true : UP == 2 ? (lane & 8) == 0 : lane < 8;
 }
 
-template <int M, int UP, int G>
+template <int M, int UP, int G, bool SC>
 __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const Gemv1Plan& P = a.plan;
@@ -195,6 +197,7 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
       mbar_init(empty0 + 8 * s, (uint32_t)NW);
     }
     mbar_init(side_bar, 1);
+    mbar_init(sbase + L.stall, 1);
     *flag = 0u;
     fence_barrier_init();
   }
@@ -204,8 +207,8 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
     // waiting for them.
     const uint32_t pb = (uint32_t)(rows * ps);
     const uint32_t sb = P.stage_side ? (uint32_t)P.side_stride : 0u;
-    mbar_arrive_expect_tx(side_bar, 256 * 8 + pb + sb);
-    bulk_load(sbase + L.tab, a.table, 256 * 8, side_bar);
+    mbar_arrive_expect_tx(side_bar, 256 * 8 * (uint32_t)P.nmem + pb + sb);
+    bulk_load(sbase + L.tab, a.table, 256 * 8 * (uint32_t)P.nmem, side_bar);
     bulk_load(sbase + L.pairs, pair_g, pb, side_bar);
     if (sb) bulk_load(sbase + L.side, side_g, sb, side_bar);
     for (int b = 0; b < NS && b < nblk; ++b) issue_block(b, b);
@@ -219,12 +222,13 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
   // convert exactly; rounding to nearest even goes through the 1.5 * 2^23
   // shifter (the low 16 bits of the sum are the two's-complement integer).
   {
-    constexpr float kShift = 12582912.0f;
     constexpr int kBatch = 4;
     const int ntask = 4 * nchunk;
     const uint4* x4 = reinterpret_cast<const uint4*>(a.x);
+    const float4* s4 = reinterpret_cast<const float4*>(a.in_scale);
     for (int t0 = 0; t0 < ntask; t0 += kBatch * nthreads) {
       uint4 raw[kBatch][2];
+      float4 sv[kBatch][4];
 #pragma unroll
       for (int q = 0; q < kBatch; ++q) {
         const int t = t0 + q * nthreads + tid;
@@ -233,39 +237,26 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
           raw[q][0] = __ldg(x4 + 2 * t);
           raw[q][1] = __ldg(x4 + 2 * t + 1);
         }
+        if constexpr (SC) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) sv[q][k] = t < ntask ? __ldg(s4 + 4 * t + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
 #pragma unroll
       for (int q = 0; q < kBatch; ++q) {
         const int tw = t0 + q * nthreads + warp * 32;  // first task of this warp
         if (tw >= ntask) break;                         // warp-uniform
         const int t = tw + lane;
-        const uint32_t* w = reinterpret_cast<const uint32_t*>(raw[q]);
-        __half2 m2 = __habs2(*reinterpret_cast<const __half2*>(&w[0]));
-#pragma unroll
-        for (int k = 1; k < 8; ++k) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __half2*>(&w[k])));
-        float mx = fmaxf(__low2float(m2), __high2float(m2));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-        const int e = mx > 0.f ? 14 - ((int)((__float_as_uint(mx) >> 23) & 0xFF) - 127) : 0;
-        const float sc = __int_as_float((127 + e) << 23);
         uint32_t Q[8];
-        int sumq = 0;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
-          Q[k] = __byte_perm(__float_as_uint(fmaf(f.x, sc, kShift)), __float_as_uint(fmaf(f.y, sc, kShift)), 0x5410);
-          sumq = dp2a_lo(Q[k], 0x0101u, sumq);
-        }
-        const int sum16 = sumq;
-        sumq += __shfl_xor_sync(kFull, sumq, 1);
-        sumq += __shfl_xor_sync(kFull, sumq, 2);
+        float xs_c;
+        int sum16, sumq;
+        convert_x_task<SC>(raw[q], sv[q], Q, xs_c, sum16, sumq);
         if (t < ntask) {
           uint4* dst = reinterpret_cast<uint4*>(xq);
           dst[xq_piece(t >> 2, 2 * (t & 3))] = make_uint4(Q[0], Q[1], Q[2], Q[3]);
           dst[xq_piece(t >> 2, 2 * (t & 3) + 1)] = make_uint4(Q[4], Q[5], Q[6], Q[7]);
-          if constexpr (G > 1) xsum16[t] = __int_as_float((127 - e) << 23) * (float)sum16;
+          if constexpr (G > 1) xsum16[t] = xs_c * (float)sum16;
           if ((t & 3) == 0) {
-            const float xs_c = __int_as_float((127 - e) << 23);
             xscale[t >> 2] = xs_c;
             xsum[t >> 2] = xs_c * (float)sumq;
           }
@@ -290,7 +281,8 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
   if (warp == 0) {
     // ---------------------------------------------------------- producer
     for (int b = 0; ok && b + NS < nblk; ++b) {
-      if (!__all_sync(kFull, mbar_wait(empty0 + 8 * (b % NS), (uint32_t)(b / NS) & 1u, kWaitLimit1Ns))) {
+      // stops early when a consumer has given up (it releases no more slots)
+      if (!__all_sync(kFull, mbar_wait_unless(empty0 + 8 * (b % NS), (uint32_t)(b / NS) & 1u, kWaitLimit1Ns, flag))) {
         ok = false;
         break;
       }
@@ -339,9 +331,16 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
     const uint8_t* ring = smem + L.ring;
     int slot = 0;
     uint32_t phase = 0;
-    for (int b = 0; b < nblk; ++b) {
+    // Test hook (stagq_debug_stall): one bounded wait that runs out, so that
+    // the give-up path below runs on a healthy launch.
+    if (a.m.debug_stall_ns && !__all_sync(kFull, mbar_wait(sbase + L.stall, 0, a.m.debug_stall_ns))) {
+      ok = false;
+      if (lane == 0) *flag = 1u;
+    }
+    for (int b = 0; ok && b < nblk; ++b) {
       if (!__all_sync(kFull, mbar_wait(full0 + 8 * slot, phase, kWaitLimit1Ns))) {
         ok = false;
+        if (lane == 0) *flag = 1u;
         break;
       }
       const uint8_t* sb = ring + slot * L.slot;
@@ -349,6 +348,7 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
       uint32_t B[UP][4];
       uint2 Pw[UP][M > 2 ? M - 2 : 1];
       float2 lm[UP];
+      const float2* tb[UP];  // the pair table of each row's member
       uint32_t pw[UP];  // G > 1: the row's G pair bytes of this chunk
 #pragma unroll
       for (int u = 0; u < UP; ++u) {
@@ -358,7 +358,8 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
         for (int k = 0; k < M - 2; ++k)
           Pw[u][k] = *reinterpret_cast<const uint2*>(sb + off_p + u * step_p + k * plane_stride);
         const int row = min(lr + RG * u, rows - 1);  // rows past the CTA's end read a valid pair byte
-        if constexpr (G == 1) lm[u] = tab[pairs[row * ps + pcol]];
+        tb[u] = tab + member_table_offset(a.m.mem_row, r0 + row);
+        if constexpr (G == 1) lm[u] = tb[u][pairs[row * ps + pcol]];
         else pw[u] = load_pairs<G>(pairs + row * ps + pcol);
       }
       float v[UP];
@@ -373,7 +374,7 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
           float acc = 0.f;
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            const float2 l = tab[(pw[u] >> (8 * g)) & 0xFFu];
+            const float2 l = tb[u][(pw[u] >> (8 * g)) & 0xFFu];
             acc = fmaf(l.y, (float)tot[g] * xs, fmaf(l.x, xsg[g], acc));
           }
           v[u] = acc;
@@ -405,9 +406,11 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
           const int j = jb + 32 * k;
           if (j < j1) {
             const uint32_t en = ents[j];
-            const int e = (int)(en & 0x7FFFu);  // x~ slot; e >> 6 is the column's 64-chunk
-            const int grp = G == 1 ? e >> gs : column_of_xq_slot(e) >> gs;  // the column's group
-            const int pb = pairs[(int)rowid[j] * ps + grp];
+            const int col = (int)(en & 0x7FFFu);
+            const int e = xq_elem(col);         // the column's x~ slot (same 64-chunk as the column)
+            const int grp = col >> gs;          // the column's group
+            const int lrow = (int)rowid[j];
+            const int pb = pairs[lrow * ps + grp] + member_table_offset(a.m.mem_row, r0 + lrow);
             const float v = __half2float(__ushort_as_half((unsigned short)(en >> 16)));
             float d;
             if constexpr (decltype(with_post)::value) {
@@ -459,13 +462,13 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
 // Opt a kernel into `smem` bytes of dynamic shared memory (and the largest
 // shared-memory carve-out) on the current device, once per (device, kernel).
 cudaError_t ensure_smem1(const void* kern, int key, size_t smem) {
-  constexpr int kMaxDev = 64;
+  constexpr int kMaxDev = 64, kKeys = 128;
   static std::mutex mu;
-  static size_t granted[kMaxDev][64] = {};
+  static size_t granted[kMaxDev][kKeys] = {};
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  if (dev < 0 || dev >= kMaxDev || key < 0 || key >= 64) return cudaErrorInvalidValue;
+  if (dev < 0 || dev >= kMaxDev || key < 0 || key >= kKeys) return cudaErrorInvalidValue;
   std::lock_guard<std::mutex> lock(mu);
   if (granted[dev][key] >= smem) return cudaSuccess;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -474,20 +477,21 @@ cudaError_t ensure_smem1(const void* kern, int key, size_t smem) {
   return err;
 }
 
-template <int M, int UP, int G>
-cudaError_t launch1_mu(const DeviceMatrix& m, const Gemv1Plan& plan, const void* x, void* y, int y_f32,
-                       cudaStream_t stream) {
+template <int M, int UP, int G, bool SC>
+cudaError_t launch1_mu(const DeviceMatrix& m, const Gemv1Plan& plan, const void* x, const float* in_scale, void* y,
+                       int y_f32, cudaStream_t stream) {
   Gemv1Args a;
   a.m = m;
   a.plan = plan;
-  a.table = m.tables + 256 * (M - 2);
-  a.dlo = m.dlo + 256 * (M - 2);
+  a.table = m.tables + 256 * m.nmem * (M - 2);
+  a.dlo = m.dlo + 256 * m.nmem * (M - 2);
   a.x = reinterpret_cast<const __half*>(x);
+  a.in_scale = in_scale;
   a.y = y;
   a.y_f32 = y_f32;
   const Smem1 L = smem1(plan, m.in, M);
-  auto kern = gemv1_kernel<M, UP, G>;
-  const int key = ((M - 2) * 3 + (UP == 4 ? 2 : UP - 1)) * 3 + (G == 4 ? 2 : G - 1);
+  auto kern = gemv1_kernel<M, UP, G, SC>;
+  const int key = (((M - 2) * 3 + (UP == 4 ? 2 : UP - 1)) * 3 + (G == 4 ? 2 : G - 1)) * 2 + (SC ? 1 : 0);
   cudaError_t err = ensure_smem1(reinterpret_cast<const void*>(kern), key, L.total);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -503,19 +507,26 @@ cudaError_t launch1_mu(const DeviceMatrix& m, const Gemv1Plan& plan, const void*
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <int M>
-cudaError_t launch1_m(const DeviceMatrix& m, const Gemv1Plan& plan, const void* x, void* y, int y_f32,
-                      cudaStream_t stream) {
+template <int M, bool SC>
+cudaError_t launch1_m(const DeviceMatrix& m, const Gemv1Plan& plan, const void* x, const float* in_scale, void* y,
+                      int y_f32, cudaStream_t stream) {
   switch (groups_per_chunk(plan.group_shift) * 8 + plan.up) {
-    case 8 + 1: return launch1_mu<M, 1, 1>(m, plan, x, y, y_f32, stream);
-    case 8 + 2: return launch1_mu<M, 2, 1>(m, plan, x, y, y_f32, stream);
-    case 8 + 4: return launch1_mu<M, 4, 1>(m, plan, x, y, y_f32, stream);
-    case 16 + 1: return launch1_mu<M, 1, 2>(m, plan, x, y, y_f32, stream);  // groups of 32
-    case 16 + 2: return launch1_mu<M, 2, 2>(m, plan, x, y, y_f32, stream);
-    case 32 + 1: return launch1_mu<M, 1, 4>(m, plan, x, y, y_f32, stream);  // groups of 16
-    case 32 + 2: return launch1_mu<M, 2, 4>(m, plan, x, y, y_f32, stream);
+    case 8 + 1: return launch1_mu<M, 1, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
+    case 8 + 2: return launch1_mu<M, 2, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
+    case 8 + 4: return launch1_mu<M, 4, 1, SC>(m, plan, x, in_scale, y, y_f32, stream);
+    case 16 + 1: return launch1_mu<M, 1, 2, SC>(m, plan, x, in_scale, y, y_f32, stream);  // groups of 32
+    case 16 + 2: return launch1_mu<M, 2, 2, SC>(m, plan, x, in_scale, y, y_f32, stream);
+    case 32 + 1: return launch1_mu<M, 1, 4, SC>(m, plan, x, in_scale, y, y_f32, stream);  // groups of 16
+    case 32 + 2: return launch1_mu<M, 2, 4, SC>(m, plan, x, in_scale, y, y_f32, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+template <int M>
+cudaError_t launch1_m(const DeviceMatrix& m, const Gemv1Plan& plan, const void* x, const float* in_scale, void* y,
+                      int y_f32, cudaStream_t stream) {
+  return in_scale ? launch1_m<M, true>(m, plan, x, in_scale, y, y_f32, stream)
+                  : launch1_m<M, false>(m, plan, x, nullptr, y, y_f32, stream);
 }
 
 }  // namespace
@@ -593,6 +604,7 @@ bool make_plan1(const DeviceMatrix& m, int bits, Gemv1Plan* p) {
   q.group_shift = 0;
   while ((1 << q.group_shift) < m.group) ++q.group_shift;
   q.pdl = 1;
+  q.nmem = m.nmem;
 
   // Row groups. Narrow: 8 consumer warps for rows of 1 or 2 K slices (RG =
   // 8 / KW), one per K slice beyond. Wide: at least kWideWarps consumer warps
@@ -627,14 +639,14 @@ bool make_plan1(const DeviceMatrix& m, int bits, Gemv1Plan* p) {
   return false;
 }
 
-cudaError_t launch_gemv1(const DeviceMatrix& m, const Gemv1Plan& plan, int bits, const void* x, void* y, int y_f32,
-                         cudaStream_t stream) {
+cudaError_t launch_gemv1(const DeviceMatrix& m, const Gemv1Plan& plan, int bits, const void* x, const float* in_scale,
+                         void* y, int y_f32, cudaStream_t stream) {
   switch (bits) {
-    case 2: return launch1_m<2>(m, plan, x, y, y_f32, stream);
-    case 3: return launch1_m<3>(m, plan, x, y, y_f32, stream);
-    case 4: return launch1_m<4>(m, plan, x, y, y_f32, stream);
-    case 5: return launch1_m<5>(m, plan, x, y, y_f32, stream);
-    case 6: return launch1_m<6>(m, plan, x, y, y_f32, stream);
+    case 2: return launch1_m<2>(m, plan, x, in_scale, y, y_f32, stream);
+    case 3: return launch1_m<3>(m, plan, x, in_scale, y, y_f32, stream);
+    case 4: return launch1_m<4>(m, plan, x, in_scale, y, y_f32, stream);
+    case 5: return launch1_m<5>(m, plan, x, in_scale, y, y_f32, stream);
+    case 6: return launch1_m<6>(m, plan, x, in_scale, y, y_f32, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -61,6 +61,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
     if ((i & 15u) == 0 && global_timer() - t0 > limit_ns) return false;
   }
 }
+// mbar_wait that also gives up as soon as *stop is nonzero (another thread of
+// the CTA gave up).
+__device__ __forceinline__ bool mbar_wait_unless(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                                 const volatile uint32_t* stop) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*stop) return false;
+    if ((i & 15u) == 0 && global_timer() - t0 > limit_ns) return false;
+  }
+}
 // 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
 // dst, src and bytes are multiples of 16.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
@@ -174,6 +186,57 @@ __device__ __forceinline__ int chunk_dot(const uint32_t (&X)[32], const uint32_t
   int t[1];
   chunk_dot_g<M, 1>(X, B, P, t);
   return t[0];
+}
+
+// One task of the conversion of x to 16-bit fixed point: 16 values of one
+// 64-element chunk (the chunk's 4 tasks sit in adjacent lanes, every lane of
+// the warp calls this). raw: the 16 fp16 values; SC: times the run-time
+// inverse activation scale s (16 fp32 values; the quantiser saw W diag(a), so
+// channel c of x is multiplied by 1/a_c, Appendix E), rounded to fp32.
+// Scale 2^e with max|x| 2^e in [2^14, 2^15) over the chunk, so the largest
+// entries convert exactly; rounding to nearest even goes through the 1.5 *
+// 2^23 shifter (the low 16 bits of the sum are the two's-complement integer).
+// Out: Q (8 pairs of int16), xs = 2^-e, sum16 = the task's sum of x~, sumq =
+// the chunk's.
+template <bool SC>
+__device__ __forceinline__ void convert_x_task(const uint4 (&raw)[2], const float4 (&s)[4], uint32_t (&Q)[8], float& xs,
+                                               int& sum16, int& sumq) {
+  constexpr float kShift = 12582912.0f;
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(raw);
+  float2 f[8];
+  float mx = 0.f;
+  if constexpr (SC) {
+    const float* sv = reinterpret_cast<const float*>(s);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      f[k] = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+      f[k].x *= sv[2 * k];
+      f[k].y *= sv[2 * k + 1];
+      mx = fmaxf(mx, fmaxf(fabsf(f[k].x), fabsf(f[k].y)));
+    }
+  } else {
+    __half2 m2 = __habs2(*reinterpret_cast<const __half2*>(&w[0]));
+#pragma unroll
+    for (int k = 1; k < 8; ++k) m2 = __hmax2(m2, __habs2(*reinterpret_cast<const __half2*>(&w[k])));
+    mx = fmaxf(__low2float(m2), __high2float(m2));
+#pragma unroll
+    for (int k = 0; k < 8; ++k) f[k] = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+  }
+  mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+  int e = mx > 0.f ? 14 - ((int)((__float_as_uint(mx) >> 23) & 0xFF) - 127) : 0;
+  if constexpr (SC) e = max(-126, min(126, e));  // 2^e and 2^-e stay normal floats
+  const float sc = __int_as_float((127 + e) << 23);
+  sumq = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    Q[k] = __byte_perm(__float_as_uint(fmaf(f[k].x, sc, kShift)), __float_as_uint(fmaf(f[k].y, sc, kShift)), 0x5410);
+    sumq = dp2a_lo(Q[k], 0x0101u, sumq);
+  }
+  sum16 = sumq;
+  sumq += __shfl_xor_sync(kFull, sumq, 1);
+  sumq += __shfl_xor_sync(kFull, sumq, 2);
+  xs = __int_as_float((127 - e) << 23);
 }
 
 // Groups per 64-weight chunk for a group size of 2^group_shift (>= 16).

@@ -2,6 +2,7 @@
 
   python -m quantized_gemv_stagq_b200.profile_case --shape 14336x4096 --bits 4 \
       [--copies 5] [--launches 5] [--group 128] [--planes 2] [--density 0.005]
+      [--kernel default|general|single]
 
 Launches rotate over `copies` device copies of the encoded matrix, so with
 copies x size above the L2 size every launch reads from HBM. Exits non-zero if
@@ -27,14 +28,16 @@ def main():
     p.add_argument("--group", type=int, default=128)
     p.add_argument("--planes", type=int, default=2)
     p.add_argument("--density", type=float, default=0.005)
+    p.add_argument("--kernel", default="default", choices=["default", "general", "single"])
     a = p.parse_args()
+    flags = {"default": 0, "general": Q.STAGQ_KERNEL_GENERAL, "single": Q.STAGQ_KERNEL_SINGLE}[a.kernel]
     out, inp = (int(v) for v in a.shape.lower().split("x"))
     S = Q.stagq_pack(Q.stagq_encode(synth.weights(out, inp, seed=1), a.group, a.planes, a.density, "fast"))
     mats = [Q.stagq_load(S, 0) for _ in range(a.copies)]
     x = torch.from_numpy(synth.activations(1, inp, seed=2)).cuda()
     y = torch.empty(1, out, dtype=torch.float16, device="cuda")
     for i in range(a.launches):
-        Q.stagq_gemv(mats[i % a.copies], a.bits, x, y)
+        Q.stagq_gemv_ex(mats[i % a.copies], a.bits, x, y, flags=flags)
     torch.cuda.synchronize()
     if not np.all(np.isfinite(y.float().cpu().numpy())):
         raise SystemExit("non-finite y")

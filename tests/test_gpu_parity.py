@@ -329,3 +329,240 @@ def test_appendix_e_codebooks_gemv_matches_oracle():
             check_close(got[j], ref[j], f"p{M} n4 col{j}")
     Q.stagq_check(m)
     m.free()
+
+
+# ------------------------------- stacked handles (q/k/v or gate/up in one launch)
+
+STACKED = [
+    # member shapes (out) at a common in, group, n_planes, density, guards
+    ((192, 64, 64), 1024, 128, 2, 0.005, None),
+    ((96, 33, 160), 2048, 64, 4, 0.01, None),
+    ((37, 100), 640, 32, 3, 0.02, None),
+    ((64, 48, 80, 16), 1024, 128, 2, 0.0, "ratio"),   # pre- and post-grid guards, four members
+]
+
+
+def _stack_fields(case, seed0):
+    outs, inp, g, npl, dens, guard = case
+    Fs = []
+    for j, out in enumerate(outs):
+        W = synth.weights(out, inp, seed0 + j)
+        if guard == "ratio":
+            Fs.append(O.encode(W, g, npl, mode="fast", guard="ratio", ratio_T=4.0, post_guard=True))
+        else:
+            Fs.append(O.encode(W, g, npl, dens, "fast"))
+    return Fs
+
+
+@pytest.mark.parametrize("case", STACKED, ids=lambda c: f"{'+'.join(map(str, c[0]))}x{c[1]}g{c[2]}p{c[3]}")
+def test_stacked_handle_matches_each_member(case):
+    """Each member's rows of a stacked handle against the oracle's GEMV of that
+    member alone (its own codebooks, pair bytes and side record), through both
+    n = 1 kernels, n = 4, and the decoded levels bit-exact."""
+    Fs = _stack_fields(case, 500)
+    assert len({tuple(F.cb_log2s.view(np.uint16)) for F in Fs}) > 1   # the members' codebooks differ
+    m = Q.stagq_load_stack([Q.stagq_pack(to_lib_fields(F)) for F in Fs], 0)
+    assert m.out == sum(F.out for F in Fs)
+    offs = np.concatenate([[0], np.cumsum([F.out for F in Fs])])
+    u = torch.empty(m.out, m.inp, dtype=torch.uint8, device="cuda")
+    x = synth.activations(4, m.inp, 77)
+    for M in range(2, 3 + Fs[0].n_planes):
+        Q.stagq_decode_levels(m, M, u)
+        torch.cuda.synchronize()
+        assert np.array_equal(u.cpu().numpy(), np.concatenate([O.decode_levels(F, M) for F in Fs])), f"levels p{M}"
+        refs = [O.gemv(F, M, x) for F in Fs]
+        for kern in (Q.STAGQ_KERNEL_GENERAL, Q.STAGQ_KERNEL_SINGLE):
+            y = _gemv(m, M, x[:1], kernel=kern)[0]
+            for j, F in enumerate(Fs):
+                check_close(y[offs[j]:offs[j + 1]], refs[j][0], f"member {j} p{M} kernel {kern}")
+        y4 = _gemv(m, M, x)
+        for j, F in enumerate(Fs):
+            for c in range(4):
+                check_close(y4[c][offs[j]:offs[j + 1]], refs[j][c], f"member {j} p{M} n4 col{c}")
+        # x read once, one row-pointer array for the whole stack
+        assert Q.stagq_bytes(m, M) == sum(O.model_bytes(F.out, F.inp, F.group, F.nnz, M) for F in Fs) \
+            - (len(Fs) - 1) * (2 * m.inp + 4)
+    Q.stagq_check(m)
+    m.free()
+
+
+@pytest.mark.parametrize("name,members", [("qkv", ("q_proj", "k_proj", "v_proj")), ("gate_up", ("gate_proj", "up_proj"))])
+def test_full_size_stacked_llama_sampled_rows(name, members):
+    """The bench's stacked Llama-3.1-8B handles (q/k/v: 6144 x 4096, gate/up:
+    28672 x 4096): library encoder per member, every member's sampled rows and
+    first / last rows against the oracle's own encoding of that member."""
+    shapes = [synth.LLAMA31_8B_LINEARS[n] for n in members]
+    Ws = [synth.weights(o, i, seed=5000 + j) for j, (o, i) in enumerate(shapes)]
+    Ps = [Q.stagq_encode(W, 128, 2, 0.005, "fast") for W in Ws]
+    m = Q.stagq_load_stack([Q.stagq_pack(P) for P in Ps], 0)
+    x = synth.activations(1, shapes[0][1], seed=8)
+    rng = np.random.default_rng(9)
+    off = 0
+    ys = {M: {k: _gemv(m, M, x, f32=False, kernel=k)[0] for k in _kernels()} for M in (2, 3, 4)}
+    for j, ((o, i), W) in enumerate(zip(shapes, Ws)):
+        rows = np.unique(np.concatenate([[0, o - 1], rng.choice(o, 24, replace=False)]))
+        F = O.encode(W, 128, 2, 0.005, "fast", rows=rows)
+        assert np.array_equal(F.pair_idx, Ps[j].pair_idx[rows]) and np.array_equal(F.q, Ps[j].q[rows])
+        for M in (2, 3, 4):
+            ref = O.gemv(F, M, x)[0]
+            for k, y in ys[M].items():
+                check_close(y[off + rows].astype(np.float64), ref, f"{name} member {j} p{M} kernel {k}")
+        off += o
+    Q.stagq_check(m)
+    m.free()
+
+
+# ------------------------- run-time inverse activation scale (Appendix E)
+
+def _in_scale(inp, seed):
+    """1/a_c for AWQ-like channel scales a_c spread over [0.25, 4] (log-uniform)."""
+    rng = np.random.default_rng(seed)
+    return (2.0 ** rng.uniform(-2.0, 2.0, inp)).astype(np.float32)
+
+
+def _gemv_scaled(m, bits, x_np, s_np, f32=True, kernel=0):
+    x = torch.from_numpy(np.ascontiguousarray(x_np)).cuda()
+    s = torch.from_numpy(np.ascontiguousarray(s_np)).cuda()
+    n = x.shape[0]
+    y = torch.empty(n, m.out, dtype=torch.float32 if f32 else torch.float16, device="cuda")
+    Q.stagq_gemv_scaled(m, bits, x, s, y, n=n, flags=(Q.STAGQ_Y_F32 if f32 else 0) | kernel)
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+@pytest.mark.parametrize("case", [SMALL[0], SMALL[1], SMALL[3], SMALL[10], SMALL[12]],
+                         ids=lambda c: f"{c[0]}x{c[1]}g{c[2]}p{c[3]}d{c[4]}")
+def test_scaled_gemv_matches_oracle(case):
+    """y = W_hat (x * in_scale) against the oracle's gemv(in_scale=), through
+    both n = 1 kernels and n = 4 in one launch."""
+    out, inp, g, npl, dens, mode, seed = case
+    F = O.encode(synth.weights(out, inp, seed), g, npl, dens, mode)
+    m = _load(F)
+    s = _in_scale(inp, seed + 1)
+    x = synth.activations(4, inp, seed + 300)
+    for M in range(2, 3 + npl):
+        ref = O.gemv(F, M, x, in_scale=s)
+        for kern in (Q.STAGQ_KERNEL_GENERAL, Q.STAGQ_KERNEL_SINGLE):
+            check_close(_gemv_scaled(m, M, x[:1], s, kernel=kern)[0], ref[0], f"p{M} kernel {kern}")
+        got = _gemv_scaled(m, M, x, s)
+        for j in range(4):
+            check_close(got[j], ref[j], f"p{M} n4 col{j}")
+        # a scale of ones is the unscaled GEMV
+        ones = _gemv_scaled(m, M, x[:1], np.ones(inp, np.float32))
+        check_close(ones[0], O.gemv(F, M, x[:1])[0], f"p{M} ones")
+    Q.stagq_check(m)
+    m.free()
+
+
+@pytest.mark.parametrize("name", ["gate_proj", "q_proj"])
+def test_full_size_scaled_sampled_rows(name):
+    """The Llama-3.1-8B gate (single-vector kernel) and q (general kernel)
+    shapes with an inverse activation scale, n = 1 and 4, sampled rows."""
+    out, inp = synth.LLAMA31_8B_LINEARS[name]
+    W = synth.weights(out, inp, seed=6000 + out)
+    P = Q.stagq_encode(W, 128, 2, 0.005, "fast")
+    m = Q.stagq_load(Q.stagq_pack(P), 0)
+    rows = np.unique(np.concatenate([[0, out - 1], np.random.default_rng(3).choice(out, 32, replace=False)]))
+    F = O.encode(W, 128, 2, 0.005, "fast", rows=rows)
+    s = _in_scale(inp, 5)
+    x = synth.activations(4, inp, seed=6)
+    for M in (2, 4):
+        ref = O.gemv(F, M, x, in_scale=s)
+        y1 = _gemv_scaled(m, M, x[:1], s, f32=False)[0]
+        check_close(y1[rows].astype(np.float64), ref[0], f"{name} p{M} n1")
+        y4 = _gemv_scaled(m, M, x, s, f32=False)
+        for j in range(4):
+            check_close(y4[j][rows].astype(np.float64), ref[j], f"{name} p{M} n4 col{j}")
+    Q.stagq_check(m)
+    m.free()
+
+
+# --------------------------- the side record as the device holds it (Eq. 4)
+
+def _expected_entries(F):
+    """The oracle's side record per row: (column | post-grid flag << 15, fp16 bits)."""
+    cols = lib_columns(F)
+    vals = F.val.view(np.uint16)
+    return [[(int(cols[e]), int(vals[e])) for e in range(F.row_ptr[r], F.row_ptr[r + 1])] for r in range(F.out)]
+
+
+def _decode_cuts(out, lay, cut, cut1):
+    """Rebuild each row's entries from the two device cuts (the layout of
+    stagq_debug_side_record), independently of the loader's code."""
+    rows_general = [[] for _ in range(out)]
+    G, S, RG, KW, CR = lay["grid"], lay["stride"], lay["row_groups"], lay["k_slices"], lay["class_rows"]
+    for b in range(G):
+        blk = cut[b * S:(b + 1) * S]
+        offs = blk[:4 * RG * KW * (CR + 1)].view(np.int32).reshape(RG, KW, CR + 1)
+        ents = blk[lay["ent_off"]:].view(np.uint32)
+        ra, rb = b * out // G, (b + 1) * out // G
+        for rg in range(RG):
+            nm = (rb - ra - rg + RG - 1) // RG if rb - ra > rg else 0
+            for kw in range(KW):
+                for mm in range(nm):
+                    r = ra + rg + RG * mm
+                    for e in ents[offs[rg, kw, mm]:offs[rg, kw, mm + 1]]:
+                        rows_general[r].append((int(e & 0xFFFF), int(e >> 16)))
+    rows_single = [[] for _ in range(out)]
+    G1, S1 = lay["grid1"], lay["stride1"]
+    for b in range(G1):
+        blk = cut1[b * S1:(b + 1) * S1]
+        ra, rb = b * out // G1, (b + 1) * out // G1
+        offs = blk[:4 * (rb - ra + 1)].view(np.int32)
+        ents = blk[lay["ent_off1"]:].view(np.uint32)
+        for r in range(ra, rb):
+            for e in ents[offs[r - ra]:offs[r - ra + 1]]:
+                rows_single[r].append((int(e & 0xFFFF), int(e >> 16)))
+    return rows_general, rows_single
+
+
+@pytest.mark.parametrize("kind", ["tiny", "ragged", "dense60", "all", "guarded", "wideK", "stacked"])
+def test_device_side_record_bit_exact(kind):
+    """Both device cuts of the side record hold exactly the oracle's CSR:
+    row, column, post-grid flag and fp16 value of every entry, in column
+    order within a row."""
+    if kind == "tiny":
+        Fs = [O.encode(synth.weights(512, 512, 1), 128, 2, 0.005, "search")]
+    elif kind == "ragged":
+        Fs = [O.encode(synth.weights(37, 640, 3), 128, 2, 0.02, "fast")]
+    elif kind == "dense60":
+        Fs = [O.encode(synth.weights(296, 4096, 9), 128, 2, 0.6, "fast")]
+    elif kind == "all":
+        Fs = [O.encode(synth.weights(64, 768, 7), 16, 2, 1.0, "fast")]
+    elif kind == "guarded":
+        Fs = [_guarded_fields(GUARDED[0])]
+    elif kind == "wideK":
+        Fs = [O.encode(synth.weights(300, 32768, 10), 128, 4, 0.005, "fast")]
+    else:
+        Fs = _stack_fields(STACKED[3], 700)
+    m = Q.stagq_load_stack([Q.stagq_pack(to_lib_fields(F)) for F in Fs], 0)
+    lay, cut, cut1 = Q.stagq_debug_side_record(m)
+    want = [row for F in Fs for row in _expected_entries(F)]
+    assert sum(len(r) for r in want) == sum(F.nnz for F in Fs)
+    got_general, got_single = _decode_cuts(m.out, lay, cut, cut1)
+    assert got_general == want
+    assert got_single == want
+    m.free()
+
+
+# ----------------------------- the bounded waits' give-up path (no GPU fault)
+
+@pytest.mark.parametrize("kernel", ["general", "single"])
+def test_wait_that_runs_out_is_reported_and_the_handle_recovers(kernel):
+    """A launch whose bounded wait runs out (stagq_debug_stall: a barrier
+    nothing completes, 20 us) lets its copies land, returns, and stagq_check
+    reports STAGQ_ETIMEOUT; with the hook off the next call matches the
+    oracle and stagq_check is clean."""
+    flag = Q.STAGQ_KERNEL_GENERAL if kernel == "general" else Q.STAGQ_KERNEL_SINGLE
+    F = O.encode(synth.weights(1024, 4096, 55), 128, 2, 0.005, "fast")
+    m = _load(F)
+    x = synth.activations(1, 4096, 56)
+    Q.stagq_debug_stall(m, 20000)
+    _gemv(m, 3, x, kernel=flag)
+    with pytest.raises(Q.StagqError) as e:
+        Q.stagq_check(m)
+    assert e.value.status == 7                       # STAGQ_ETIMEOUT
+    Q.stagq_debug_stall(m, 0)
+    check_close(_gemv(m, 3, x, kernel=flag)[0], O.gemv(F, 3, x)[0], "after the stall")
+    Q.stagq_check(m)                                  # the status word was cleared
+    m.free()

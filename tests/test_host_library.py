@@ -318,3 +318,29 @@ def test_binding_refuses_tensors_that_do_not_fit_the_call():
         Q.stagq_gemv_host(m, 2, np.zeros((1, 512), np.float16), np.zeros((1, 32), np.float16))
     with pytest.raises(TypeError, match="x_host"):
         Q.stagq_gemv_host_noalloc(m, 2, np.zeros((1, 512), np.float32), np.zeros((1, 64), np.float16))
+
+
+def test_stacked_load_checks_its_members():
+    """stagq_load_stack (members applied to one x) refuses bad counts and
+    members that differ in in / group / n_planes before any device work."""
+    a = _stream()
+    b = Q.stagq_pack(Q.stagq_encode(synth.weights(8, 512, seed=3), 128, 2, 0.0, "fast"))
+    with pytest.raises(Q.StagqError) as e:
+        Q.stagq_load_stack([], 0)
+    assert e.value.status == 1
+    with pytest.raises(Q.StagqError) as e:
+        Q.stagq_load_stack([a] * 5, 0)
+    assert e.value.status == 1
+    c = Q.stagq_pack(Q.stagq_encode(synth.weights(8, a.inp, seed=4), a.group, a.n_planes + 1, 0.0, "fast"))
+    with pytest.raises(Q.StagqError) as e:              # n_planes differ
+        Q.stagq_load_stack([a, c], 0)
+    assert e.value.status == 1
+    if a.inp != b.inp:
+        with pytest.raises(Q.StagqError) as e:
+            Q.stagq_load_stack([a, b], 0)
+        assert e.value.status == 1
+    bad = Q.HostStream(**{**a.__dict__, "row_ptr": a.row_ptr.copy()})
+    bad.row_ptr[2] = bad.row_ptr[3] + 1
+    with pytest.raises(Q.StagqError) as e:              # a malformed member
+        Q.stagq_load_stack([a, bad], 0)
+    assert e.value.status == 2
