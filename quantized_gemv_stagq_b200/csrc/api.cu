@@ -275,19 +275,14 @@ int load_impl(const stagq_host_stream* s, const stagq_host_stream* const* member
   if (m.smem_pair_budget > smem_limit) m.smem_pair_budget = smem_limit;
   for (int b = 2; b <= 2 + np; ++b)
     for (int nb = 1; nb <= STAGQ_MAX_BATCH; ++nb) h->plan_ok[b][nb] = make_plan(m, b, nb, &h->plan[b][nb]);
-  // The single-vector kernel serves n = 1 on matrices of more than 2^24
-  // weights (Llama-3.1-8B gate/up/down, Phi-4 and OLMo-2 q/o/gate/up/down):
-  // there its faster block loop outweighs its extra once-per-launch phases
-  // (entry rows, side-record terms, row sums), measured on chains of GEMVs at
-  // 2..6 bits. On smaller matrices those phases dominate and the general
-  // kernel is faster.
-  // Groups below 64 weights give the general kernel one row per warp per
-  // block (registers); the single-vector kernel keeps two, so it serves them
-  // at any size.
-  const bool large = (int64_t)s->out * s->in > ((int64_t)1 << 24) || s->group < 64;
+  // The single-vector kernel serves every n = 1 launch it can plan: one CTA
+  // per SM that has the SM to itself. A chain of launches of one shape of CTA
+  // stays evenly placed (see make_plan1); on the Llama-3.1-8B layer chain
+  // this measured 24 % faster than giving the general kernel (whose CTAs share
+  // an SM) the matrices of up to 2^24 weights.
   for (int b = 2; b <= 2 + np; ++b) {
     h->plan1_ok[b] = make_plan1(m, b, &h->plan1[b]);
-    h->prefer1[b] = large;
+    h->prefer1[b] = true;
   }
   if (!h->plan_ok[2][1]) {
     cudaFree(h->d_mem);

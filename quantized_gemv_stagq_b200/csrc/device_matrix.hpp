@@ -74,7 +74,7 @@ struct DeviceMatrix {
   uint32_t debug_stall_ns;    // test hook: launches include one bounded wait of this length that runs out
   int num_sms;
   int smem_limit;             // opt-in shared memory per block
-  int smem_pair_budget;       // shared memory per block that still lets two blocks share an SM
+  int smem_pair_budget;       // shared memory per block that still lets two blocks share an SM (general kernel)
 };
 
 // How one GEMV is laid out over the GPU (see gemv.cu).

@@ -203,6 +203,9 @@ __device__ __forceinline__ void rows_dot_nb(const int16_t* xq, const float* xsca
   uint32_t B[NR][4];
   uint2 Pw[NR][M > 2 ? M - 2 : 1];
   uint32_t pr[NR];
+  // up to two planes: the code words are decoded once for all NB vectors
+  constexpr bool kCodes = M <= 4;
+  uint32_t cw[kCodes ? NR : 1][16];
 #pragma unroll
   for (int u = 0; u < NR; ++u) {
     const uint4 b4 = *reinterpret_cast<const uint4*>(sb + off.b + u * step.b);
@@ -211,6 +214,7 @@ __device__ __forceinline__ void rows_dot_nb(const int16_t* xq, const float* xsca
     for (int k = 0; k < M - 2; ++k)
       Pw[u][k] = *reinterpret_cast<const uint2*>(sb + off.p + u * step.p + k * plane_stride);
     pr[u] = load_pairs<G>(sb + off.g + u * step.g);
+    if constexpr (kCodes) chunk_codes<M>(B[u], Pw[u], cw[u]);
   }
 #pragma unroll
   for (int j = 0; j < NB; ++j) {
@@ -240,7 +244,8 @@ __device__ __forceinline__ void rows_dot_nb(const int16_t* xq, const float* xsca
 #pragma unroll
     for (int u = 0; u < NR; ++u) {
       int tot[G];
-      chunk_dot_g<M, G>(X, B[u], Pw[u], tot);
+      if constexpr (kCodes) chunk_dot_codes<M, G>(X, cw[u], tot);
+      else chunk_dot_g<M, G>(X, B[u], Pw[u], tot);
       v[j][u] = group_affine<G>(tb[u], pr[u], tot, xs, xsg, lo[u]);
     }
   }
@@ -654,6 +659,8 @@ cudaError_t launch_gemv_mu(const DeviceMatrix& m, const GemvPlan& plan, const vo
   a.y = y;
   a.y_f32 = y_f32;
   const SmemLayout L = smem_layout(plan, m.in, M);
+  // every region that bulk copies fill or 16-byte accesses read starts on 16 bytes
+  if ((L.tab | L.xq | L.side | L.ring | L.slot | L.plane_piece | L.pair_piece) & 15u) return cudaErrorInvalidValue;
   auto kern = m.has_post ? gemv_kernel<M, UP, NB, G, true, SC> : gemv_kernel<M, UP, NB, G, false, SC>;
   const int key = (((((M - 2) * 3 + (UP == 4 ? 2 : UP - 1)) * 4 + (NB - 1)) * 3 + (G == 4 ? 2 : G - 1)) * 2 +
                    (m.has_post ? 1 : 0)) * 2 + (SC ? 1 : 0);

@@ -15,12 +15,12 @@
 //    memory ring slot with 1 + (M - 2) bulk copies. Warps 1..NW are consumers:
 //    KW K slices (2048 weights: 32 lanes x one 64-weight chunk) x RG row
 //    groups; in every block a consumer takes UP rows of its group in its slice.
-//  * The CTA uses at most half of an SM (<= 9 warps x 96 registers, <= half
-//    the shared memory) wherever its ring still fits, so the next GEMV's CTA
-//    is resident beside it and fills its ring -- weights, pair table, the
-//    CTA's pair bytes and side record do not depend on earlier kernels --
-//    before this one finishes. Where it does not fit, the CTA has 12 or more
-//    consumer warps and the SM to itself (make_plan1).
+//  * The CTA has the SM to itself, with as many consumer warps as the
+//    register file holds (make_plan1); with programmatic dependent launch it
+//    starts as soon as the previous launch's CTA on its SM has left, and its
+//    copies -- weights, pair table, the CTA's pair bytes and side record, none
+//    of which depend on earlier kernels -- are in flight while the previous
+//    grid drains.
 //  * x is converted once per CTA to 16-bit fixed point with a power-of-two
 //    scale per 64-element chunk (|error| <= 2^-16 max|x_chunk|); each lane keeps
 //    its chunk's 64 activations in registers; code bytes / nibble composites
@@ -54,7 +54,7 @@ namespace {
 
 using namespace kernels;
 
-constexpr int kRegs1 = 96;             // registers per thread: two 9-warp CTAs fit one SM, or one of 20
+constexpr int kRegs1 = 128;            // registers per thread: one CTA of up to 16 warps per SM
 constexpr int kParts1 = 8;             // partial sums per (row, K slice), each over 4 lanes
 
 struct Gemv1Args {
@@ -94,6 +94,7 @@ __host__ __device__ inline Smem1 smem1(const Gemv1Plan& p, int in, int M) {
   L.side_bar = o; o += 8;            // pair table, pair bytes and side record landed
   L.flag = o; o += 8;                // a wait gave up (any thread)
   L.stall = o; o += 8;               // test hook: a barrier nothing completes
+  o = up16(o);                       // bulk-copy destinations and 16-byte accesses from here on
   L.tab = o; o += 256 * 8 * (uint32_t)p.nmem;  // the pair table of each stacked member
   L.xq = o; o += 2 * in;
   L.xscale = o; o += 4 * nchunk;
@@ -490,6 +491,8 @@ cudaError_t launch1_mu(const DeviceMatrix& m, const Gemv1Plan& plan, const void*
   a.y = y;
   a.y_f32 = y_f32;
   const Smem1 L = smem1(plan, m.in, M);
+  // every region that bulk copies fill or 16-byte accesses read starts on 16 bytes
+  if ((L.tab | L.xq | L.pairs | L.side | L.part | L.ring | L.slot | L.plane_piece) & 15u) return cudaErrorInvalidValue;
   auto kern = gemv1_kernel<M, UP, G, SC>;
   const int key = (((M - 2) * 3 + (UP == 4 ? 2 : UP - 1)) * 3 + (G == 4 ? 2 : G - 1)) * 2 + (SC ? 1 : 0);
   cudaError_t err = ensure_smem1(reinterpret_cast<const void*>(kern), key, L.total);
@@ -537,34 +540,33 @@ int gemv1_grid(int out, int num_sms) {
   return g;
 }
 
-// Ring depth and shape (measured on B200 over the Llama-3.1-8B, Phi-4 and
-// OLMo-2 linears at 2..6 bits, alone and in a layer's chain of GEMVs):
-//  * A CTA that takes at most half of an SM (registers and shared memory)
-//    lets the next GEMV's CTA, whatever its kernel, start beside it; in a
-//    chain of different GEMVs that overlap is worth more than any ring shape,
-//    so such a plan is taken whenever one fits (side record staged, 2 or more
-//    rows per warp per block, 3 or more slots or all blocks).
+// Launch shape (measured on B200 over the Llama-3.1-8B, Phi-4 and OLMo-2
+// linears at 2..6 bits, alone and as a layer's chain of launches):
+//  * One CTA per SM that has the SM to itself, with as many consumer warps
+//    as the register file holds at kRegs1 registers (14-15 for the Llama
+//    shapes). Every single-vector launch having the same shape keeps a chain
+//    of launches evenly placed: a CTA starts only where its predecessor's CTA
+//    has left, one per SM, and its ring fills while the predecessor grid
+//    drains (programmatic dependent launch). Plans that let a CTA share its
+//    SM with the next launch's measured faster alone but slower in chains
+//    that mix shapes: an SM freed early could take two of the next launch's
+//    CTAs while another took none.
 //  * About 60 KB of weights in flight per SM hide the HBM latency: the ring
-//    grows to that from 3 slots where the budget allows.
-//  * A CTA that cannot be that small gets the SM to itself, and then 12 or
-//    more consumer warps (the loop is bound by integer issue, and more warps
-//    hide its latencies).
+//    grows to that from 3 slots where the shared memory allows.
 //  * Larger blocks (UP = 4) amortise the per-block waits and sums, as long as
 //    the CTA's rows still make about 5 blocks to pipeline.
 constexpr uint32_t kInflightTarget = 60u * 1024u;
-constexpr int kWideWarps = 12;
 constexpr int kMinBlocks = 5;
 
-// Plan for one (row groups, shared-memory budget): false if nothing fits.
-// `strict`: only plans with the side record staged and 2 or more rows per
-// warp per block.
-bool plan1_fit(const DeviceMatrix& m, int bits, const Gemv1Plan& q, uint32_t budget, bool strict, Gemv1Plan* out) {
+// The ring for given row groups: false if nothing fits the shared memory.
+bool plan1_fit(const DeviceMatrix& m, int bits, const Gemv1Plan& q, Gemv1Plan* out) {
+  const uint32_t budget = (uint32_t)m.smem_limit;
   const int nblk4 = (q.rows_cap + 4 * q.RG - 1) / (4 * q.RG);
   const int nblk2 = (q.rows_cap + 2 * q.RG - 1) / (2 * q.RG);
   // groups below 64 weights (several pairs per chunk): at most 2 rows per warp per block
   const int up0 = q.group_shift < 6 ? 2 : (nblk4 >= kMinBlocks || nblk2 < kMinBlocks) ? 4 : 2;
-  for (int stage = 1; stage >= (strict ? 1 : 0); --stage) {
-    for (int up = up0; up >= (strict ? 2 : 1); up /= 2) {
+  for (int stage = 1; stage >= 0; --stage) {   // side record staged in shared memory where it fits
+    for (int up = up0; up >= 1; up /= 2) {
       Gemv1Plan t = q;
       t.up = up;
       t.br = q.RG * up;
@@ -590,10 +592,11 @@ bool plan1_fit(const DeviceMatrix& m, int bits, const Gemv1Plan& q, uint32_t bud
 }
 
 bool make_plan1(const DeviceMatrix& m, int bits, Gemv1Plan* p) {
-  constexpr int kRegFileWarps = 4 * (16384 / (32 * kRegs1));  // warps the register file holds
+  // warps the register file holds at kRegs1 registers a thread (a sub-partition: 16384 registers)
+  constexpr int kRegFileWarps = 4 * (16384 / (32 * kRegs1));
   Gemv1Plan q = {};
   q.KW = (m.in / kChunk + 31) / 32;
-  if (q.KW < 1 || q.KW > kMaxWarps) return false;
+  if (q.KW < 1 || q.KW + 1 > kRegFileWarps) return false;
   q.grid = m.side1_grid;
   if (q.grid < 1) return false;
   q.rows_cap = (m.out + q.grid - 1) / q.grid;
@@ -605,38 +608,10 @@ bool make_plan1(const DeviceMatrix& m, int bits, Gemv1Plan* p) {
   while ((1 << q.group_shift) < m.group) ++q.group_shift;
   q.pdl = 1;
   q.nmem = m.nmem;
-
-  // Row groups. Narrow: 8 consumer warps for rows of 1 or 2 K slices (RG =
-  // 8 / KW), one per K slice beyond. Wide: at least kWideWarps consumer warps
-  // where the register file holds them.
-  const int rg_narrow = row_groups(q.KW);
-  int rg_wide = (kWideWarps + q.KW - 1) / q.KW;
-  while (rg_wide > rg_narrow && q.KW * rg_wide + 1 > kRegFileWarps) --rg_wide;
-  if (rg_wide < rg_narrow) rg_wide = rg_narrow;
-  if (q.KW * rg_narrow + 1 > kRegFileWarps) return false;
-  Gemv1Plan t;
-
-  // Half an SM (registers and shared memory) when it fits and has 8 consumer
-  // warps or one per K slice, else the wide CTA alone on its SM. Rows of 3 K
-  // slices would leave a half-SM CTA 6 warps, a sixth of their lanes idle;
-  // wide, the Phi-4 layer chain (q/o 5120x5120, gate/up 17920x5120) measured
-  // 27-30 % faster.
-  const bool narrow_full = q.KW * rg_narrow >= 8 || q.KW >= 5;
-  if (narrow_full && 2 * (q.KW * rg_narrow + 1) <= kRegFileWarps) {
-    q.RG = rg_narrow;
-    q.NW = q.KW * q.RG;
-    if (plan1_fit(m, bits, q, (uint32_t)m.smem_pair_budget, true, &t)) {
-      *p = t;
-      return true;
-    }
-  }
-  q.RG = rg_wide;
+  // row groups: as many as the register file holds beside the producer warp
+  q.RG = (kRegFileWarps - 1) / q.KW;
   q.NW = q.KW * q.RG;
-  if (plan1_fit(m, bits, q, (uint32_t)m.smem_limit, false, &t)) {
-    *p = t;
-    return true;
-  }
-  return false;
+  return plan1_fit(m, bits, q, p);
 }
 
 cudaError_t launch_gemv1(const DeviceMatrix& m, const Gemv1Plan& plan, int bits, const void* x, const float* in_scale,

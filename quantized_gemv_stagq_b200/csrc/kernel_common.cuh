@@ -180,6 +180,73 @@ __device__ __forceinline__ void chunk_dot_g(const uint32_t (&X)[32], const uint3
   }
 }
 
+// Decoding and dot product of chunk_dot_g split in two, for launches with
+// several activation vectors (M <= 4): chunk_codes turns the chunk's base /
+// plane words into its 16 masked code words once, and chunk_dot_codes dots
+// them with one vector's x~ (the same dp2a sequence as chunk_dot_g, so the
+// integer result is identical).
+//   M = 2:     cw[4 i + s] = base word i & (0x03030303 << 2 s)  (bytes q 4^s)
+//   M = 3, 4:  per word pair w, the low / high nibbles of the composites
+//              E0, O0, E1, O1 (layout.cuh: nibble 4q + 2 b3 + b4)
+template <int M>
+__device__ __forceinline__ void chunk_codes(const uint32_t (&B)[4], const uint2* P, uint32_t (&cw)[16]) {
+  static_assert(M >= 2 && M <= 4, "codes of up to two planes");
+  if constexpr (M == 2) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int s = 0; s < 4; ++s) cw[4 * i + s] = B[i] & (0x03030303u << (2 * s));
+  } else {
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const uint32_t p3 = w ? P[0].y : P[0].x;
+      uint32_t p4 = 0u;
+      if constexpr (M >= 4) p4 = w ? P[1].y : P[1].x;
+      uint32_t E0, O0, E1, O1;
+      nibble_words(B[2 * w], B[2 * w + 1], p3, p4, E0, O0, E1, O1);
+      cw[8 * w + 0] = E0 & 0x0F0F0F0Fu; cw[8 * w + 1] = E0 & 0xF0F0F0F0u;
+      cw[8 * w + 2] = O0 & 0x0F0F0F0Fu; cw[8 * w + 3] = O0 & 0xF0F0F0F0u;
+      cw[8 * w + 4] = E1 & 0x0F0F0F0Fu; cw[8 * w + 5] = E1 & 0xF0F0F0F0u;
+      cw[8 * w + 6] = O1 & 0x0F0F0F0Fu; cw[8 * w + 7] = O1 & 0xF0F0F0F0u;
+    }
+  }
+}
+template <int M, int G>
+__device__ __forceinline__ void chunk_dot_codes(const uint32_t (&X)[32], const uint32_t (&cw)[16], int (&tot)[G]) {
+  constexpr int WPG = 4 / G;  // chunk words per group
+  if constexpr (M == 2) {
+    int a[G][4];
+#pragma unroll
+    for (int g = 0; g < G; ++g) a[g][0] = a[g][1] = a[g][2] = a[g][3] = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int g = i / WPG;
+#pragma unroll
+      for (int s = 0; s < 4; ++s) a[g][s] = dot4(X, i, s, cw[4 * i + s], a[g][s]);
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) tot[g] = a[g][0] + (a[g][1] >> 2) + (a[g][2] >> 4) + (a[g][3] >> 6);
+  } else {
+    int lo[G], hi[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) lo[g] = hi[g] = 0;
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      const int i0 = 2 * w, i1 = 2 * w + 1, g0 = i0 / WPG, g1 = i1 / WPG;
+      lo[g0] = dot4(X, i0, 1, cw[8 * w + 0], lo[g0]);
+      hi[g0] = dot4(X, i0, 3, cw[8 * w + 1], hi[g0]);
+      lo[g0] = dot4(X, i0, 0, cw[8 * w + 2], lo[g0]);
+      hi[g0] = dot4(X, i0, 2, cw[8 * w + 3], hi[g0]);
+      lo[g1] = dot4(X, i1, 1, cw[8 * w + 4], lo[g1]);
+      hi[g1] = dot4(X, i1, 3, cw[8 * w + 5], hi[g1]);
+      lo[g1] = dot4(X, i1, 0, cw[8 * w + 6], lo[g1]);
+      hi[g1] = dot4(X, i1, 2, cw[8 * w + 7], hi[g1]);
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) tot[g] = lo[g] + (hi[g] >> 4);
+  }
+}
+
 // The whole chunk as one group (groups of 64 weights or more).
 template <int M>
 __device__ __forceinline__ int chunk_dot(const uint32_t (&X)[32], const uint32_t (&B)[4], const uint2* P) {

@@ -48,3 +48,16 @@ def check_close(y, y_ref, what=""):
     assert rel <= REL_L2_TOL, f"{what}: rel L2 {rel:.3e} > {REL_L2_TOL}"
     assert mabs <= MAX_ABS_TOL * max(scale, 1e-300), f"{what}: max abs {mabs:.3e} > {MAX_ABS_TOL} * {scale:.3e}"
     return rel, mabs
+
+
+# The single-vector kernel holds one warp per 2048-weight K slice plus its
+# producer warp in the register file: it plans K up to 15 slices (30720).
+SINGLE_MAX_IN = 15 * 2048
+
+
+def n1_kernels(inp, include_default=False):
+    """The n = 1 kernels that can serve a matrix with K = inp (flags)."""
+    ks = ([0] if include_default else []) + [Q.STAGQ_KERNEL_GENERAL]
+    if inp <= SINGLE_MAX_IN:
+        ks.append(Q.STAGQ_KERNEL_SINGLE)
+    return tuple(ks)

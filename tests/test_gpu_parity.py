@@ -13,7 +13,7 @@ torch = pytest.importorskip("torch")
 import quantized_gemv_stagq_b200 as Q
 from oracle import stagq as O
 from quantized_gemv_stagq_b200 import synth
-from tests.helpers import check_close, fields_equal, to_lib_fields
+from tests.helpers import check_close, fields_equal, lib_columns, n1_kernels, to_lib_fields
 
 pytestmark = pytest.mark.gpu
 
@@ -80,7 +80,7 @@ def test_gemv_matches_oracle(case):
     x = synth.activations(1, inp, seed + 100)
     for M in range(2, 3 + npl):
         ref = O.gemv(F, M, x)
-        for kern in (Q.STAGQ_KERNEL_GENERAL, Q.STAGQ_KERNEL_SINGLE):  # both n = 1 kernels
+        for kern in n1_kernels(inp):  # both n = 1 kernels
             check_close(_gemv(m, M, x, f32=True, kernel=kern), ref, f"fp32 y p{M} kernel {kern}")
             check_close(_gemv(m, M, x, f32=False, kernel=kern).astype(np.float64), ref, f"fp16 y p{M} kernel {kern}")
     Q.stagq_check(m)
@@ -565,4 +565,45 @@ def test_wait_that_runs_out_is_reported_and_the_handle_recovers(kernel):
     Q.stagq_debug_stall(m, 0)
     check_close(_gemv(m, 3, x, kernel=flag)[0], O.gemv(F, 3, x)[0], "after the stall")
     Q.stagq_check(m)                                  # the status word was cleared
+    m.free()
+
+
+# --------------------------------- full size, every row against the oracle
+
+@pytest.mark.parametrize("name", ["gate_proj", "q_proj"])
+def test_full_size_every_row(name):
+    """Llama-3.1-8B gate (14336 x 4096, the single-vector kernel by default)
+    and q (4096 x 4096, the general kernel by default): the oracle encodes the
+    whole matrix (fast pair rule), the GPU reads the oracle's own fields, and
+    every row of y is compared with the oracle's fp64 GEMV, through each n = 1
+    kernel, at 2/3/4 bits; the CTA row partitions and per-CTA side-record cuts
+    of the full grid are all exercised."""
+    out, inp = synth.LLAMA31_8B_LINEARS[name]
+    F = O.encode(synth.weights(out, inp, seed=7000 + out), 128, 2, 0.005, "fast")
+    m = _load(F)
+    x = synth.activations(1, inp, seed=7001)
+    for M in (2, 3, 4):
+        ref = O.gemv(F, M, x)[0]
+        for kern in _kernels():
+            check_close(_gemv(m, M, x, f32=True, kernel=kern)[0], ref, f"{name} p{M} kernel {kern} fp32")
+        check_close(_gemv(m, M, x, f32=False)[0].astype(np.float64), ref, f"{name} p{M} fp16")
+    Q.stagq_check(m)
+    m.free()
+
+
+def test_full_size_stacked_qkv_every_row():
+    """The stacked q/k/v handle of the bench (6144 x 4096), every row of every
+    member against the oracle's GEMV of that member."""
+    Fs = [O.encode(synth.weights(*synth.LLAMA31_8B_LINEARS[n], seed=7100 + j), 128, 2, 0.005, "fast")
+          for j, n in enumerate(("q_proj", "k_proj", "v_proj"))]
+    m = Q.stagq_load_stack([Q.stagq_pack(to_lib_fields(F)) for F in Fs], 0)
+    x = synth.activations(1, 4096, seed=7101)
+    for M in (2, 4):
+        for kern in _kernels():
+            y = _gemv(m, M, x, kernel=kern)[0]
+            off = 0
+            for j, F in enumerate(Fs):
+                check_close(y[off:off + F.out], O.gemv(F, M, x)[0], f"member {j} p{M} kernel {kern}")
+                off += F.out
+    Q.stagq_check(m)
     m.free()
