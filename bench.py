@@ -59,7 +59,7 @@ GROUP, N_PLANES, DENSITY = 128, 2, 0.005
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["quantized_gemv_stagq_b200/csrc/gemv.cu", "quantized_gemv_stagq_b200/csrc/gemv1.cu",
                   "quantized_gemv_stagq_b200/csrc/kernel_common.cuh", "quantized_gemv_stagq_b200/csrc/layout.cuh"]
-LARGE_WEIGHTS = 1 << 24  # above this many weights, n = 1 runs the single-vector kernel (gemv1)
+SINGLE_MAX_IN = 15 * 2048  # up to this many columns, n = 1 runs the single-vector kernel (gemv1)
 
 
 def _args():
@@ -166,8 +166,7 @@ def _launch_kernel(key):
     """Name of the kernel that serves the step launch `name@pM` at n = 1."""
     from quantized_gemv_stagq_b200 import synth
     members = dict(LAYER_LAUNCHES)[key.split("@")[0]]
-    weights = sum(synth.LLAMA31_8B_LINEARS[n][0] * synth.LLAMA31_8B_LINEARS[n][1] for n in members)
-    return "gemv1_kernel" if weights > LARGE_WEIGHTS else "gemv_kernel"
+    return "gemv1_kernel" if synth.LLAMA31_8B_LINEARS[members[0]][1] <= SINGLE_MAX_IN else "gemv_kernel"
 
 
 def _layer_shapes():
@@ -342,11 +341,12 @@ def run_extra(args):
             if (out, inp) not in streams:
                 streams[(out, inp)] = Q.stagq_pack(Q.stagq_encode(synth.weights(out, inp, seed=out + 3 * inp),
                                                                   group, n_planes, density, "fast", **enc))
-        shape = dict(linears)
-        groups = [("q", "k", "v"), ("o",), ("gate", "up"), ("down",)]
+        # linears come in the order q, k, v, o, gate, up, down
+        assert len(linears) == 7
+        groups = [(0, 1, 2), (3,), (4, 5), (6,)]
 
         def load():
-            return [Q.stagq_load_stack([streams[shape[n]] for n in grp], 0) for grp in groups]
+            return [Q.stagq_load_stack([streams[linears[i][1]] for i in grp], 0) for grp in groups]
         first = load()
         C = copies_for(Q, sum(m.device_bytes for m in first), l2, minimum=2)
         mats = [first] + [load() for _ in range(C - 1)]
