@@ -69,8 +69,8 @@ extern "C" {
 /* Flags of stagq_gemv_ex. */
 #define STAGQ_Y_F32 1u          /* y is fp32 instead of fp16 */
 /* Kernel choice for n = 1 (default: by shape and precision, see below). */
-#define STAGQ_KERNEL_GENERAL 2u /* the kernel of any vector count (two CTAs per SM on large matrices) */
-#define STAGQ_KERNEL_SINGLE 4u  /* the single-vector kernel (one CTA per SM beside the next GEMV's) */
+#define STAGQ_KERNEL_GENERAL 2u /* the kernel of any vector count (one or two CTAs per SM) */
+#define STAGQ_KERNEL_SINGLE 4u  /* the single-vector kernel (one CTA per SM, with the SM to itself) */
 
 typedef struct stagq_matrix* stagq_handle;   /* opaque; owned by the library */
 
@@ -249,9 +249,8 @@ int stagq_gemv_n(stagq_handle h, int bits, const void* x, int n, void* y, void* 
  * As stagq_gemv_n; flags STAGQ_Y_F32 makes y fp32. For n = 1 the library has
  * two kernels with the same arithmetic per vector (results agree to fp32
  * rounding, each is deterministic): by default the single-vector kernel
- * serves matrices of more than 2^24 weights or with groups below 64, where it
- * measured faster, and the
- * general kernel everything else.
+ * serves every n = 1 call whose K it can plan (K <= 30720), where it measured
+ * faster, and the general kernel the rest.
  * STAGQ_KERNEL_GENERAL / STAGQ_KERNEL_SINGLE force one of them (for tests and
  * measurements); forcing the single-vector kernel on a shape it cannot plan
  * returns STAGQ_EINVAL, and with n > 1 it is an error.

@@ -29,12 +29,12 @@
 //  * Two shuffle stages leave 8 partial sums per (row, K slice) in shared
 //    memory, and the slot goes back to the producer.
 //  * The held-out entries are taken apart from the blocks, where they would
-//    add a chain of dependent shared-memory reads to every block: each entry's
-//    local row is written once after the x conversion; after its blocks, every
-//    warp computes the terms x~_c (v - lo_M) of an equal share of the CTA's
-//    entries, independently of each other, into shared memory.
-//  * Finally one thread per row adds its partials and its entries' terms in a
-//    fixed order and stores y: deterministic, no atomics on data, no
+//    add a chain of dependent shared-memory reads to every block; a warp
+//    beside the blocks would have to compete with them for the shared memory.
+//  * Finally T lanes per row (T = 32 / rows per warp, as many as the CTA's
+//    threads allow) each add a share of the row's partials and of its held-out
+//    terms x~_c (v - lo_M); a fixed shuffle tree sums the T shares and the
+//    row's first lane stores y: deterministic, no atomics on data, no
 //    workspace, one launch.
 //  * Every mbarrier wait is bounded in time; on expiry the kernel records it
 //    in the handle's status word, waits (bounded) for its own copies and
@@ -77,7 +77,7 @@ constexpr uint64_t kDrainLimit1Ns = 100000000ull;  // after a failure: wait for 
 __host__ __device__ inline int part_stride1(int KW) { return KW * kParts1 + 4; }
 
 struct Smem1 {
-  uint32_t full, empty, side_bar, flag, stall, tab, xq, xscale, xsum, xsum16, pairs, side, part, rowid, term, ring;
+  uint32_t full, empty, side_bar, flag, stall, tab, xq, xscale, xsum, xsum16, pairs, side, part, ring;
   uint32_t slot;         // bytes of one ring slot
   uint32_t plane_piece;  // offset of the first read plane inside a slot (base rows at 0)
   uint32_t total;
@@ -87,7 +87,7 @@ __host__ __device__ inline uint32_t up16(uint32_t v) { return (v + 15u) & ~15u; 
 
 __host__ __device__ inline Smem1 smem1(const Gemv1Plan& p, int in, int M) {
   Smem1 L;
-  const uint32_t nchunk = in / kChunk, BR = p.br, rc = (uint32_t)p.rows_cap, sm = (uint32_t)p.side_max;
+  const uint32_t nchunk = in / kChunk, BR = p.br, rc = (uint32_t)p.rows_cap;
   uint32_t o = 0;
   L.full = o; o += 8 * kMaxSlots;    // block landed in the slot (producer arrive + bytes)
   L.empty = o; o += 8 * kMaxSlots;   // every consumer warp is done with the slot
@@ -105,8 +105,6 @@ __host__ __device__ inline Smem1 smem1(const Gemv1Plan& p, int in, int M) {
   L.side = o; o += p.stage_side ? (uint32_t)p.side_stride : 0u;
   o = up16(o);
   L.part = o; o += 4u * rc * (uint32_t)part_stride1(p.KW);
-  L.term = o; o += 4u * sm;          // x~_c (v - lo_M) of each held-out entry
-  L.rowid = o; o += up16(2u * sm);   // local row of each held-out entry
   o = (o + 127u) & ~127u;
   L.ring = o;
   L.plane_piece = BR * (in / 4);
@@ -161,8 +159,6 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
   float* xsum = reinterpret_cast<float*>(smem + L.xsum);
   float* xsum16 = reinterpret_cast<float*>(smem + L.xsum16);
   float* part = reinterpret_cast<float*>(smem + L.part);  // [row][part_stride1(KW)]: [KW][8] used
-  float* term = reinterpret_cast<float*>(smem + L.term);
-  uint16_t* rowid = reinterpret_cast<uint16_t*>(smem + L.rowid);
   volatile uint32_t* flag = reinterpret_cast<volatile uint32_t*>(smem + L.flag);
   const uint32_t full0 = sbase + L.full, empty0 = sbase + L.empty, side_bar = sbase + L.side_bar;
 
@@ -265,19 +261,9 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
       }
     }
   }
-  // Every warp takes the same branch: the term pass reads the entries' local
-  // rows, which all warps write.
+  // x~ is complete; every warp takes the same branch on the pair table, pair
+  // bytes and side record having landed.
   bool ok = __syncthreads_and(mbar_wait(side_bar, 0, kWaitLimit1Ns)) != 0;
-  const int32_t* offs = reinterpret_cast<const int32_t*>(side);
-  const uint32_t* ents = reinterpret_cast<const uint32_t*>(side + P.side_ent_off);
-  // local row of each held-out entry (a thread per row)
-  if (ok) {
-    for (int r = tid; r < rows; r += nthreads) {
-      const int j1 = offs[r + 1];
-      for (int j = offs[r]; j < j1; ++j) rowid[j] = (uint16_t)r;
-    }
-  }
-  __syncthreads();
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
@@ -393,64 +379,61 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
     }
   }
 
-  // ------------------------------------------------------------ side record
-  // Warp w takes entries [E w / (NW + 1), E (w + 1) / (NW + 1)), lane l every
-  // 32nd from l, four at a time; each term lands in its own slot.
-  if (ok) {
-    const int nw = NW + 1, E = offs[rows];
-    const int j0 = (int)((int64_t)E * warp / nw), j1 = (int)((int64_t)E * (warp + 1) / nw);
-    // pre-grid entry: v - lo_M; post-grid entry (bit 15): r + (lo - lo_M), Eq. (4)
-    auto terms = [&](auto with_post) {
-      for (int jb = j0 + lane; jb < j1; jb += 4 * 32) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int j = jb + 32 * k;
-          if (j < j1) {
-            const uint32_t en = ents[j];
-            const int col = (int)(en & 0x7FFFu);
-            const int e = xq_elem(col);         // the column's x~ slot (same 64-chunk as the column)
-            const int grp = col >> gs;          // the column's group
-            const int lrow = (int)rowid[j];
-            const int pb = pairs[lrow * ps + grp] + member_table_offset(a.m.mem_row, r0 + lrow);
-            const float v = __half2float(__ushort_as_half((unsigned short)(en >> 16)));
-            float d;
-            if constexpr (decltype(with_post)::value) {
-              if (en & 0x8000u) d = v + __ldg(a.dlo + pb);
-              else d = v - tab[pb].x;
-            } else {
-              d = v - tab[pb].x;
-            }
-            term[j] = (float)xq[e] * xscale[e >> 6] * d;
-          }
-        }
-      }
-    };
-    if (a.m.has_post) terms(std::true_type{});
-    else terms(std::false_type{});
-  }
   if (!ok && lane == 0) *flag = 1u;
   __syncthreads();
 
   if (*flag == 0u) {
     // ---------------------------------------------------------- y
-    for (int r = tid; r < rows; r += nthreads) {
-      // four interleaved sums (a fixed order), 16-byte loads of the partials
-      const float4* pr = reinterpret_cast<const float4*>(part + r * PST);
-      float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int k = 0; k < KW * kParts1 / 4; ++k) {
-        const float4 q = pr[k];
-        t.x += q.x; t.y += q.y; t.z += q.z; t.w += q.w;
+    // T lanes per row: lane sub of a row's group takes the row's partials
+    // (float4) sub, sub + T, ... and its held-out entries sub, sub + T, ...;
+    // a pre-grid entry adds x~_c (v - lo_M), a post-grid entry (bit 15)
+    // x~_c (r + lo - lo_M), Eq. (4).
+    const int32_t* offs = reinterpret_cast<const int32_t*>(side);
+    const uint32_t* ents = reinterpret_cast<const uint32_t*>(side + P.side_ent_off);
+    int T = 32;
+    while (T > 1 && rows * T > nthreads) T >>= 1;
+    const int sub = lane & (T - 1), rpw = 32 / T;  // rows per warp per pass
+    auto y_pass = [&](auto with_post) {
+      // warp-uniform trip count: every lane takes part in the shuffles
+      for (int rb = warp * rpw; rb < rows; rb += (nthreads / 32) * rpw) {
+        const int r = rb + lane / T;
+        float t0 = 0.f, t1 = 0.f, t2 = 0.f, t3 = 0.f;
+        if (r < rows) {
+          const float4* pr = reinterpret_cast<const float4*>(part + r * PST);
+          for (int k = sub; k < KW * kParts1 / 4; k += T) {
+            const float4 q = pr[k];
+            t0 += q.x; t1 += q.y; t2 += q.z; t3 += q.w;
+          }
+          const uint8_t* prow = pairs + r * ps;
+          const int moff = member_table_offset(a.m.mem_row, r0 + r);
+          auto term = [&](int j) {
+            const uint32_t en = ents[j];
+            const int col = (int)(en & 0x7FFFu);
+            const int e = xq_elem(col);  // the column's x~ slot (same 64-chunk as the column)
+            const int pb = prow[col >> gs] + moff;
+            const float v = __half2float(__ushort_as_half((unsigned short)(en >> 16)));
+            float d;
+            if constexpr (decltype(with_post)::value) d = (en & 0x8000u) ? v + __ldg(a.dlo + pb) : v - tab[pb].x;
+            else d = v - tab[pb].x;
+            return (float)xq[e] * xscale[e >> 6] * d;
+          };
+          const int e1 = offs[r + 1];
+          int j = offs[r] + sub;
+          for (; j + 3 * T < e1; j += 4 * T) {
+            t0 += term(j); t1 += term(j + T); t2 += term(j + 2 * T); t3 += term(j + 3 * T);
+          }
+          for (; j < e1; j += T) t0 += term(j);
+        }
+        float t = (t0 + t1) + (t2 + t3);
+        for (int o = T >> 1; o >= 1; o >>= 1) t += __shfl_xor_sync(kFull, t, o);
+        if (sub == 0 && r < rows) {
+          if (a.y_f32) reinterpret_cast<float*>(a.y)[r0 + r] = t;
+          else reinterpret_cast<__half*>(a.y)[r0 + r] = __float2half_rn(t);
+        }
       }
-      const int e1 = offs[r + 1];
-      int j = offs[r];
-      for (; j + 3 < e1; j += 4) {
-        t.x += term[j]; t.y += term[j + 1]; t.z += term[j + 2]; t.w += term[j + 3];
-      }
-      for (; j < e1; ++j) t.x += term[j];
-      const float acc = (t.x + t.y) + (t.z + t.w);
-      if (a.y_f32) reinterpret_cast<float*>(a.y)[r0 + r] = acc;
-      else reinterpret_cast<__half*>(a.y)[r0 + r] = __float2half_rn(acc);
-    }
+    };
+    if (a.m.has_post) y_pass(std::true_type{});
+    else y_pass(std::false_type{});
   } else if (tid == 0) {
     atomicOr(a.m.status, 1u);
     // Gave up: let this CTA's copies in flight land before it exits.
