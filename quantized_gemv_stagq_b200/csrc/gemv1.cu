@@ -29,13 +29,17 @@
 //  * Two shuffle stages leave 8 partial sums per (row, K slice) in shared
 //    memory, and the slot goes back to the producer.
 //  * The held-out entries are taken apart from the blocks, where they would
-//    add a chain of dependent shared-memory reads to every block; a warp
-//    beside the blocks would have to compete with them for the shared memory.
-//  * Finally T lanes per row (T = 32 / rows per warp, as many as the CTA's
-//    threads allow) each add a share of the row's partials and of its held-out
-//    terms x~_c (v - lo_M); a fixed shuffle tree sums the T shares and the
-//    row's first lane stores y: deterministic, no atomics on data, no
-//    workspace, one launch.
+//    add a chain of dependent shared-memory reads to every block. T lanes per
+//    row (T = 32 / rows per warp, as many as the CTA's threads allow) each sum
+//    a share of the row's terms x~_c (v - lo_M), and a fixed shuffle tree adds
+//    the shares: right after the x conversion, into one float per row, where
+//    the CTA refills ring slots (the later slots land meanwhile); otherwise in
+//    the final pass.
+//  * Finally T lanes per row add the row's partials the same way, with the
+//    row's held-out terms, and the row's first lane stores y: deterministic,
+//    no atomics on data, no workspace, one launch.
+//  * x is read before the copies of all but the first block are issued: those
+//    copies would otherwise delay the L2 reads of x that every warp waits for.
 //  * Every mbarrier wait is bounded in time; on expiry the kernel records it
 //    in the handle's status word, waits (bounded) for its own copies and
 //    returns.
@@ -77,7 +81,7 @@ constexpr uint64_t kDrainLimit1Ns = 100000000ull;  // after a failure: wait for 
 __host__ __device__ inline int part_stride1(int KW) { return KW * kParts1 + 4; }
 
 struct Smem1 {
-  uint32_t full, empty, side_bar, flag, stall, tab, xq, xscale, xsum, xsum16, pairs, side, part, ring;
+  uint32_t full, empty, side_bar, flag, stall, tab, xq, xscale, xsum, xsum16, pairs, side, part, rowterm, ring;
   uint32_t slot;         // bytes of one ring slot
   uint32_t plane_piece;  // offset of the first read plane inside a slot (base rows at 0)
   uint32_t total;
@@ -105,6 +109,7 @@ __host__ __device__ inline Smem1 smem1(const Gemv1Plan& p, int in, int M) {
   L.side = o; o += p.stage_side ? (uint32_t)p.side_stride : 0u;
   o = up16(o);
   L.part = o; o += 4u * rc * (uint32_t)part_stride1(p.KW);
+  L.rowterm = o; o += 4u * rc;       // each row's sum of x~_c (v - lo_M) over its held-out entries
   o = (o + 127u) & ~127u;
   L.ring = o;
   L.plane_piece = BR * (in / 4);
@@ -159,6 +164,7 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
   float* xsum = reinterpret_cast<float*>(smem + L.xsum);
   float* xsum16 = reinterpret_cast<float*>(smem + L.xsum16);
   float* part = reinterpret_cast<float*>(smem + L.part);  // [row][part_stride1(KW)]: [KW][8] used
+  float* rowterm = reinterpret_cast<float*>(smem + L.rowterm);
   volatile uint32_t* flag = reinterpret_cast<volatile uint32_t*>(smem + L.flag);
   const uint32_t full0 = sbase + L.full, empty0 = sbase + L.empty, side_bar = sbase + L.side_bar;
 
@@ -171,6 +177,16 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
   const int rb = in / 4, rp = in / 8;
   const uint8_t* side_g = a.m.side1 + (int64_t)blockIdx.x * P.side_stride;
   const uint8_t* pair_g = a.m.pair + (int64_t)r0 * ps;
+  // Parameters of the later phases, read here with the first ones: the first
+  // read of a parameter's cache line in a launch waits about as long as a
+  // load from L2, and this way those waits overlap instead of adding up.
+  const uint4* const x4 = reinterpret_cast<const uint4*>(a.x);
+  const float4* const s4 = reinterpret_cast<const float4*>(a.in_scale);
+  void* const yout = a.y;
+  const float* const dlo = a.dlo;
+  const int y_f32 = a.y_f32, has_post = a.m.has_post;
+  const uint32_t side_ent_off = (uint32_t)P.side_ent_off;
+  asm volatile("" ::"l"(x4), "l"(s4), "l"(yout), "l"(dlo), "r"(y_f32), "r"(has_post), "r"(side_ent_off));
   const uint8_t* pairs = smem + L.pairs;
   const uint8_t* side = P.stage_side ? smem + L.side : side_g;
 
@@ -208,7 +224,9 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
     bulk_load(sbase + L.tab, a.table, 256 * 8 * (uint32_t)P.nmem, side_bar);
     bulk_load(sbase + L.pairs, pair_g, pb, side_bar);
     if (sb) bulk_load(sbase + L.side, side_g, sb, side_bar);
-    for (int b = 0; b < NS && b < nblk; ++b) issue_block(b, b);
+    // Only the first block before x: the copies of later blocks would delay
+    // the L2 reads of x that every warp waits for.
+    if (nblk > 0) issue_block(0, 0);
   }
   grid_launch_dependents();
   grid_dependency_wait();  // x may come from the previous kernel; y may be read by it
@@ -221,8 +239,6 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
   {
     constexpr int kBatch = 4;
     const int ntask = 4 * nchunk;
-    const uint4* x4 = reinterpret_cast<const uint4*>(a.x);
-    const float4* s4 = reinterpret_cast<const float4*>(a.in_scale);
     for (int t0 = 0; t0 < ntask; t0 += kBatch * nthreads) {
       uint4 raw[kBatch][2];
       float4 sv[kBatch][4];
@@ -264,6 +280,74 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
   // x~ is complete; every warp takes the same branch on the pair table, pair
   // bytes and side record having landed.
   bool ok = __syncthreads_and(mbar_wait(side_bar, 0, kWaitLimit1Ns)) != 0;
+  if (tid == 0)
+    for (int b = issued; b < NS && b < nblk; ++b) issue_block(b, b);
+
+  // T lanes per row (as many as the CTA's threads allow, up to a warp) for the
+  // per-row passes below; rpw rows per warp at a time.
+  int T = 32;
+  while (T > 1 && rows * T > nthreads) T >>= 1;
+  const int sub = lane & (T - 1), rpw = 32 / T;
+  // ------------------------------------------------ per-row passes
+  // Lane sub of a row's group takes the row's partials (float4) sub, sub + T,
+  // ... (final pass) and its held-out entries sub, sub + T, ... (terms); a
+  // pre-grid entry adds x~_c (v - lo_M), a post-grid entry (bit 15)
+  // x~_c (r + lo - lo_M), Eq. (4). A fixed shuffle tree sums the T shares.
+  // Where the CTA refills ring slots, the terms are summed before the blocks,
+  // while the later slots are landing, into one float per row; otherwise in
+  // the final pass, where they cost less than delaying the only blocks.
+  const bool terms_first = nblk > NS;
+  const int32_t* offs = reinterpret_cast<const int32_t*>(side);
+  const uint32_t* ents = reinterpret_cast<const uint32_t*>(side + side_ent_off);
+  auto row_pass = [&](auto with_post, bool terms, bool final) {
+    for (int rb = warp * rpw; rb < rows; rb += (nthreads / 32) * rpw) {  // warp-uniform trip count
+      const int r = rb + lane / T;
+      float t0 = 0.f, t1 = 0.f, t2 = 0.f, t3 = 0.f;
+      if (r < rows && final) {
+        const float4* pr = reinterpret_cast<const float4*>(part + r * PST);
+        for (int k = sub; k < KW * kParts1 / 4; k += T) {
+          const float4 q = pr[k];
+          t0 += q.x; t1 += q.y; t2 += q.z; t3 += q.w;
+        }
+      }
+      if (r < rows && terms) {
+        const uint8_t* prow = pairs + r * ps;
+        const int moff = member_table_offset(a.m.mem_row, r0 + r);
+        auto term = [&](int j) {
+          const uint32_t en = ents[j];
+          const int col = (int)(en & 0x7FFFu);
+          const int e = xq_elem(col);  // the column's x~ slot (same 64-chunk as the column)
+          const int pb = prow[col >> gs] + moff;
+          const float v = __half2float(__ushort_as_half((unsigned short)(en >> 16)));
+          float d;
+          if constexpr (decltype(with_post)::value) d = (en & 0x8000u) ? v + __ldg(dlo + pb) : v - tab[pb].x;
+          else d = v - tab[pb].x;
+          return (float)xq[e] * xscale[e >> 6] * d;
+        };
+        const int e1 = offs[r + 1];
+        int j = offs[r] + sub;
+        for (; j + 3 * T < e1; j += 4 * T) {
+          t0 += term(j); t1 += term(j + T); t2 += term(j + 2 * T); t3 += term(j + 3 * T);
+        }
+        for (; j < e1; j += T) t0 += term(j);
+      }
+      float t = (t0 + t1) + (t2 + t3);
+      for (int o = T >> 1; o >= 1; o >>= 1) t += __shfl_xor_sync(kFull, t, o);
+      if (sub == 0 && r < rows) {
+        if (!final) {
+          rowterm[r] = t;
+        } else {
+          if (!terms) t += rowterm[r];
+          if (y_f32) reinterpret_cast<float*>(yout)[r0 + r] = t;
+          else reinterpret_cast<__half*>(yout)[r0 + r] = __float2half_rn(t);
+        }
+      }
+    }
+  };
+  if (ok && terms_first) {
+    if (has_post) row_pass(std::true_type{}, true, false);
+    else row_pass(std::false_type{}, true, false);
+  }
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
@@ -384,56 +468,8 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
 
   if (*flag == 0u) {
     // ---------------------------------------------------------- y
-    // T lanes per row: lane sub of a row's group takes the row's partials
-    // (float4) sub, sub + T, ... and its held-out entries sub, sub + T, ...;
-    // a pre-grid entry adds x~_c (v - lo_M), a post-grid entry (bit 15)
-    // x~_c (r + lo - lo_M), Eq. (4).
-    const int32_t* offs = reinterpret_cast<const int32_t*>(side);
-    const uint32_t* ents = reinterpret_cast<const uint32_t*>(side + P.side_ent_off);
-    int T = 32;
-    while (T > 1 && rows * T > nthreads) T >>= 1;
-    const int sub = lane & (T - 1), rpw = 32 / T;  // rows per warp per pass
-    auto y_pass = [&](auto with_post) {
-      // warp-uniform trip count: every lane takes part in the shuffles
-      for (int rb = warp * rpw; rb < rows; rb += (nthreads / 32) * rpw) {
-        const int r = rb + lane / T;
-        float t0 = 0.f, t1 = 0.f, t2 = 0.f, t3 = 0.f;
-        if (r < rows) {
-          const float4* pr = reinterpret_cast<const float4*>(part + r * PST);
-          for (int k = sub; k < KW * kParts1 / 4; k += T) {
-            const float4 q = pr[k];
-            t0 += q.x; t1 += q.y; t2 += q.z; t3 += q.w;
-          }
-          const uint8_t* prow = pairs + r * ps;
-          const int moff = member_table_offset(a.m.mem_row, r0 + r);
-          auto term = [&](int j) {
-            const uint32_t en = ents[j];
-            const int col = (int)(en & 0x7FFFu);
-            const int e = xq_elem(col);  // the column's x~ slot (same 64-chunk as the column)
-            const int pb = prow[col >> gs] + moff;
-            const float v = __half2float(__ushort_as_half((unsigned short)(en >> 16)));
-            float d;
-            if constexpr (decltype(with_post)::value) d = (en & 0x8000u) ? v + __ldg(a.dlo + pb) : v - tab[pb].x;
-            else d = v - tab[pb].x;
-            return (float)xq[e] * xscale[e >> 6] * d;
-          };
-          const int e1 = offs[r + 1];
-          int j = offs[r] + sub;
-          for (; j + 3 * T < e1; j += 4 * T) {
-            t0 += term(j); t1 += term(j + T); t2 += term(j + 2 * T); t3 += term(j + 3 * T);
-          }
-          for (; j < e1; j += T) t0 += term(j);
-        }
-        float t = (t0 + t1) + (t2 + t3);
-        for (int o = T >> 1; o >= 1; o >>= 1) t += __shfl_xor_sync(kFull, t, o);
-        if (sub == 0 && r < rows) {
-          if (a.y_f32) reinterpret_cast<float*>(a.y)[r0 + r] = t;
-          else reinterpret_cast<__half*>(a.y)[r0 + r] = __float2half_rn(t);
-        }
-      }
-    };
-    if (a.m.has_post) y_pass(std::true_type{});
-    else y_pass(std::false_type{});
+    if (has_post) row_pass(std::true_type{}, !terms_first, true);
+    else row_pass(std::false_type{}, !terms_first, true);
   } else if (tid == 0) {
     atomicOr(a.m.status, 1u);
     // Gave up: let this CTA's copies in flight land before it exits.
