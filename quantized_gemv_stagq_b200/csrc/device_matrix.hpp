@@ -101,6 +101,7 @@ struct Gemv1Plan {
   int up, br;            // rows per warp per block, rows per block (RG * up)
   int ns;                // ring slots
   int rows_cap;          // most rows of one CTA
+  int rows_q, rows_rem;  // out = rows_q * grid + rows_rem: CTA b starts at row b rows_q + floor(b rows_rem / grid)
   int stage_side;        // the CTA's side record is copied into shared memory
   int side_stride, side_ent_off, side_max;
   int group_shift;       // log2(group)

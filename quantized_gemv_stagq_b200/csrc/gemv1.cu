@@ -171,8 +171,11 @@ __global__ void __maxnreg__(kRegs1) gemv1_kernel(const Gemv1Args a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthreads = blockDim.x;
   const int KW = P.KW, NW = P.NW, NS = P.ns, BR = P.br, ps = P.pair_stride, gs = P.group_shift;
   const int PST = part_stride1(KW);
-  const int r0 = (int)((int64_t)blockIdx.x * a.m.out / gridDim.x);
-  const int rows = (int)((int64_t)(blockIdx.x + 1) * a.m.out / gridDim.x) - r0;
+  // rows [b out / grid, (b + 1) out / grid) of CTA b, without a 64-bit division
+  const uint32_t bx = blockIdx.x, gx = gridDim.x;
+  const int f0 = (int)(bx * (uint32_t)P.rows_rem / gx), f1 = (int)((bx + 1) * (uint32_t)P.rows_rem / gx);
+  const int r0 = (int)bx * P.rows_q + f0;
+  const int rows = P.rows_q + f1 - f0;
   const int nblk = (rows + BR - 1) / BR;
   const int rb = in / 4, rp = in / 8;
   const uint8_t* side_g = a.m.side1 + (int64_t)blockIdx.x * P.side_stride;
@@ -619,6 +622,8 @@ bool make_plan1(const DeviceMatrix& m, int bits, Gemv1Plan* p) {
   q.grid = m.side1_grid;
   if (q.grid < 1) return false;
   q.rows_cap = (m.out + q.grid - 1) / q.grid;
+  q.rows_q = m.out / q.grid;
+  q.rows_rem = m.out % q.grid;
   q.pair_stride = m.pair_stride;
   q.side_stride = m.side1_stride;
   q.side_ent_off = m.side1_ent_off;
