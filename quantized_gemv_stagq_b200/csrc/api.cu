@@ -20,8 +20,8 @@ struct stagq_matrix {
   stagq::DeviceMatrix dm{};
   stagq::GemvPlan plan[7][STAGQ_MAX_BATCH + 1]{};  // per precision (bits) and vector count
   bool plan_ok[7][STAGQ_MAX_BATCH + 1]{};
-  stagq::Gemv1Plan plan1[7]{};   // single-vector kernel, per precision
-  bool plan1_ok[7]{};
+  stagq::Gemv1Plan plan1[7][STAGQ_MAX_BATCH + 1]{};  // single-vector kernel, per precision and vector count
+  bool plan1_ok[7][STAGQ_MAX_BATCH + 1]{};
   bool prefer1[7]{};             // the single-vector kernel serves n = 1 by default
   void* d_mem = nullptr;
   size_t d_bytes = 0;
@@ -281,7 +281,7 @@ int load_impl(const stagq_host_stream* s, const stagq_host_stream* const* member
   // this measured 24 % faster than giving the general kernel (whose CTAs share
   // an SM) the matrices of up to 2^24 weights.
   for (int b = 2; b <= 2 + np; ++b) {
-    h->plan1_ok[b] = make_plan1(m, b, &h->plan1[b]);
+    for (int nb = 1; nb <= STAGQ_MAX_BATCH; ++nb) h->plan1_ok[b][nb] = make_plan1(m, b, nb, &h->plan1[b][nb]);
     h->prefer1[b] = true;
   }
   if (!h->plan_ok[2][1]) {
@@ -384,15 +384,15 @@ int gemv_impl(stagq_handle h, int bits, const void* x, int n, const float* in_sc
   if (flags & ~(STAGQ_Y_F32 | STAGQ_KERNEL_GENERAL | STAGQ_KERNEL_SINGLE)) return fail(STAGQ_EINVAL, "unknown flags");
   const bool force_general = flags & STAGQ_KERNEL_GENERAL, force_single = flags & STAGQ_KERNEL_SINGLE;
   if (force_general && force_single) return fail(STAGQ_EINVAL, "both kernels forced");
-  if (force_single && (n != 1 || !h->plan1_ok[bits]))
-    return fail(STAGQ_EINVAL, "the single-vector kernel serves n = 1 on shapes it can plan");
+  if (force_single && !h->plan1_ok[bits][n])
+    return fail(STAGQ_EINVAL, "the single-vector kernel cannot plan this shape and vector count");
   DeviceGuard guard(h->device);
   if (!guard.ok) return fail(STAGQ_ECUDA, "cudaSetDevice failed");
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   const int yf32 = (flags & STAGQ_Y_F32) ? 1 : 0;
   const size_t ysz = yf32 ? 4 : 2;
-  if (force_single || (n == 1 && !force_general && h->plan1_ok[bits] && h->prefer1[bits])) {
-    cudaError_t e = launch_gemv1(h->dm, h->plan1[bits], bits, x, in_scale, y, yf32, stream);
+  if (force_single || (!force_general && h->plan1_ok[bits][n] && h->prefer1[bits])) {
+    cudaError_t e = launch_gemv1(h->dm, h->plan1[bits][n], bits, x, in_scale, y, yf32, stream);
     if (e != cudaSuccess) return cuda_fail(e, "GEMV launch");
     return STAGQ_OK;
   }

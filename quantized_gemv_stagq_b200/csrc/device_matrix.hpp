@@ -96,6 +96,7 @@ struct GemvPlan {
 
 // Launch plan of the single-vector kernel (gemv1.cu).
 struct Gemv1Plan {
+  int nb;                // activation vectors (1..4); above 1 a lane takes half a chunk
   int grid;              // CTAs (= side1_grid, at most one per SM)
   int KW, RG, NW;        // K slices, row groups, consumer warps (KW * RG); one producer warp more
   int up, br;            // rows per warp per block, rows per block (RG * up)
@@ -110,9 +111,9 @@ struct Gemv1Plan {
   int nmem;              // stacked members (pair tables)
 };
 
-// Plan for the single-vector kernel at `bits`; false if it cannot be planned
-// (the general kernel then serves n = 1 too).
-bool make_plan1(const DeviceMatrix& m, int bits, Gemv1Plan* plan);
+// Plan for the single-vector kernel at `bits` with `nb` activation vectors;
+// false if it cannot be planned (the general kernel then serves the call).
+bool make_plan1(const DeviceMatrix& m, int bits, int nb, Gemv1Plan* plan);
 int gemv1_grid(int out, int num_sms);
 // in_scale: null, or device fp32 [in] multiplying x channel by channel first.
 cudaError_t launch_gemv1(const DeviceMatrix& m, const Gemv1Plan& plan, int bits, const void* x, const float* in_scale,

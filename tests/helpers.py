@@ -61,3 +61,16 @@ def n1_kernels(inp, include_default=False):
     if inp <= SINGLE_MAX_IN:
         ks.append(Q.STAGQ_KERNEL_SINGLE)
     return tuple(ks)
+
+
+# With several vectors a lane of the single-vector kernel takes half a chunk:
+# it plans K up to 15 slices of 1024 weights, for groups of 64 or more.
+SINGLE_MAX_IN_NB = 15 * 1024
+
+
+def nb_kernels(inp, group):
+    """The kernels that can serve n = 2..4 vectors of a matrix with K = inp."""
+    ks = [Q.STAGQ_KERNEL_GENERAL]
+    if inp <= SINGLE_MAX_IN_NB and group >= 64:
+        ks.append(Q.STAGQ_KERNEL_SINGLE)
+    return tuple(ks)

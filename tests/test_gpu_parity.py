@@ -13,7 +13,7 @@ torch = pytest.importorskip("torch")
 import quantized_gemv_stagq_b200 as Q
 from oracle import stagq as O
 from quantized_gemv_stagq_b200 import synth
-from tests.helpers import check_close, fields_equal, lib_columns, n1_kernels, to_lib_fields
+from tests.helpers import check_close, fields_equal, lib_columns, n1_kernels, nb_kernels, to_lib_fields
 
 pytestmark = pytest.mark.gpu
 
@@ -98,10 +98,13 @@ def test_batched_gemv_matches_oracle(case):
         x = synth.activations(n, inp, seed + 200 + n)
         for M in range(2, 3 + npl):
             ref = O.gemv(F, M, x)
-            got = _gemv(m, M, x, f32=True)
-            for j in range(n):
-                check_close(got[j], ref[j], f"n{n} col{j} p{M}")
-            # each column equals the single-vector launch of that column (same kernel arithmetic)
+            for kern in (0,) + nb_kernels(inp, g):  # the default and every kernel that serves n > 1
+                got = _gemv(m, M, x, f32=True, kernel=kern)
+                for j in range(n):
+                    check_close(got[j], ref[j], f"n{n} col{j} p{M} kernel {kern}")
+                got16 = _gemv(m, M, x, f32=False, kernel=kern).astype(np.float64)
+                check_close(got16[n - 1], ref[n - 1], f"n{n} fp16 last col p{M} kernel {kern}")
+            # each column agrees with the single-vector launch of that column
             one = _gemv(m, M, x[n - 1:n], f32=True)
             check_close(got[n - 1:n], one, f"n{n} last col vs n1 p{M}")
     Q.stagq_check(m)
@@ -187,8 +190,12 @@ def test_bad_calls_return_errors():
         Q.stagq_gemv_ex(m, 2, x, y, flags=Q.STAGQ_KERNEL_GENERAL | Q.STAGQ_KERNEL_SINGLE)
     x4 = torch.zeros(4, 512, dtype=torch.float16, device="cuda")
     y4 = torch.zeros(4, 64, dtype=torch.float16, device="cuda")
-    with pytest.raises(Q.StagqError):  # the single-vector kernel with n > 1
-        Q.stagq_gemv_ex(m, 2, x4, y4, n=4, flags=Q.STAGQ_KERNEL_SINGLE)
+    m32 = _load(O.encode(synth.weights(64, 512, 42), 32, 2, 0.005, "fast"))
+    with pytest.raises(Q.StagqError):  # the single-vector kernel with n > 1 and groups below 64
+        Q.stagq_gemv_ex(m32, 2, x4, y4, n=4, flags=Q.STAGQ_KERNEL_SINGLE)
+    Q.stagq_gemv_ex(m, 2, x4, y4, n=4, flags=Q.STAGQ_KERNEL_SINGLE)  # groups of 128: planned
+    torch.cuda.synchronize()
+    m32.free()
     m.free()
 
 
@@ -220,10 +227,11 @@ def _sampled_rows_case(out, inp, group, n_planes, density, seed, bits_list, kern
             check_close(y[rows].astype(np.float64), ref1, f"{out}x{inp} p{M} kernel {kern}")
             assert np.all(np.isfinite(y))
         if batch4:
-            y4 = _gemv(m, M, x, f32=False)  # batch 4 in one launch
             ref4 = O.gemv(F, M, x)
-            for j in range(4):
-                check_close(y4[j][rows].astype(np.float64), ref4[j], f"{out}x{inp} p{M} n4 col{j}")
+            for kern in (0,) + nb_kernels(inp, group):  # batch 4 in one launch
+                y4 = _gemv(m, M, x, f32=False, kernel=kern)
+                for j in range(4):
+                    check_close(y4[j][rows].astype(np.float64), ref4[j], f"{out}x{inp} p{M} n4 col{j} kernel {kern}")
     Q.stagq_check(m)
     m.free()
 
@@ -444,9 +452,10 @@ def test_scaled_gemv_matches_oracle(case):
         ref = O.gemv(F, M, x, in_scale=s)
         for kern in (Q.STAGQ_KERNEL_GENERAL, Q.STAGQ_KERNEL_SINGLE):
             check_close(_gemv_scaled(m, M, x[:1], s, kernel=kern)[0], ref[0], f"p{M} kernel {kern}")
-        got = _gemv_scaled(m, M, x, s)
-        for j in range(4):
-            check_close(got[j], ref[j], f"p{M} n4 col{j}")
+        for kern in (0,) + nb_kernels(inp, g):
+            got = _gemv_scaled(m, M, x, s, kernel=kern)
+            for j in range(4):
+                check_close(got[j], ref[j], f"p{M} n4 col{j} kernel {kern}")
         # a scale of ones is the unscaled GEMV
         ones = _gemv_scaled(m, M, x[:1], np.ones(inp, np.float32))
         check_close(ones[0], O.gemv(F, M, x[:1])[0], f"p{M} ones")
