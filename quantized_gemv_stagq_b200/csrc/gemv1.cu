@@ -160,17 +160,18 @@ __device__ __forceinline__ bool keeps_partial1(int lane) {
 // pair w = h, and the x~ of the half are chunk words 16 h .. 16 h + 15.
 
 // The half chunk's masked code words, decoded once for every vector:
-// cw[0..7] as chunk_codes for one word pair (M = 2: base word i & (0x03030303
-// << 2 s) at 4 i + s; M >= 3: the nibble composites' low / high nibbles), and
+// cw[0..7] as chunk_codes for one word pair (M = 2: the bytes q of base word i,
+// slot s, (word >> 2 s) & 0x03030303, at 4 i + s; M >= 3: the nibble
+// composites' low / high nibbles), and
 // for M >= 5 the plane-5 / plane-6 bits of base word i, slot s, at 4 i + s.
 template <int M>
 __device__ __forceinline__ void half_codes(uint2 B, const uint32_t* P, uint32_t (&cw)[8], uint32_t (&c5)[8],
                                            uint32_t (&c6)[8]) {
-  if constexpr (M == 2) {
+  if constexpr (M == 2) {  // shifted down to bytes q, so that one sum serves every slot
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
-      cw[s] = B.x & (0x03030303u << (2 * s));
-      cw[4 + s] = B.y & (0x03030303u << (2 * s));
+      cw[s] = (B.x >> (2 * s)) & 0x03030303u;
+      cw[4 + s] = (B.y >> (2 * s)) & 0x03030303u;
     }
   } else {
     uint32_t E0, O0, E1, O1;
@@ -204,12 +205,13 @@ template <int M>
 __device__ __forceinline__ int half_dot(const uint32_t (&X)[16], const uint32_t (&cw)[8], const uint32_t (&c5)[8],
                                         const uint32_t (&c6)[8]) {
   if constexpr (M == 2) {
-    int a[4] = {0, 0, 0, 0};
+    int a0 = 0, a1 = 0;  // two chains for latency
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-      for (int s = 0; s < 4; ++s) a[s] = hdot4(X, i, s, cw[4 * i + s], a[s]);
-    return a[0] + (a[1] >> 2) + (a[2] >> 4) + (a[3] >> 6);  // slot s carries q 4^s
+    for (int s = 0; s < 4; ++s) {
+      a0 = hdot4(X, 0, s, cw[s], a0);
+      a1 = hdot4(X, 1, s, cw[4 + s], a1);
+    }
+    return a0 + a1;
   } else {
     int lo = 0, hi = 0;
     lo = hdot4(X, 0, 1, cw[0], lo);
