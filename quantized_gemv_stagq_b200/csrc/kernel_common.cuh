@@ -261,8 +261,10 @@ __device__ __forceinline__ int chunk_dot(const uint32_t (&X)[32], const uint32_t
 // inverse activation scale s (16 fp32 values; the quantiser saw W diag(a), so
 // channel c of x is multiplied by 1/a_c, Appendix E), rounded to fp32.
 // Scale 2^e with max|x| 2^e in [2^14, 2^15) over the chunk, so the largest
-// entries convert exactly; rounding to nearest even goes through the 1.5 *
-// 2^23 shifter (the low 16 bits of the sum are the two's-complement integer).
+// entries of fp16 x convert exactly; rounding to nearest even goes through the
+// 1.5 * 2^23 shifter (the low 16 bits of the sum are the two's-complement
+// integer). With SC the largest scaled fp32 product can round up to 2^15, so
+// the result is clamped to 2^15 - 1.
 // Out: Q (8 pairs of int16), xs = 2^-e, sum16 = the task's sum of x~, sumq =
 // the chunk's.
 template <bool SC>
@@ -297,7 +299,12 @@ __device__ __forceinline__ void convert_x_task(const uint4 (&raw)[2], const floa
   sumq = 0;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    Q[k] = __byte_perm(__float_as_uint(fmaf(f[k].x, sc, kShift)), __float_as_uint(fmaf(f[k].y, sc, kShift)), 0x5410);
+    float vx = fmaf(f[k].x, sc, kShift), vy = fmaf(f[k].y, sc, kShift);
+    if constexpr (SC) {  // |x s| 2^e < 2^15 before rounding; keep the rounded value inside int16
+      vx = fminf(fmaxf(vx, kShift - 32768.f), kShift + 32767.f);
+      vy = fminf(fmaxf(vy, kShift - 32768.f), kShift + 32767.f);
+    }
+    Q[k] = __byte_perm(__float_as_uint(vx), __float_as_uint(vy), 0x5410);
     sumq = dp2a_lo(Q[k], 0x0101u, sumq);
   }
   sum16 = sumq;

@@ -463,6 +463,27 @@ def test_scaled_gemv_matches_oracle(case):
     m.free()
 
 
+def test_scaled_product_that_rounds_to_the_int16_limit():
+    """x = 1 and s = 1 - 2^-17: every scaled product is 32767.75 after the
+    chunk's power-of-two scale, which rounds to 2^15; the fixed-point value
+    must stay inside int16 (a wrapped -2^15 would flip the sign of the chunk)."""
+    out, inp = 64, 512
+    F = O.encode(synth.weights(out, inp, 43), 128, 2, 0.005, "fast")
+    m = _load(F)
+    s = np.full(inp, 1.0 - 2.0 ** -17, np.float32)
+    x = np.ones((4, inp), np.float16)
+    for M in (2, 3, 4):
+        ref = O.gemv(F, M, x, in_scale=s)
+        for kern in (Q.STAGQ_KERNEL_GENERAL, Q.STAGQ_KERNEL_SINGLE):
+            check_close(_gemv_scaled(m, M, x[:1], s, kernel=kern)[0], ref[0], f"p{M} kernel {kern}")
+        for kern in (0, Q.STAGQ_KERNEL_GENERAL):
+            got = _gemv_scaled(m, M, x, s, kernel=kern)
+            for j in range(4):
+                check_close(got[j], ref[j], f"p{M} n4 col{j} kernel {kern}")
+    Q.stagq_check(m)
+    m.free()
+
+
 @pytest.mark.parametrize("name", ["gate_proj", "q_proj"])
 def test_full_size_scaled_sampled_rows(name):
     """The Llama-3.1-8B gate (single-vector kernel) and q (general kernel)
