@@ -246,14 +246,16 @@ int stagq_gemv(stagq_handle h, int bits, const void* x, void* y, void* cuda_stre
 int stagq_gemv_n(stagq_handle h, int bits, const void* x, int n, void* y, void* cuda_stream);
 
 /*
- * As stagq_gemv_n; flags STAGQ_Y_F32 makes y fp32. For n = 1 the library has
- * two kernels with the same arithmetic per vector (results agree to fp32
- * rounding, each is deterministic): by default the single-vector kernel
- * serves every n = 1 call whose K it can plan (K <= 30720), where it measured
- * faster, and the general kernel the rest.
- * STAGQ_KERNEL_GENERAL / STAGQ_KERNEL_SINGLE force one of them (for tests and
- * measurements); forcing the single-vector kernel on a shape it cannot plan
- * returns STAGQ_EINVAL, and with n > 1 it is an error.
+ * As stagq_gemv_n; flags STAGQ_Y_F32 makes y fp32. The library has two
+ * kernels with the same integer dot products (results agree to fp32
+ * rounding, each is deterministic). By default the single-vector kernel
+ * serves every call it can plan, where it measured faster:
+ *   - n = 1 with K <= 30720;
+ *   - n = 2..4 with K <= 15360 and groups of 64 or more.
+ * The general kernel serves the rest.
+ * STAGQ_KERNEL_GENERAL / STAGQ_KERNEL_SINGLE force one of them, for tests and
+ * measurements. Forcing the single-vector kernel on a shape and n it cannot
+ * plan returns STAGQ_EINVAL.
  */
 int stagq_gemv_ex(stagq_handle h, int bits, const void* x, int n, void* y, uint32_t flags,
                   void* cuda_stream);
