@@ -68,7 +68,7 @@ extern "C" {
 
 /* Flags of stagq_gemv_ex. */
 #define STAGQ_Y_F32 1u          /* y is fp32 instead of fp16 */
-/* Kernel choice for n = 1 (default: by shape and precision, see below). */
+/* Kernel choice (default: by shape and vector count, see stagq_gemv_ex). */
 #define STAGQ_KERNEL_GENERAL 2u /* the kernel of any vector count (one or two CTAs per SM) */
 #define STAGQ_KERNEL_SINGLE 4u  /* the single-vector kernel (one CTA per SM, with the SM to itself) */
 

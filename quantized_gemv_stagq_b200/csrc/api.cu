@@ -22,7 +22,7 @@ struct stagq_matrix {
   bool plan_ok[7][STAGQ_MAX_BATCH + 1]{};
   stagq::Gemv1Plan plan1[7][STAGQ_MAX_BATCH + 1]{};  // single-vector kernel, per precision and vector count
   bool plan1_ok[7][STAGQ_MAX_BATCH + 1]{};
-  bool prefer1[7]{};             // the single-vector kernel serves n = 1 by default
+  bool prefer1[7]{};             // the single-vector kernel serves the calls it can plan by default
   void* d_mem = nullptr;
   size_t d_bytes = 0;
   void* d_stage = nullptr;      // x / y staging for stagq_gemv_host
@@ -275,11 +275,13 @@ int load_impl(const stagq_host_stream* s, const stagq_host_stream* const* member
   if (m.smem_pair_budget > smem_limit) m.smem_pair_budget = smem_limit;
   for (int b = 2; b <= 2 + np; ++b)
     for (int nb = 1; nb <= STAGQ_MAX_BATCH; ++nb) h->plan_ok[b][nb] = make_plan(m, b, nb, &h->plan[b][nb]);
-  // The single-vector kernel serves every n = 1 launch it can plan: one CTA
-  // per SM that has the SM to itself. A chain of launches of one shape of CTA
-  // stays evenly placed (see make_plan1); on the Llama-3.1-8B layer chain
-  // this measured 24 % faster than giving the general kernel (whose CTAs share
-  // an SM) the matrices of up to 2^24 weights.
+  // The single-vector kernel serves every launch it can plan (n = 1, and
+  // n = 2..4 with groups of 64 or more): one CTA per SM that has the SM to
+  // itself. A chain of launches of one shape of CTA stays evenly placed (see
+  // make_plan1); on the Llama-3.1-8B layer chain this measured 24 % faster
+  // than giving the general kernel (whose CTAs share an SM) the matrices of up
+  // to 2^24 weights, and at n = 4 it takes 28 % less time than the general
+  // kernel.
   for (int b = 2; b <= 2 + np; ++b) {
     for (int nb = 1; nb <= STAGQ_MAX_BATCH; ++nb) h->plan1_ok[b][nb] = make_plan1(m, b, nb, &h->plan1[b][nb]);
     h->prefer1[b] = true;
