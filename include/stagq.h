@@ -283,6 +283,30 @@ int stagq_gemv_host(stagq_handle h, int bits, const void* x_host, int n, void* y
                     void* cuda_stream);
 
 /*
+ * Several GEMVs with HOST buffers and one synchronization: for i in
+ * [0, count), copies x_hosts[i] (host [ns[i]*in_i] fp16) to the device, then
+ * runs y_i = W_hat_i^(bits[i]) x_i with handle hs[i] (ns[i] = 1..4 vectors),
+ * then copies y_i back to y_hosts[i] (host [ns[i]*out_i] fp16). Every copy
+ * and launch goes on `cuda_stream` in that order: all x copies, all GEMVs (so
+ * consecutive launches overlap as in a device-side chain), all y copies. The
+ * call returns after the last copy of y has completed.
+ *   - Handles may repeat, and every handle must live on the same device.
+ *   - count is 1..STAGQ_MAX_MANY.
+ *   - Pinned host memory makes the copies asynchronous; pageable memory also
+ *     works.
+ *   - The device staging buffer is owned by the library, one per device. It
+ *     is allocated on first use and grown as needed. Calls on one device must
+ *     not overlap.
+ * Errors: STAGQ_EINVAL for a bad count, a null array or pointer, an n outside
+ * 1..STAGQ_MAX_BATCH, or handles on different devices; as stagq_gemv_ex for
+ * the GEMVs; STAGQ_ENOMEM if staging cannot be allocated. On an error no y_i
+ * is guaranteed to be written.
+ */
+#define STAGQ_MAX_MANY 1024
+int stagq_gemv_host_many(int count, const stagq_handle* hs, const int* bits, const void* const* x_hosts,
+                         const int* ns, void* const* y_hosts, void* cuda_stream);
+
+/*
  * As stagq_gemv_host, but allocates nothing: x and y are staged through a
  * statically reserved device array of STAGQ_NOALLOC_STAGE_BYTES (x in its
  * first 256 KiB, y in the rest), where stagq_gemv_host would cudaMalloc a

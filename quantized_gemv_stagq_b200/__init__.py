@@ -28,6 +28,7 @@ STAGQ_CODEBOOK_RULES = 0x100
 STAGQ_MAX_PLANES = 4
 STAGQ_MAX_BATCH = 4
 STAGQ_MAX_STACK = 4
+STAGQ_MAX_MANY = 1024
 
 _c_p = ctypes.c_void_p
 _i32, _i64, _u32, _dbl = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_double
@@ -74,6 +75,7 @@ _SIGNATURES = {
     "stagq_gemv_ex": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _u32, _c_p]),
     "stagq_gemv_scaled": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _c_p, _u32, _c_p]),
     "stagq_gemv_host": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _c_p]),
+    "stagq_gemv_host_many": (ctypes.c_int, [ctypes.c_int, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p]),
     "stagq_gemv_host_noalloc": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, ctypes.c_int, _c_p, _c_p]),
     "stagq_decode_levels": (ctypes.c_int, [_c_p, ctypes.c_int, _c_p, _c_p]),
     "stagq_bytes": (_i64, [_c_p, ctypes.c_int, ctypes.c_int]),
@@ -394,6 +396,24 @@ def stagq_gemv_host(m: Matrix, bits: int, x_host: np.ndarray, y_host: np.ndarray
     _check_host_array(y_host, "y_host", n * m.out)
     _check(lib().stagq_gemv_host(m.handle, bits, x_host.ctypes.data, n, y_host.ctypes.data,
                                  _stream_ptr(stream)), "stagq_gemv_host")
+
+
+def stagq_gemv_host_many(mats, bits, x_hosts, y_hosts, ns=None, stream=None) -> None:
+    """Several GEMVs with host buffers and one synchronization: every x copied
+    in, every GEMV run, every y copied out, in that order on one stream."""
+    count = len(mats)
+    ns = [1] * count if ns is None else list(ns)
+    if not (len(bits) == len(x_hosts) == len(y_hosts) == len(ns) == count):
+        raise ValueError("mats, bits, x_hosts, y_hosts and ns must have one entry per GEMV")
+    for m, x, y, n in zip(mats, x_hosts, y_hosts, ns):
+        _check_host_array(x, "x_host", n * m.inp)
+        _check_host_array(y, "y_host", n * m.out)
+    H = (ctypes.c_void_p * count)(*[m.handle.value for m in mats])
+    B = (ctypes.c_int * count)(*bits)
+    X = (ctypes.c_void_p * count)(*[x.ctypes.data for x in x_hosts])
+    N = (ctypes.c_int * count)(*ns)
+    Y = (ctypes.c_void_p * count)(*[y.ctypes.data for y in y_hosts])
+    _check(lib().stagq_gemv_host_many(count, H, B, X, N, Y, _stream_ptr(stream)), "stagq_gemv_host_many")
 
 
 def stagq_gemv_host_noalloc(m: Matrix, bits: int, x_host: np.ndarray, y_host: np.ndarray, n: int = 1,

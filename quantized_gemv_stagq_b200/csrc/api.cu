@@ -466,6 +466,78 @@ extern "C" int stagq_gemv_host(stagq_handle h, int bits, const void* x_host, int
   return STAGQ_OK;
 }
 
+namespace {
+// Device staging of stagq_gemv_host_many: one growing buffer per device.
+struct ManyStage {
+  std::mutex mu;
+  void* ptr[64] = {};
+  size_t bytes[64] = {};
+};
+ManyStage& many_stage() {
+  static ManyStage s;
+  return s;
+}
+}  // namespace
+
+extern "C" int stagq_gemv_host_many(int count, const stagq_handle* hs, const int* bits, const void* const* x_hosts,
+                                    const int* ns, void* const* y_hosts, void* cuda_stream) {
+  if (count < 1 || count > STAGQ_MAX_MANY) return fail(STAGQ_EINVAL, "count outside 1..STAGQ_MAX_MANY");
+  if (!hs || !bits || !x_hosts || !ns || !y_hosts) return fail(STAGQ_EINVAL, "null array");
+  size_t need = 0;
+  for (int i = 0; i < count; ++i) {
+    int st = check_handle_bits(hs[i], bits[i]);
+    if (st) return st;
+    if (!x_hosts[i] || !y_hosts[i]) return fail(STAGQ_EINVAL, "null x or y");
+    if (ns[i] < 1 || ns[i] > STAGQ_MAX_BATCH) return fail(STAGQ_EINVAL, "n outside 1..STAGQ_MAX_BATCH");
+    if (hs[i]->device != hs[0]->device) return fail(STAGQ_EINVAL, "handles on different devices");
+    need += align_up((size_t)ns[i] * hs[i]->dm.in * 2, 256) + align_up((size_t)ns[i] * hs[i]->dm.out * 2, 256);
+  }
+  const int dev = hs[0]->device;
+  if (dev < 0 || dev >= 64) return fail(STAGQ_EINVAL, "device index outside 0..63");
+  DeviceGuard guard(dev);
+  if (!guard.ok) return fail(STAGQ_ECUDA, "cudaSetDevice failed");
+  ManyStage& ms = many_stage();
+  std::lock_guard<std::mutex> lock(ms.mu);
+  if (ms.bytes[dev] < need) {
+    if (ms.ptr[dev]) cudaFree(ms.ptr[dev]);
+    ms.ptr[dev] = nullptr;
+    ms.bytes[dev] = 0;
+    cudaError_t e = cudaMalloc(&ms.ptr[dev], need);
+    if (e != cudaSuccess) { cudaGetLastError(); return fail(STAGQ_ENOMEM, "staging allocation failed"); }
+    ms.bytes[dev] = need;
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+  // x regions first, then y regions, each on 256 bytes
+  uint8_t* base = static_cast<uint8_t*>(ms.ptr[dev]);
+  size_t off = 0;
+  for (int i = 0; i < count; ++i) {
+    const size_t xb = (size_t)ns[i] * hs[i]->dm.in * 2;
+    cudaError_t e = cudaMemcpyAsync(base + off, x_hosts[i], xb, cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "copy of x");
+    off += align_up(xb, 256);
+  }
+  const size_t y0 = off;
+  off = 0;
+  size_t yoff = y0;
+  for (int i = 0; i < count; ++i) {
+    const size_t xb = (size_t)ns[i] * hs[i]->dm.in * 2, yb = (size_t)ns[i] * hs[i]->dm.out * 2;
+    int st = stagq_gemv_ex(hs[i], bits[i], base + off, ns[i], base + yoff, 0u, cuda_stream);
+    if (st) return st;
+    off += align_up(xb, 256);
+    yoff += align_up(yb, 256);
+  }
+  yoff = y0;
+  for (int i = 0; i < count; ++i) {
+    const size_t yb = (size_t)ns[i] * hs[i]->dm.out * 2;
+    cudaError_t e = cudaMemcpyAsync(y_hosts[i], base + yoff, yb, cudaMemcpyDeviceToHost, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "copy of y");
+    yoff += align_up(yb, 256);
+  }
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  return STAGQ_OK;
+}
+
 extern "C" int stagq_decode_levels(stagq_handle h, int bits, uint8_t* u_dev, void* cuda_stream) {
   int st = check_handle_bits(h, bits);
   if (st) return st;

@@ -463,6 +463,37 @@ def test_scaled_gemv_matches_oracle(case):
     m.free()
 
 
+def test_host_many_matches_single_host_calls():
+    """stagq_gemv_host_many runs several GEMVs with host buffers and one
+    synchronization; a repeated handle, three precisions and n = 1 and 4: each
+    y equals the single-call host GEMV bit for bit, and equals the oracle."""
+    Fa = O.encode(synth.weights(300, 1024, 51), 128, 2, 0.005, "fast")
+    Fb = O.encode(synth.weights(96, 2048, 52), 64, 4, 0.01, "fast")
+    ma, mb = _load(Fa), _load(Fb)
+    xa1 = np.ascontiguousarray(synth.activations(1, 1024, 60))
+    xb4 = np.ascontiguousarray(synth.activations(4, 2048, 61))
+    xa4 = np.ascontiguousarray(synth.activations(4, 1024, 62))
+    calls = [(ma, Fa, 2, xa1, 1), (mb, Fb, 5, xb4, 4), (ma, Fa, 4, xa4, 4), (ma, Fa, 3, xa1, 1)]
+    ys = [np.zeros((n, m.out), np.float16) for m, _, _, _, n in calls]
+    Q.stagq_gemv_host_many([c[0] for c in calls], [c[2] for c in calls], [c[3] for c in calls], ys,
+                           ns=[c[4] for c in calls])
+    for (m, F, b, x, n), y in zip(calls, ys):
+        one = np.zeros((n, m.out), np.float16)
+        Q.stagq_gemv_host(m, b, x, one, n=n)
+        assert np.array_equal(y, one), f"p{b} n{n}"
+        ref = O.gemv(F, b, x)
+        for j in range(n):
+            check_close(y[j].astype(np.float64), ref[j], f"p{b} n{n} col{j}")
+    with pytest.raises(Q.StagqError):  # no GEMV
+        Q.stagq_gemv_host_many([], [], [], [])
+    with pytest.raises(Q.StagqError):  # bits outside the stream
+        Q.stagq_gemv_host_many([ma], [7], [xa1], [ys[0]])
+    with pytest.raises(Q.StagqError):  # n outside 1..4
+        Q.stagq_gemv_host_many([ma], [2], [np.zeros((5, 1024), np.float16)], [np.zeros((5, 300), np.float16)], ns=[5])
+    ma.free()
+    mb.free()
+
+
 def test_scaled_product_that_rounds_to_the_int16_limit():
     """x = 1 and s = 1 - 2^-17: every scaled product is 32767.75 after the
     chunk's power-of-two scale, which rounds to 2^15; the fixed-point value
