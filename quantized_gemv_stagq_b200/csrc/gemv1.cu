@@ -843,9 +843,13 @@ int gemv1_grid(int out, int num_sms) {
 //  * About 60 KB of weights in flight per SM hide the HBM latency: the ring
 //    grows to that from 3 slots where the shared memory allows.
 //  * Larger blocks (UP = 4) amortise the per-block waits and sums, as long as
-//    the CTA's rows still make about 5 blocks to pipeline.
+//    the CTA's rows still make about 5 blocks to pipeline; with fewer rows, 2
+//    rows per warp while that makes at least 3 blocks (measured on q/k/v
+//    stacked, 41 rows per CTA: 2 rows in 3 blocks beat 4 rows in 2 by up to
+//    0.8 us), else 4.
 constexpr uint32_t kInflightTarget = 60u * 1024u;
-constexpr int kMinBlocks = 5;
+constexpr int kMinBlocks = 5;   // 4 rows per warp per block from this many blocks up
+constexpr int kMinBlocks2 = 3;  // below it, 2 rows from this many blocks up (else 4, fewer blocks)
 
 // The ring for given row groups: false if nothing fits the shared memory.
 bool plan1_fit(const DeviceMatrix& m, int bits, const Gemv1Plan& q, Gemv1Plan* out) {
@@ -854,7 +858,7 @@ bool plan1_fit(const DeviceMatrix& m, int bits, const Gemv1Plan& q, Gemv1Plan* o
   const int nblk2 = (q.rows_cap + 2 * q.RG - 1) / (2 * q.RG);
   // groups below 64 weights (several pairs per chunk): at most 2 rows per warp per block;
   // several vectors: 2 rows (1 with more than two planes), for the registers
-  int up0 = q.group_shift < 6 ? 2 : (nblk4 >= kMinBlocks || nblk2 < kMinBlocks) ? 4 : 2;
+  int up0 = q.group_shift < 6 ? 2 : (nblk4 >= kMinBlocks || nblk2 < kMinBlocks2) ? 4 : 2;
   if (q.nb > 1) up0 = bits > 4 ? 1 : 2;
   for (int stage = 1; stage >= 0; --stage) {   // side record staged in shared memory where it fits
     for (int up = up0; up >= 1; up /= 2) {
