@@ -318,6 +318,15 @@ def test_binding_refuses_tensors_that_do_not_fit_the_call():
         Q.stagq_gemv_host(m, 2, np.zeros((1, 512), np.float16), np.zeros((1, 32), np.float16))
     with pytest.raises(TypeError, match="x_host"):
         Q.stagq_gemv_host_noalloc(m, 2, np.zeros((1, 512), np.float32), np.zeros((1, 64), np.float16))
+    # several GEMVs with host buffers: one entry per GEMV in every list, each
+    # buffer checked against its own handle and n
+    xh, yh = np.zeros((1, 512), np.float16), np.zeros((1, 64), np.float16)
+    with pytest.raises(ValueError, match="one entry per GEMV"):
+        Q.stagq_gemv_host_many([m, m], [2], [xh, xh], [yh, yh])
+    with pytest.raises(ValueError, match="y_host holds 64 elements; the call needs 256"):
+        Q.stagq_gemv_host_many([m, m], [2, 3], [xh, np.zeros((4, 512), np.float16)], [yh, yh], ns=[1, 4])
+    with pytest.raises(TypeError, match="x_host"):
+        Q.stagq_gemv_host_many([m], [2], [xh.astype(np.float32)], [yh])
 
 
 def test_stacked_load_checks_its_members():
