@@ -353,3 +353,19 @@ def test_stacked_load_checks_its_members():
     with pytest.raises(Q.StagqError) as e:              # a malformed member
         Q.stagq_load_stack([a, bad], 0)
     assert e.value.status == 2
+
+
+def test_host_many_refuses_bad_arguments_before_any_device_work():
+    """stagq_gemv_host_many checks its count and arrays through the C ABI
+    before it touches a device, so this runs without a GPU (status 1 =
+    STAGQ_EINVAL)."""
+    import ctypes
+    L = Q.lib()
+    one = (ctypes.c_void_p * 1)(None)
+    bits = (ctypes.c_int * 1)(2)
+    ns = (ctypes.c_int * 1)(1)
+    assert L.stagq_gemv_host_many(0, one, bits, one, ns, one, None) == 1
+    assert L.stagq_gemv_host_many(Q.STAGQ_MAX_MANY + 1, one, bits, one, ns, one, None) == 1
+    assert L.stagq_gemv_host_many(1, None, bits, one, ns, one, None) == 1
+    assert L.stagq_gemv_host_many(1, one, None, one, ns, one, None) == 1
+    assert L.stagq_gemv_host_many(1, one, bits, one, ns, one, None) == 1  # null handle
